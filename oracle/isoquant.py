@@ -1,0 +1,557 @@
+"""Float64 CPU oracle of IsoQuant KV compression and compressed-space decode attention.
+
+TEST INFRASTRUCTURE ONLY.  The test suite, the package smoke check and the
+benchmark's CPU-baseline / reference leg are the only code allowed to import
+this module.  The product (the CUDA library behind ``include/isoq.h`` and its
+Python binding) never imports, links or calls it, and this module imports
+nothing from the product.  It is deliberately plain and slow: every step is
+written out in float64 in the order the sources give it, vectorised only across
+independent vectors, with no blocking, fusion or reordering of one vector's
+arithmetic.
+
+Sources, cited by page title and section:
+
+  [RQ]  "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via Fused
+        Compressed-Space Attention" (arXiv 2608.08081):
+        §3.2 Algorithm 1 and Steps 1-4, eq. (2), "Rotation cost analysis";
+        §3.3 eq. (5); §3.4 Table 2 (kernels A-D); Appendix A (inner-product
+        preservation, compressed-space attention); Appendix B (SO(4)
+        quaternion parameterisation).
+  [IQ]  "IsoQuant: Hardware-Aligned SO(4) Isoclinic Rotations for LLM KV Cache
+        Compression" (arXiv 2603.28430), abstract: T(v) = q_L v conj(q_R),
+        IsoQuant-Full and IsoQuant-Fast, FMA counts 1,024 / 512 at d = 128.
+
+Readings taken where the pages are silent (each is listed with its reason in
+the repository's design notes):
+
+  * WHT: H_d is the +-1 Sylvester matrix in natural order,
+    H_ij = (-1)^popcount(i & j); the orthonormal transform is H_d / sqrt(d);
+    no random sign diagonal.  The rotation is R = R_SO4 o (H_d / sqrt(d)).
+  * A 4-block (x0, x1, x2, x3) is the quaternion x0 + x1 i + x2 j + x3 k,
+    real part first, Hamilton convention ij = k.
+  * Full: u = q_L (x) v (x) conj(q_R); Fast: u = q_L (x) v (left-isoclinic,
+    q_R stored as the identity (1, 0, 0, 0)).
+  * Parameters: per head d/4 blocks of 8 floats (q_L then q_R, each w,x,y,z),
+    Haar-random unit quaternions from SplitMix64 + Box-Muller (see
+    ``make_params``), rounded to float32.
+  * Codebook: Lloyd-Max for N(0, 1/d), 2^b levels, the same for K and V and
+    all heads; code = #{k : y > t_k} (ties go to the lower code).
+  * Bit-pack: LSB-first little-endian bitstream per vector, code i at bits
+    [b*i, b*i + b); vectors are contiguous with no padding.
+  * Scale: s = ||x||_2 is stored as float16 (round to nearest even); the
+    vector is normalised by the unrounded s; dequantisation multiplies by the
+    stored float16 s.  s = 0 gives x_hat = 0.
+  * Decode attention: q is not normalised; q~ = R_K q; scores use the
+    K-rotation of the query's KV head kvh = qh // G; the output is
+    o = R_V^T o~; softmax is the natural-exponent softmax with the maximum
+    subtracted; tokens j >= min(seq_len[b], Tmax) are masked; seq_len <= 0
+    gives a zero output row.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+FULL = 0
+FAST = 1
+
+_MASK64 = (1 << 64) - 1
+
+
+# ---------------------------------------------------------------------------
+# Parameter generator: SplitMix64 -> uniform (0, 1] -> Box-Muller -> Haar S^3
+# ---------------------------------------------------------------------------
+
+class SplitMix64:
+    """SplitMix64 generator (Steele, Lea & Flood, "Fast splittable
+    pseudorandom number generators", OOPSLA 2014).
+
+    The state is a 64-bit counter advanced by the odd constant
+    0x9E3779B97F4A7C15 each call; the output is the counter passed through
+    the published three-step xor-shift-multiply finaliser.
+    """
+
+    def __init__(self, seed: int):
+        self.state = int(seed) & _MASK64
+
+    def next_u64(self) -> int:
+        self.state = (self.state + 0x9E3779B97F4A7C15) & _MASK64
+        z = self.state
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _MASK64
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _MASK64
+        return z ^ (z >> 31)
+
+    def next_uniform(self) -> float:
+        """A uniform double in (0, 1]: the top 53 bits, plus one, times 2^-53."""
+        return float((self.next_u64() >> 11) + 1) * 2.0 ** -53
+
+
+def gaussian_stream(rng: SplitMix64):
+    """Standard normal draws by the Box-Muller transform (Box & Muller 1958).
+
+    Each pair of uniforms (u1, u2) yields r cos(2 pi u2) and then
+    r sin(2 pi u2), with r = sqrt(-2 ln u1), in that order.
+    """
+    while True:
+        u1 = rng.next_uniform()
+        u2 = rng.next_uniform()
+        r = math.sqrt(-2.0 * math.log(u1))
+        theta = 2.0 * math.pi * u2
+        yield r * math.cos(theta)
+        yield r * math.sin(theta)
+
+
+def _unit4(v):
+    n = math.sqrt(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3])
+    return [v[0] / n, v[1] / n, v[2] / n, v[3] / n]
+
+
+def make_params(d: int, variant: int, seed: int, n_heads: int = 1) -> np.ndarray:
+    """Per-head SO(4) block parameters, float32 [n_heads][d/4][8].
+
+    [RQ] Appendix B: each of the d/4 blocks stores a pair of unit quaternions
+    (q_L, q_R), 8 floats per block, 256 floats per head at d = 128.
+    [RQ] §3.2 calls them learnable while its checklist says no training is
+    done; this oracle draws them at random.  A normalised N(0, I_4) draw is
+    uniform (Haar) on S^3.  Draw order: heads, then blocks, then q_L (4
+    normals), then q_R (4 normals).  IsoQuant-Fast ([IQ]) keeps only q_L: its
+    q_L equals Full's for the same seed (q_R's draws are still consumed) and
+    its q_R slot holds the identity (1, 0, 0, 0).
+    """
+    if d % 4:
+        raise ValueError("d must be a multiple of 4")
+    g = gaussian_stream(SplitMix64(seed))
+    out = np.empty((n_heads, d // 4, 8), dtype=np.float32)
+    for h in range(n_heads):
+        for i in range(d // 4):
+            ql = _unit4([next(g) for _ in range(4)])
+            qr = _unit4([next(g) for _ in range(4)])
+            out[h, i, 0:4] = ql
+            out[h, i, 4:8] = qr if variant == FULL else [1.0, 0.0, 0.0, 0.0]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Lloyd-Max scalar quantiser for a Gaussian source
+# ---------------------------------------------------------------------------
+
+_SQRT2 = math.sqrt(2.0)
+_INV_SQRT_2PI = 1.0 / math.sqrt(2.0 * math.pi)
+
+
+def _phi(x: float) -> float:
+    """Standard normal density (0 at +-inf)."""
+    if math.isinf(x):
+        return 0.0
+    return _INV_SQRT_2PI * math.exp(-0.5 * x * x)
+
+
+def _cell_mass(a: float, b: float) -> float:
+    """P(a < X < b) for X ~ N(0, 1), using the tail form that keeps precision."""
+    if a >= 0.0:
+        # both edges in the upper tail: Q(a) - Q(b), Q(x) = erfc(x / sqrt 2) / 2
+        return 0.5 * (math.erfc(a / _SQRT2) - math.erfc(b / _SQRT2))
+    if b <= 0.0:
+        return 0.5 * (math.erfc(-b / _SQRT2) - math.erfc(-a / _SQRT2))
+    return 1.0 - 0.5 * math.erfc(b / _SQRT2) - 0.5 * math.erfc(-a / _SQRT2)
+
+
+def _normal_quantile(p: float) -> float:
+    """Inverse of the standard normal CDF by bisection (initialisation only)."""
+    lo, hi = -40.0, 40.0
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        if 0.5 * math.erfc(-mid / _SQRT2) < p:
+            lo = mid
+        else:
+            hi = mid
+    return 0.5 * (lo + hi)
+
+
+def lloyd_max_gaussian(bits: int, sigma: float = 1.0, tol: float = 2e-15,
+                       max_iter: int = 100000):
+    """Lloyd-Max quantiser for N(0, sigma^2) with 2^bits levels.
+
+    [RQ] §3.2 Step 3: each rotated coordinate is quantised with a Lloyd-Max
+    optimal codebook (Lloyd 1982; Max 1960).  Lloyd's iteration alternates the
+    two optimality conditions: thresholds at the midpoints of adjacent
+    centroids, and each centroid the conditional mean of its cell,
+    E[X | a < X < b] = (phi(a) - phi(b)) / (Phi(b) - Phi(a)) in sigma units.
+    It starts from the Gaussian quantiles (k + 1/2) / L and stops when no
+    centroid moves by more than ``tol`` (sigma units).  The Gaussian density
+    is log-concave and even, so the fixed point is unique and odd-symmetric
+    (c_k = -c_{L-1-k}, middle threshold 0); each iterate is symmetrised,
+    (c_k - c_{L-1-k}) / 2, so that rounding cannot break that symmetry.
+
+    Returns (centroids[L], thresholds[L-1]) as float64, scaled by sigma.
+    """
+    levels = 1 << bits
+
+    def symmetrise(c):
+        return [0.5 * (c[k] - c[levels - 1 - k]) for k in range(levels)]
+
+    c = symmetrise([_normal_quantile((k + 0.5) / levels) for k in range(levels)])
+    for _ in range(max_iter):
+        t = [0.5 * (c[k] + c[k + 1]) for k in range(levels - 1)]
+        edges = [-math.inf] + t + [math.inf]
+        new_c = []
+        for k in range(levels):
+            a, b = edges[k], edges[k + 1]
+            new_c.append((_phi(a) - _phi(b)) / _cell_mass(a, b))
+        new_c = symmetrise(new_c)
+        delta = max(abs(x - y) for x, y in zip(new_c, c))
+        c = new_c
+        if delta <= tol:
+            break
+    t = [0.5 * (c[k] + c[k + 1]) for k in range(levels - 1)]
+    return np.array(c) * sigma, np.array(t) * sigma
+
+
+def make_codebook(d: int, bits: int):
+    """Codebook for the post-rotation marginal of a unit vector in R^d.
+
+    Reading of [RQ] §3.2 Step 3 ("post-rotation marginal"): after the WHT each
+    coordinate of a unit vector has variance 1/d ([RQ] §3.2, "Why structured
+    rotation works"); the codebook is Lloyd-Max for N(0, 1/d).
+    """
+    return lloyd_max_gaussian(bits, sigma=1.0 / math.sqrt(d))
+
+
+# ---------------------------------------------------------------------------
+# Walsh-Hadamard transform and quaternion block maps
+# ---------------------------------------------------------------------------
+
+def wht(x, counter=None):
+    """Unnormalised Walsh-Hadamard transform H_d x along the last axis.
+
+    [RQ] §3.2 Step 2 / eq. (2) and "Rotation cost analysis": the WHT is
+    applied by its butterfly, d log2 d operations.  Stage h (h = 1, 2, 4, ...,
+    d/2) replaces each pair (x_i, x_{i+h}), i with bit h clear, by
+    (x_i + x_{i+h}, x_i - x_{i+h}).  The product of the stages is the Sylvester
+    matrix in natural order.  ``counter`` (a one-element list) accumulates the
+    number of add/subtract operations.
+    """
+    y = np.array(x, dtype=np.float64, copy=True)
+    d = y.shape[-1]
+    if d & (d - 1):
+        raise ValueError("d must be a power of two")
+    h = 1
+    while h < d:
+        for start in range(0, d, 2 * h):
+            a = y[..., start:start + h].copy()
+            b = y[..., start + h:start + 2 * h].copy()
+            y[..., start:start + h] = a + b
+            y[..., start + h:start + 2 * h] = a - b
+            if counter is not None:
+                counter[0] += 2 * h
+        h *= 2
+    return y
+
+
+def hamilton(p, q, counter=None):
+    """Quaternion product p (x) q on arrays [..., 4] ordered (w, x, y, z).
+
+    Hamilton's rules i^2 = j^2 = k^2 = ijk = -1.  Each output component is a
+    sum of four products, so one product is 16 multiply-adds; ``counter`` (a
+    one-element list) accumulates that count per product and per vector.
+    """
+    p = np.asarray(p, dtype=np.float64)
+    q = np.asarray(q, dtype=np.float64)
+    pw, px, py, pz = p[..., 0], p[..., 1], p[..., 2], p[..., 3]
+    qw, qx, qy, qz = q[..., 0], q[..., 1], q[..., 2], q[..., 3]
+    out = np.empty(np.broadcast_shapes(p.shape, q.shape), dtype=np.float64)
+    out[..., 0] = pw * qw - px * qx - py * qy - pz * qz
+    out[..., 1] = pw * qx + px * qw + py * qz - pz * qy
+    out[..., 2] = pw * qy - px * qz + py * qw + pz * qx
+    out[..., 3] = pw * qz + px * qy - py * qx + pz * qw
+    if counter is not None:
+        counter[0] += 16 * int(np.prod(out.shape[:-1], dtype=np.int64))
+    return out
+
+
+def qconj(q):
+    """Quaternion conjugate (w, -x, -y, -z)."""
+    q = np.asarray(q, dtype=np.float64)
+    return q * np.array([1.0, -1.0, -1.0, -1.0])
+
+
+def so4_forward(v, ql, qr, variant, counter=None):
+    """[IQ] abstract / [RQ] Algorithm 1: T(v) = q_L v conj(q_R) per 4-block.
+
+    v: [..., nblk, 4]; ql, qr: [nblk, 4].  Full applies both products; Fast
+    keeps only the left isoclinic factor, T(v) = q_L v.
+    """
+    u = hamilton(ql, v, counter)
+    if variant == FULL:
+        u = hamilton(u, qconj(qr), counter)
+    return u
+
+
+def so4_inverse(u, ql, qr, variant):
+    """Inverse block map: conj(q_L) u q_R (Full) or conj(q_L) u (Fast).
+
+    [RQ] §3.4 / Table 2 kernel D: the inverse rotation uses the transposed
+    SO(4) blocks; for unit quaternions the transpose of v -> q_L v conj(q_R)
+    is u -> conj(q_L) u q_R.
+    """
+    v = hamilton(qconj(ql), u)
+    if variant == FULL:
+        v = hamilton(v, qr)
+    return v
+
+
+def rotate(xhat, params_head, variant):
+    """R x = R_SO4(H_d x / sqrt(d)) along the last axis ([RQ] eq. (2))."""
+    xhat = np.asarray(xhat, dtype=np.float64)
+    d = xhat.shape[-1]
+    p = np.asarray(params_head, dtype=np.float64).reshape(d // 4, 8)
+    z = wht(xhat) / math.sqrt(d)
+    blocks = z.reshape(z.shape[:-1] + (d // 4, 4))
+    return so4_forward(blocks, p[:, 0:4], p[:, 4:8], variant).reshape(xhat.shape)
+
+
+def rotate_inverse(y, params_head, variant):
+    """R^T y = H_d (R_SO4^T y) / sqrt(d) ([RQ] Appendix A: R^-1 = R^T)."""
+    y = np.asarray(y, dtype=np.float64)
+    d = y.shape[-1]
+    p = np.asarray(params_head, dtype=np.float64).reshape(d // 4, 8)
+    blocks = y.reshape(y.shape[:-1] + (d // 4, 4))
+    v = so4_inverse(blocks, p[:, 0:4], p[:, 4:8], variant).reshape(y.shape)
+    return wht(v) / math.sqrt(d)
+
+
+# ---------------------------------------------------------------------------
+# Scalar quantiser and bit-pack
+# ---------------------------------------------------------------------------
+
+def quantize_scalar(y, thresholds):
+    """Lloyd-Max code of each coordinate: #{k : y > t_k} ([RQ] Algorithm 1)."""
+    y = np.asarray(y, dtype=np.float64)
+    codes = np.zeros(y.shape, dtype=np.int64)
+    for t in thresholds:
+        codes += (y > t)
+    return codes
+
+
+def packed_bytes(d: int, bits: int) -> int:
+    """Bytes per packed vector, d * b / 8 ([RQ] §3.2 Step 4: 48 at d=128, b=3)."""
+    return d * bits // 8
+
+
+def bitpack(codes, bits: int):
+    """BitPack_b ([RQ] Algorithm 1): LSB-first bitstream, code i at bit b*i.
+
+    codes: integer array [..., d]; returns uint8 [..., d*b/8].  Written bit by
+    bit: bit k of code i goes to stream position b*i + k, which is bit
+    (b*i + k) % 8 of byte (b*i + k) // 8.
+    """
+    codes = np.asarray(codes, dtype=np.int64)
+    d = codes.shape[-1]
+    out = np.zeros(codes.shape[:-1] + (packed_bytes(d, bits),), dtype=np.int64)
+    for i in range(d):
+        for k in range(bits):
+            pos = bits * i + k
+            out[..., pos // 8] |= ((codes[..., i] >> k) & 1) << (pos % 8)
+    return out.astype(np.uint8)
+
+
+def bitunpack(packed, bits: int, d: int):
+    """Inverse of ``bitpack``: uint8 [..., d*b/8] -> int64 codes [..., d]."""
+    packed = np.asarray(packed, dtype=np.int64)
+    codes = np.zeros(packed.shape[:-1] + (d,), dtype=np.int64)
+    for i in range(d):
+        for k in range(bits):
+            pos = bits * i + k
+            codes[..., i] |= ((packed[..., pos // 8] >> (pos % 8)) & 1) << k
+    return codes
+
+
+# ---------------------------------------------------------------------------
+# Algorithm 1: quantise, and its inverse
+# ---------------------------------------------------------------------------
+
+def quantize(x, params, bits: int, variant: int, return_rotated: bool = False):
+    """IsoQuant compression of every vector ([RQ] §3.2, Algorithm 1).
+
+    x: [n_heads][n_vec][d] (any real dtype; its values are taken exactly);
+    params: [n_heads][d/4][8].  Per vector: s = ||x||_2 (Step 1);
+    x_hat = x / s (x_hat = 0 when s = 0); y = R_SO4(H_d x_hat / sqrt d)
+    (Step 2, eq. 2); code_i = #{k : y_i > t_k} (Step 3); BitPack_b (Step 4).
+    Returns (packed uint8 [n_heads][n_vec][d*b/8], norms float16
+    [n_heads][n_vec]) and, with ``return_rotated``, also y (float64), whose
+    distance to the nearest threshold tells how close each code is to a
+    decision boundary.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    n_heads, n_vec, d = x.shape
+    _, thresholds = make_codebook(d, bits)
+    packed = np.empty((n_heads, n_vec, packed_bytes(d, bits)), dtype=np.uint8)
+    norms = np.empty((n_heads, n_vec), dtype=np.float16)
+    ys = np.empty_like(x) if return_rotated else None
+    for h in range(n_heads):
+        s = np.sqrt(np.sum(x[h] * x[h], axis=-1))
+        safe = np.where(s > 0, s, 1.0)
+        xhat = np.where(s[:, None] > 0, x[h] / safe[:, None], 0.0)
+        y = rotate(xhat, params[h], variant)
+        packed[h] = bitpack(quantize_scalar(y, thresholds), bits)
+        norms[h] = s.astype(np.float16)
+        if return_rotated:
+            ys[h] = y
+    if return_rotated:
+        return packed, norms, ys
+    return packed, norms
+
+
+def dequantize(packed, norms, params, bits: int, variant: int, d: int):
+    """Reconstruction s16 * R^T c[codes] ([RQ] §3.4 kernel D, Appendix A).
+
+    packed: uint8 [n_heads][n_vec][d*b/8]; norms: float16 [n_heads][n_vec].
+    Returns float64 [n_heads][n_vec][d]: x = float(s16) * H_d(R_SO4^T c) / sqrt d.
+    """
+    centroids, _ = make_codebook(d, bits)
+    packed = np.asarray(packed)
+    n_heads, n_vec, _ = packed.shape
+    out = np.empty((n_heads, n_vec, d), dtype=np.float64)
+    for h in range(n_heads):
+        c = centroids[bitunpack(packed[h], bits, d)]
+        out[h] = rotate_inverse(c, params[h], variant) * \
+            np.asarray(norms[h], dtype=np.float64)[:, None]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Decode attention: compressed space (A) and reconstructed (B)
+# ---------------------------------------------------------------------------
+
+def _softmax_weights(z):
+    m = np.max(z)
+    p = np.exp(z - m)
+    return p / np.sum(p)
+
+
+def _valid_len(seq_len, tmax):
+    return int(min(max(int(seq_len), 0), tmax))
+
+
+def decode_attention(q, packed_k, packed_v, norms_k, norms_v, seq_lens,
+                     params_k, params_v, bits: int, variant: int, scale: float):
+    """Fused decode attention in the rotated domain ([RQ] Appendix A, §3.4).
+
+    q: [B][Hq][d]; packed_k/v: uint8 [B][Hkv][Tmax][d*b/8];
+    norms_k/v: float16 [B][Hkv][Tmax]; seq_lens: [B];
+    params_k/v: [Hkv][d/4][8].  For each (b, qh), kvh = qh // (Hq / Hkv),
+    T = min(seq_len[b], Tmax):
+      q~ = R_K q;   z_j = s^K_j <q~, c[codeK_j]> * scale;
+      alpha = softmax(z);   o~ = sum_j alpha_j s^V_j c[codeV_j];
+      o = R_V^T o~   (the inverse rotation is applied once, to the output).
+    Returns float64 [B][Hq][d]; rows with T = 0 are zero.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    bsz, hq, d = q.shape
+    hkv, tmax = packed_k.shape[1], packed_k.shape[2]
+    group = hq // hkv
+    centroids, _ = make_codebook(d, bits)
+    out = np.zeros((bsz, hq, d), dtype=np.float64)
+    for b in range(bsz):
+        t = _valid_len(seq_lens[b], tmax)
+        if t == 0:
+            continue
+        for kvh in range(hkv):
+            kt = centroids[bitunpack(packed_k[b, kvh, :t], bits, d)] * \
+                np.asarray(norms_k[b, kvh, :t], dtype=np.float64)[:, None]
+            vt = centroids[bitunpack(packed_v[b, kvh, :t], bits, d)] * \
+                np.asarray(norms_v[b, kvh, :t], dtype=np.float64)[:, None]
+            for g in range(group):
+                qh = kvh * group + g
+                q_rot = rotate(q[b, qh], params_k[kvh], variant)
+                alpha = _softmax_weights((kt @ q_rot) * scale)
+                out[b, qh] = rotate_inverse(alpha @ vt, params_v[kvh], variant)
+    return out
+
+
+def decode_attention_reconstructed(q, packed_k, packed_v, norms_k, norms_v,
+                                   seq_lens, params_k, params_v, bits: int,
+                                   variant: int, scale: float):
+    """Ordinary attention over the dequantised K and V ([RQ] Figure 1, top).
+
+    K_hat_j = dequantize(codeK_j, s^K_j), V_hat_j likewise;
+    o = sum_j softmax(<q, K_hat_j> * scale)_j V_hat_j.  By orthogonality of R
+    ([RQ] Appendix A) this equals ``decode_attention`` up to rounding.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    bsz, hq, d = q.shape
+    hkv, tmax = packed_k.shape[1], packed_k.shape[2]
+    group = hq // hkv
+    out = np.zeros((bsz, hq, d), dtype=np.float64)
+    for b in range(bsz):
+        t = _valid_len(seq_lens[b], tmax)
+        if t == 0:
+            continue
+        for kvh in range(hkv):
+            k_hat = dequantize(packed_k[b, kvh:kvh + 1, :t], norms_k[b, kvh:kvh + 1, :t],
+                               params_k[kvh:kvh + 1], bits, variant, d)[0]
+            v_hat = dequantize(packed_v[b, kvh:kvh + 1, :t], norms_v[b, kvh:kvh + 1, :t],
+                               params_v[kvh:kvh + 1], bits, variant, d)[0]
+            for g in range(group):
+                qh = kvh * group + g
+                alpha = _softmax_weights((k_hat @ q[b, qh]) * scale)
+                out[b, qh] = alpha @ v_hat
+    return out
+
+
+def split_partials(z, values, bounds):
+    """Split-K partial states of softmax attention for one query row.
+
+    z: scores [T]; values: [T][d]; bounds: increasing token offsets
+    [0, t1, ..., T].  For each split k over [bounds[k], bounds[k+1]):
+    m_k = max z, l_k = sum exp(z - m_k), acc_k = sum exp(z - m_k) v.
+    Empty splits give (m = -inf, l = 0, acc = 0).
+    """
+    parts = []
+    for k in range(len(bounds) - 1):
+        lo, hi = bounds[k], bounds[k + 1]
+        if hi <= lo:
+            parts.append((-math.inf, 0.0, np.zeros(values.shape[1])))
+            continue
+        m = float(np.max(z[lo:hi]))
+        p = np.exp(z[lo:hi] - m)
+        parts.append((m, float(np.sum(p)), p @ values[lo:hi]))
+    return parts
+
+
+def combine_partials(parts):
+    """Merge split-K partials: m* = max m_k, l = sum l_k e^(m_k - m*),
+    o = sum acc_k e^(m_k - m*) / l (the flash-decode combine; [RQ] §2
+    "Efficient attention" names FlashAttention as the analogue)."""
+    m_star = max(m for m, _, _ in parts)
+    l_tot = 0.0
+    acc = np.zeros_like(parts[0][2])
+    for m, l_k, a in parts:
+        if l_k == 0.0:
+            continue
+        w = math.exp(m - m_star)
+        l_tot += l_k * w
+        acc = acc + a * w
+    return acc / l_tot
+
+
+# ---------------------------------------------------------------------------
+# Operation counts the pages quote
+# ---------------------------------------------------------------------------
+
+def wht_op_count(d: int) -> int:
+    """Add/subtract operations of one butterfly WHT, counted by running it."""
+    counter = [0]
+    wht(np.zeros((d,)), counter)
+    return counter[0]
+
+
+def so4_fma_count(d: int, variant: int) -> int:
+    """Multiply-adds of the block rotation of one vector, counted by running it."""
+    counter = [0]
+    blocks = np.zeros((d // 4, 4))
+    q = np.tile(np.array([1.0, 0.0, 0.0, 0.0]), (d // 4, 1))
+    so4_forward(blocks, q, q, variant, counter)
+    return counter[0]
