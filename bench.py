@@ -1,0 +1,494 @@
+#!/usr/bin/env python
+"""Benchmark of the IsoQuant hot path on B200: packed 3-bit decode attention
+KV GB/s (fraction of HBM peak) and quantize Mvec/s.
+
+One step is one pass of the whole path over one batch of synthetic input:
+  1. stage-1 round trip: isoq_quantize then isoq_dequantize of 2^20 float16
+     unit vectors, d=128, 3-bit, IsoQuant-Full;
+  2. long-context decode: isoq_decode_split + isoq_decode_combine for batch 32
+     x 65,536 tokens, 16 query / 8 KV heads, d=256, 3-bit Full, over a packed
+     cache compressed from Student-t (nu=4) K/V with outlier channels and RoPE.
+The headline ``value`` is the decode's packed K/V bytes (codes + float16
+norms) divided by the decode's device time (split + combine, CUDA events on
+the launching stream, max over ranks).  Each step streams 3.3 GB of packed
+K/V, more than 26x the 126 MB L2, so no step finds its inputs in L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl isoq|reference]
+
+Multi-GPU runs are weak-scaled replicas: every rank runs the same per-GPU
+workload on its own data; there is no data-path collective (the (b, kvh)
+pairs are independent).  ``--impl reference`` times the float64 oracle on the
+host cores on a bounded sample of the same decode workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "packed-3-bit decode attn KV GB/s (% of HBM peak); quantize Mvec/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["compressed_space_attention_b200/csrc/isoq_decode.cu",
+                  "compressed_space_attention_b200/csrc/decode_mma.cuh",
+                  "compressed_space_attention_b200/csrc/common.cuh"]
+TRAFFIC_PROFILE = "profiles/decode_split_b32_gqa16_8_d256_t65536.md"
+
+WORKLOADS = {
+    # name: (B, Hq, Hkv, T, d)
+    "long_context_decode_b32_gqa16_8_d256_t65536": (32, 16, 8, 65536, 256),
+    "decode_b1_gqa32_4_d128_t32768": (1, 32, 4, 32768, 128),
+    "decode_b16_gqa32_4_d128_t8192_ragged": (16, 32, 4, 8192, 128),
+}
+DEFAULT_WORKLOAD = "long_context_decode_b32_gqa16_8_d256_t65536"
+STAGE1 = dict(n=1 << 20, d=128, bits=3)
+
+
+def env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def kv_bytes_per_token_head(d, bits=3):
+    return 2 * (d * bits // 8 + 2)
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic():
+    """Per-launch DRAM bytes of the decode split kernel from the committed ncu
+    summary, if that summary was taken on the current kernel source."""
+    path = os.path.join(ROOT, TRAFFIC_PROFILE)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    m_val = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_val or m_hash.group(1) != source_hash():
+        return None
+    return float(m_val.group(1))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling (NVML) during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons of one GPU from a host thread."""
+
+    REASONS = {
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, torch_device_index):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            handle = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    handle = h
+            if handle is None and pynvml.nvmlDeviceGetCount() == 1:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.handle = handle
+            self.nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = handle is not None
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the float64 oracle on a bounded sample of the decode workload
+# ---------------------------------------------------------------------------
+
+def oracle_decode_sample(workload, budget_s=20.0, min_s=8.0, tokens=None, seed=1000):
+    """Times the oracle's decode attention on one (b, kvh) pair of the
+    workload (its G query heads), token count chosen to take ~min_s..budget_s.
+    Returns (GB/s, seconds, description)."""
+    from threadpoolctl import threadpool_limits
+
+    import oracle as O
+    import synth
+
+    B, Hq, Hkv, T, d = WORKLOADS[workload]
+    g = Hq // Hkv
+    t = tokens or T
+    k, v = synth.student_t_kv(1, t, d, seed=seed)
+    prk = O.make_params(d, O.FULL, seed=1)
+    prv = O.make_params(d, O.FULL, seed=2)
+    pk, nk = O.quantize(k[0].astype(np.float64), prk, 3, O.FULL)
+    pv, nv = O.quantize(v[0].astype(np.float64), prv, 3, O.FULL)
+    q = synth.queries(1, g, d, seed=seed + 1)
+    args = (q, pk[None], pv[None], nk[None], nv[None], [t], prk, prv, 3, O.FULL, 1 / math.sqrt(d))
+    reps, elapsed = 0, 0.0
+    with threadpool_limits(limits=1):
+        while elapsed < min_s and elapsed < budget_s:
+            t0 = time.perf_counter()
+            O.decode_attention(*args)
+            elapsed += time.perf_counter() - t0
+            reps += 1
+    nbytes = reps * t * kv_bytes_per_token_head(d)
+    desc = (f"oracle decode of 1 of {B * Hkv} (b, kvh) pairs ({g} query heads, {t} tokens, d={d}), "
+            f"{reps} repetitions, float64 NumPy, BLAS threads 1")
+    return nbytes / elapsed / 1e9, elapsed, desc
+
+
+def oracle_quantize_rate(n=4096, seed=77):
+    from threadpoolctl import threadpool_limits
+
+    import oracle as O
+    import synth
+
+    x = synth.unit_vectors(n, STAGE1["d"], seed=seed, dtype=np.float16).astype(np.float64)
+    p = O.make_params(STAGE1["d"], O.FULL, seed=1)
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        O.quantize(x, p, STAGE1["bits"], O.FULL)
+        dt = time.perf_counter() - t0
+    return n / dt / 1e6
+
+
+# ---------------------------------------------------------------------------
+# Reference arm
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = env_int("RANK", 0)
+    if rank != 0:
+        return 0
+    workload = args.workload
+    B, Hq, Hkv, T, d = WORKLOADS[workload]
+    # Size each step so that warm-up + timed steps take about two minutes.
+    rate_gbs, secs, _ = oracle_decode_sample(workload, budget_s=5, min_s=0.5, tokens=4096)
+    tok_per_s = rate_gbs * 1e9 / kv_bytes_per_token_head(d)
+    per_step_s = 120.0 / max(1, args.steps + args.warmup)
+    t_step = int(min(T, max(1024, tok_per_s * per_step_s)) // 1024 * 1024)
+
+    import oracle as O
+    import synth
+    from threadpoolctl import threadpool_limits
+
+    g = Hq // Hkv
+    k, v = synth.student_t_kv(1, t_step, d, seed=2000)
+    prk = O.make_params(d, O.FULL, seed=1)
+    prv = O.make_params(d, O.FULL, seed=2)
+    pk, nk = O.quantize(k[0].astype(np.float64), prk, 3, O.FULL)
+    pv, nv = O.quantize(v[0].astype(np.float64), prv, 3, O.FULL)
+    q = synth.queries(1, g, d, seed=2001)
+    call = (q, pk[None], pv[None], nk[None], nv[None], [t_step], prk, prv, 3, O.FULL, 1 / math.sqrt(d))
+    with threadpool_limits(limits=1):
+        for _ in range(args.warmup):
+            O.decode_attention(*call)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            O.decode_attention(*call)
+        elapsed = time.perf_counter() - t0
+    nbytes = args.steps * t_step * kv_bytes_per_token_head(d)
+    value = nbytes / elapsed / 1e9
+    sample = (f"per step: oracle decode of 1 of {B * Hkv} (b, kvh) pairs, {g} query heads, "
+              f"{t_step} of {T} tokens, d={d}, float64 NumPy, BLAS threads 1")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(workload, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(workload, n_gpus):
+    B, Hq, Hkv, T, d = WORKLOADS[workload]
+    return {
+        "workload": workload + "+stage1_quantize_dequantize_d128_b3_f16_n1048576",
+        "batch": B, "context": T, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d, "bits": 3,
+        "variant": "IsoQuant-Full", "stage1_vectors": STAGE1["n"],
+        "l2": "inputs larger than L2: each step streams the whole packed K/V cache (no explicit flush)",
+        "parallelism": f"replicas x{n_gpus} (weak; no data-path collective)",
+    }
+
+
+# ---------------------------------------------------------------------------
+# CUDA arm
+# ---------------------------------------------------------------------------
+
+def run_isoq(args):
+    import torch
+
+    import compressed_space_attention_b200 as isoq
+    import synth
+
+    world = env_int("WORLD_SIZE", 1)
+    rank = env_int("RANK", 0)
+    local_rank = env_int("LOCAL_RANK", 0)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+
+    B, Hq, Hkv, T, d = WORKLOADS[args.workload]
+    bits, variant = 3, isoq.ISOQ_FULL
+    pb = d * bits // 8
+    seed0 = 1000 * rank
+
+    # ---- decode inputs: compress Student-t K/V into the packed cache ----
+    prk = torch.from_numpy(np.tile(isoq.isoq_make_params(d, variant, 1, Hkv), (1, 1, 1))).to(dev)
+    prv = torch.from_numpy(isoq.isoq_make_params(d, variant, 2, Hkv)).to(dev)
+    pk = torch.empty((B, Hkv, T, pb), dtype=torch.uint8, device=dev)
+    pv = torch.empty_like(pk)
+    nk = torch.empty((B, Hkv, T), dtype=torch.float16, device=dev)
+    nv = torch.empty_like(nk)
+    bchunk = max(1, min(B, (1 << 28) // (Hkv * T * d)))  # bound the float16 staging size
+    for b0 in range(0, B, bchunk):
+        b1 = min(B, b0 + bchunk)
+        k, v = synth.student_t_kv_torch(b1 - b0, Hkv, T, d, seed=seed0 + b0, device=dev)
+        prk_t = prk.repeat(b1 - b0, 1, 1)
+        prv_t = prv.repeat(b1 - b0, 1, 1)
+        isoq.isoq_quantize(k.view(-1, T, d), prk_t, bits, variant,
+                           codes=pk[b0:b1].view(-1, T, pb), norms=nk[b0:b1].view(-1, T))
+        isoq.isoq_quantize(v.view(-1, T, d), prv_t, bits, variant,
+                           codes=pv[b0:b1].view(-1, T, pb), norms=nv[b0:b1].view(-1, T))
+        del k, v
+    q = synth.queries_torch(B, Hq, d, seed=seed0 + 7, device=dev)
+    if "ragged" in args.workload:
+        lens_np = synth.ragged_lengths(B, T // 2, T, seed=0)
+    else:
+        lens_np = np.full(B, T, dtype=np.int32)
+    lens = torch.from_numpy(lens_np).to(dev)
+    out = torch.empty((B, Hq, d), dtype=torch.float16, device=dev)
+    ws = torch.empty(isoq.isoq_decode_workspace_size(B, Hq, Hkv, T, d), dtype=torch.uint8, device=dev)
+    kv_bytes = int(lens_np.clip(0, T).sum()) * Hkv * kv_bytes_per_token_head(d, bits)
+    torch.cuda.synchronize()
+
+    # ---- stage-1 inputs ----
+    n1, d1 = STAGE1["n"], STAGE1["d"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed0 + 11)
+    x1 = torch.randn((1, n1, d1), generator=gen, device=dev)
+    x1 = (x1 / x1.norm(dim=-1, keepdim=True)).half()
+    p1 = torch.from_numpy(isoq.isoq_make_params(d1, variant, 1, 1)).to(dev)
+    c1 = torch.empty((1, n1, d1 * bits // 8), dtype=torch.uint8, device=dev)
+    s1 = torch.empty((1, n1), dtype=torch.float16, device=dev)
+    r1 = torch.empty((1, n1, d1), dtype=torch.float16, device=dev)
+    q_bytes = n1 * (d1 * 2 + d1 * bits // 8 + 2)
+    dq_bytes = n1 * (d1 * bits // 8 + 2 + d1 * 2)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        isoq.isoq_quantize(x1, p1, bits, variant, codes=c1, norms=s1)
+        if ev:
+            ev[1].record(stream)
+        isoq.isoq_dequantize(c1, s1, p1, d1, bits, variant, out=r1)
+        if ev:
+            ev[2].record(stream)
+        isoq.isoq_decode_split(q, pk, pv, nk, nv, lens, prk, bits, variant, ws)
+        if ev:
+            ev[3].record(stream)
+        isoq.isoq_decode_combine(out, lens, B, Hq, Hkv, T, d, variant, prv, ws)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert isoq.isoq_check_device_error() == 0
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        start.record(stream)
+        for i in range(args.steps):
+            step(events[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    t_quant = sum(e[0].elapsed_time(e[1]) for e in events)
+    t_deq = sum(e[1].elapsed_time(e[2]) for e in events)
+    t_split = sum(e[2].elapsed_time(e[3]) for e in events)
+    t_comb = sum(e[3].elapsed_time(e[4]) for e in events)
+    t_decode = t_split + t_comb
+    assert isoq.isoq_check_device_error() == 0
+
+    # ---- end to end through the API with host buffers (decode half) ----
+    e2e_steps = max(1, min(args.steps, 3))
+    host = [t.cpu().pin_memory() for t in (q, pk, pv, nk, nv, lens)]
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = out_host.numel() * out_host.element_size()
+    dev_bufs = [torch.empty_like(t, device=dev) for t in host]
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for hb, db in zip(host, dev_bufs):
+            db.copy_(hb, non_blocking=True)
+        isoq.isoq_decode_attention(dev_bufs[0], dev_bufs[1], dev_bufs[2], dev_bufs[3], dev_bufs[4],
+                                   dev_bufs[5], prk, prv, bits, variant, out=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        dist.barrier()
+
+    # ---- reduce over ranks: max time, summed bytes ----
+    vals = torch.tensor([total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms = vals.tolist()
+    n_ranks = world
+
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    value = n_ranks * kv_bytes * args.steps / (t_decode * 1e-3) / 1e9
+    split_avg_s = t_split / args.steps * 1e-3
+    achieved = kv_bytes / split_avg_s / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_ranks, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": workload_config(args.workload, n_ranks),
+        "frac_of_hbm_peak": value / n_ranks / hbm,
+        "roofline": {"bound": "hbm", "kernel": "split_mma_kernel<256,Full> (decode split)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": read_traffic(), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                     "algorithmic_bytes_per_launch": kv_bytes},
+        "quantize": {"value": n_ranks * n1 * args.steps / (t_quant * 1e-3) / 1e6, "unit": "Mvec/s",
+                     "gbps": q_bytes * args.steps / (t_quant * 1e-3) / 1e9,
+                     "frac": q_bytes * args.steps / (t_quant * 1e-3) / 1e9 / hbm,
+                     "workload": "2^20 float16 unit vectors, d=128, 3-bit, Full"},
+        "dequantize": {"value": n_ranks * n1 * args.steps / (t_deq * 1e-3) / 1e6, "unit": "Mvec/s",
+                       "gbps": dq_bytes * args.steps / (t_deq * 1e-3) / 1e9},
+        "step_ms": {"quantize": t_quant / args.steps, "dequantize": t_deq / args.steps,
+                    "decode_split": t_split / args.steps, "decode_combine": t_comb / args.steps},
+        "e2e": {"value": n_ranks * kv_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "path": "pinned host cache -> device copy -> isoq_decode_attention -> host copy of the output"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        gbs, secs, desc = oracle_decode_sample(args.workload)
+        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": desc, "seconds": secs,
+                                "quantize_mvec_s": oracle_quantize_rate()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["isoq", "reference"], default="isoq")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_isoq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,473 @@
+// Compressed-space split-K decode attention on sm_100a.
+//
+// RotaryQuant (arXiv 2608.08081) Figure 1 (bottom), §3.4 Table 2 kernels A-D,
+// eq. (5) and Appendix A: the query is rotated once (q~ = R_K q), scores and
+// the value sum are computed directly on the packed codes in the rotated
+// domain, and the inverse rotation R_V^T is applied once to the merged output.
+// K and V are never written out dequantised.
+//
+// Two launches:
+//   split:   grid (n_splits, Hkv, B).  Each CTA owns one token chunk of one
+//            (b, kvh) and all G = Hq/Hkv query heads sharing it; it writes one
+//            partial state (m, l, acc[d]) per query head into the workspace,
+//            acc in the rotated domain (online softmax, natural exponent).
+//   combine: grid (Hq, B).  Merges the partials (m* = max m_k,
+//            l = sum l_k e^(m_k - m*), o~ = sum acc_k e^(m_k - m*) / l), then
+//            applies R_V^T = H_d R_SO4^T / sqrt(d) and stores the output.
+//
+// This file holds the generic split kernel (CUDA-core FMAs; any dtype, d and
+// bits) and the combine kernel; decode_mma.cuh (included below) holds the
+// tensor-core split kernel used for float16 queries with 3-bit codes.
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "common.cuh"
+#include "decode.h"
+#include "internal.h"
+
+namespace isoq {
+namespace decode {
+
+using namespace isoq::dev;
+
+__device__ unsigned int g_decode_error = 0;
+
+// Forward rotation q~ = R q of one vector held in shared memory, by all
+// threads of the CTA: WHT butterflies (stride h = 1 ... d/2), 1/sqrt(d), then
+// the per-block quaternion map.
+template <int D, bool FULL>
+__device__ void rotate_forward_cta(float *v, const float *params_head) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+#pragma unroll 1
+  for (int h = 1; h < D; h <<= 1) {
+    for (int p = tid; p < D / 2; p += nt) {
+      const int i = (p / h) * 2 * h + (p % h);
+      const float a = v[i], b = v[i + h];
+      v[i] = a + b;
+      v[i + h] = a - b;
+    }
+    __syncthreads();
+  }
+  const float inv = rsqrtf(static_cast<float>(D));
+  for (int bi = tid; bi < D / 4; bi += nt) {
+    const Quat x{v[4 * bi] * inv, v[4 * bi + 1] * inv, v[4 * bi + 2] * inv, v[4 * bi + 3] * inv};
+    const Quat u = block_forward(load_quat(params_head + 8 * bi), load_quat(params_head + 8 * bi + 4), x, FULL);
+    v[4 * bi] = u.w;
+    v[4 * bi + 1] = u.x;
+    v[4 * bi + 2] = u.y;
+    v[4 * bi + 3] = u.z;
+  }
+  __syncthreads();
+}
+
+// Inverse rotation x = H_d R_SO4^T u / sqrt(d) of one vector in shared memory.
+template <int D, bool FULL>
+__device__ void rotate_inverse_cta(float *v, const float *params_head) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  for (int bi = tid; bi < D / 4; bi += nt) {
+    const Quat u{v[4 * bi], v[4 * bi + 1], v[4 * bi + 2], v[4 * bi + 3]};
+    const Quat x = block_inverse(load_quat(params_head + 8 * bi), load_quat(params_head + 8 * bi + 4), u, FULL);
+    v[4 * bi] = x.w;
+    v[4 * bi + 1] = x.x;
+    v[4 * bi + 2] = x.y;
+    v[4 * bi + 3] = x.z;
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int h = 1; h < D; h <<= 1) {
+    for (int p = tid; p < D / 2; p += nt) {
+      const int i = (p / h) * 2 * h + (p % h);
+      const float a = v[i], b = v[i + h];
+      v[i] = a + b;
+      v[i + h] = a - b;
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
+
+// Code of dimension i from a packed row read as 32-bit words.
+template <int BITS>
+__device__ __forceinline__ uint32_t code_at(const uint32_t *row, int i) {
+  const int bp = BITS * i;
+  const uint32_t lo = __ldg(row + (bp >> 5));
+  uint32_t c = lo >> (bp & 31);
+  if ((bp & 31) + BITS > 32) c |= __ldg(row + (bp >> 5) + 1) << (32 - (bp & 31));
+  return c & ((1u << BITS) - 1u);
+}
+
+// ---------------------------------------------------------------------------
+// Generic split kernel: each warp owns query heads g = warp, warp + 4, ...;
+// per 32-token group, lane j scores token j (QK over all d), then the warp
+// accumulates V dimension-parallel (lane owns dims lane + 32 k).
+// ---------------------------------------------------------------------------
+constexpr int kGenericThreads = 128;
+
+template <typename T, int D, int BITS, bool FULL>
+__global__ void __launch_bounds__(kGenericThreads) split_generic_kernel(const SplitArgs a) {
+  constexpr int PB = D * BITS / 8, WORDS = PB / 4, KD = D / 32;
+  __shared__ float cent[16];
+  extern __shared__ float qrot[];  // [G][D]
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.group;
+  if (tid < (1 << BITS)) cent[tid] = a.centroid[tid];
+
+  int tlen = a.seq_lens[b];
+  tlen = tlen < 0 ? 0 : (tlen > a.tmax ? static_cast<int>(a.tmax) : tlen);
+  const long long t0 = static_cast<long long>(split) * a.chunk;
+  long long t1 = t0 + a.chunk;
+  if (t1 > tlen) t1 = tlen;
+
+  // Rotate the G queries of this KV head with R_K.
+  for (int g = 0; g < G; ++g) {
+    const T *q = static_cast<const T *>(a.q) + (static_cast<long long>(b) * a.hq + kvh * G + g) * D;
+    for (int i = tid; i < D; i += kGenericThreads) qrot[g * D + i] = to_f32<T>(q[i]);
+  }
+  __syncthreads();
+  for (int g = 0; g < G; ++g) rotate_forward_cta<D, FULL>(qrot + g * D, a.params_k + static_cast<size_t>(kvh) * 2 * D);
+
+  const long long pair = static_cast<long long>(b) * a.hkv + kvh;
+  const uint8_t *kbase = a.packed_k + pair * a.tmax * PB;
+  const uint8_t *vbase = a.packed_v + pair * a.tmax * PB;
+  const uint16_t *nkbase = a.norms_k + pair * a.tmax;
+  const uint16_t *nvbase = a.norms_v + pair * a.tmax;
+
+  for (int g = warp; g < G; g += kGenericThreads / 32) {
+    const float *qg = qrot + g * D;
+    float m = -INFINITY, l = 0.f;
+    float acc[KD];
+#pragma unroll
+    for (int k = 0; k < KD; ++k) acc[k] = 0.f;
+
+    for (long long tg = t0; tg < t1; tg += 32) {
+      const long long tok = tg + lane;
+      const bool valid = tok < t1;
+      float z = -INFINITY, sv = 0.f;
+      if (valid) {
+        const uint32_t *row = reinterpret_cast<const uint32_t *>(kbase + tok * PB);
+        float dot = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < D; ++i) dot = fmaf(cent[code_at<BITS>(row, i)], qg[i], dot);
+        const float sk = __half2float(__ushort_as_half(nkbase[tok]));
+        z = dot * sk * a.scale;
+        sv = __half2float(__ushort_as_half(nvbase[tok]));
+      }
+      float zmax = z;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+      const float m_new = fmaxf(m, zmax);
+      const float alpha = (m == -INFINITY) ? 0.f : expf(m - m_new);
+      const float p = valid ? expf(z - m_new) : 0.f;
+      l = l * alpha + p;
+#pragma unroll
+      for (int k = 0; k < KD; ++k) acc[k] *= alpha;
+      m = m_new;
+      const float w = p * sv;
+      const int n = static_cast<int>(t1 - tg < 32 ? t1 - tg : 32);
+      for (int j = 0; j < n; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, j);
+        const uint32_t *row = reinterpret_cast<const uint32_t *>(vbase + (tg + j) * PB);
+#pragma unroll
+        for (int k = 0; k < KD; ++k) acc[k] = fmaf(wj, cent[code_at<BITS>(row, lane + 32 * k)], acc[k]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+
+    const long long slot = (static_cast<long long>(b) * a.hq + kvh * G + g) * a.n_splits + split;
+    float *acc_out = a.ws_acc + slot * D;
+#pragma unroll
+    for (int k = 0; k < KD; ++k) acc_out[lane + 32 * k] = acc[k];
+    if (lane == 0) a.ws_ml[slot] = make_float2(m, l);
+  }
+  (void)WORDS;
+}
+
+// ---------------------------------------------------------------------------
+// Combine + inverse rotation.
+// ---------------------------------------------------------------------------
+constexpr int kCombineThreads = 128;
+
+template <typename T, int D, bool FULL>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineArgs a) {
+  __shared__ float v[D];
+  __shared__ float red[kCombineThreads / 32];
+  __shared__ float s_mstar, s_l;
+  const int qh = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int kvh = qh / a.group;
+  const long long base = (static_cast<long long>(b) * a.hq + qh) * a.n_splits;
+
+  float mx = -INFINITY;
+  for (int s = tid; s < a.n_splits; s += kCombineThreads) mx = fmaxf(mx, a.ws_ml[base + s].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  if (tid == 0) {
+    float m = red[0];
+    for (int w = 1; w < kCombineThreads / 32; ++w) m = fmaxf(m, red[w]);
+    s_mstar = m;
+  }
+  __syncthreads();
+  const float mstar = s_mstar;
+  float lsum = 0.f;
+  for (int s = tid; s < a.n_splits; s += kCombineThreads) {
+    const float2 ml = a.ws_ml[base + s];
+    if (ml.y > 0.f) lsum += ml.y * expf(ml.x - mstar);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = lsum;
+  __syncthreads();
+  if (tid == 0) {
+    float l = 0.f;
+    for (int w = 0; w < kCombineThreads / 32; ++w) l += red[w];
+    s_l = l;
+  }
+  __syncthreads();
+  const float ltot = s_l;
+  const float inv_l = ltot > 0.f ? 1.f / ltot : 0.f;
+
+  for (int i = tid; i < D; i += kCombineThreads) {
+    float acc = 0.f;
+    for (int s = 0; s < a.n_splits; ++s) {
+      const float2 ml = a.ws_ml[base + s];
+      if (ml.y > 0.f) acc = fmaf(a.ws_acc[(base + s) * D + i], expf(ml.x - mstar), acc);
+    }
+    v[i] = acc * inv_l;
+  }
+  __syncthreads();
+  rotate_inverse_cta<D, FULL>(v, a.params_v + static_cast<size_t>(kvh) * 2 * D);
+  const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+  T *out = static_cast<T *>(a.out) + (static_cast<long long>(b) * a.hq + qh) * D;
+  for (int i = tid; i < D; i += kCombineThreads) out[i] = from_f32<T>(v[i] * inv_sqrt_d);
+}
+
+#include "decode_mma.cuh"
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+
+template <typename T, int D, int BITS, bool FULL>
+int launch_split_generic(const SplitArgs &a, cudaStream_t stream) {
+  auto kernel = split_generic_kernel<T, D, BITS, FULL>;
+  const size_t smem = static_cast<size_t>(a.group) * D * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode split: %s", cudaGetErrorString(e));
+  }
+  dim3 grid(a.n_splits, a.hkv, a.batch);
+  kernel<<<grid, kGenericThreads, smem, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
+  return ISOQ_OK;
+}
+
+template <typename T, int D, bool FULL>
+int launch_combine(const CombineArgs &a, cudaStream_t stream) {
+  dim3 grid(a.hq, a.batch);
+  combine_kernel<T, D, FULL><<<grid, kCombineThreads, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode combine launch: %s", cudaGetErrorString(e));
+  return ISOQ_OK;
+}
+
+int run_split_generic(int dtype, int d, int bits, int variant, const SplitArgs &a, cudaStream_t st) {
+#define ISOQ_GV(T, D, B) \
+  return variant == ISOQ_FULL ? launch_split_generic<T, D, B, true>(a, st) : launch_split_generic<T, D, B, false>(a, st)
+#define ISOQ_GB(T, D)              \
+  switch (bits) {                  \
+    case 2: ISOQ_GV(T, D, 2);      \
+    case 3: ISOQ_GV(T, D, 3);      \
+    default: ISOQ_GV(T, D, 4);     \
+  }
+#define ISOQ_GD(T)                 \
+  switch (d) {                     \
+    case 128: ISOQ_GB(T, 128);     \
+    case 256: ISOQ_GB(T, 256);     \
+    default: ISOQ_GB(T, 512);      \
+  }
+  if (dtype == ISOQ_F16) {
+    ISOQ_GD(__half);
+  } else {
+    ISOQ_GD(float);
+  }
+#undef ISOQ_GD
+#undef ISOQ_GB
+#undef ISOQ_GV
+}
+
+int run_combine(int dtype, int d, int variant, const CombineArgs &a, cudaStream_t st) {
+#define ISOQ_CV(T, D) \
+  return variant == ISOQ_FULL ? launch_combine<T, D, true>(a, st) : launch_combine<T, D, false>(a, st)
+#define ISOQ_CD(T)              \
+  switch (d) {                  \
+    case 128: ISOQ_CV(T, 128);  \
+    case 256: ISOQ_CV(T, 256);  \
+    default: ISOQ_CV(T, 512);   \
+  }
+  if (dtype == ISOQ_F16) {
+    ISOQ_CD(__half);
+  } else {
+    ISOQ_CD(float);
+  }
+#undef ISOQ_CD
+#undef ISOQ_CV
+}
+
+bool aligned(const void *p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int validate_common(int dtype, int B, int Hq, int Hkv, int64_t Tmax, int d, int variant,
+                    const void *ws, size_t ws_bytes) {
+  if (!supported_d(d)) return set_error(ISOQ_ERR_UNSUPPORTED, "d=%d not supported", d);
+  if (!supported_variant(variant)) return set_error(ISOQ_ERR_UNSUPPORTED, "variant=%d", variant);
+  if (!supported_dtype(dtype)) return set_error(ISOQ_ERR_UNSUPPORTED, "dtype=%d", dtype);
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tmax <= 0)
+    return set_error(ISOQ_ERR_INVALID_ARG, "B, Hq, Hkv and Tmax must be positive");
+  if (Hq % Hkv) return set_error(ISOQ_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+  if (Hq / Hkv > kMaxGroup) return set_error(ISOQ_ERR_UNSUPPORTED, "Hq/Hkv > %d", kMaxGroup);
+  if (Tmax >= (1ll << 31) || B > 65535 || Hkv > 65535 || Hq > (1 << 24))
+    return set_error(ISOQ_ERR_INVALID_ARG, "shape too large");
+  if (!ws) return set_error(ISOQ_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(ws, 256)) return set_error(ISOQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < isoq_decode_workspace_size(B, Hq, Hkv, Tmax, d))
+    return set_error(ISOQ_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes,
+                     isoq_decode_workspace_size(B, Hq, Hkv, Tmax, d));
+  return ISOQ_OK;
+}
+
+void workspace_views(void *ws, int B, int Hq, int n_splits, int d, float **acc, float2 **ml) {
+  *acc = static_cast<float *>(ws);
+  *ml = reinterpret_cast<float2 *>(static_cast<float *>(ws) + static_cast<size_t>(B) * Hq * n_splits * d);
+}
+
+}  // namespace decode
+}  // namespace isoq
+
+using namespace isoq;
+
+extern "C" {
+
+int isoq_decode_split(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
+                      const uint8_t *packed_v_dev, const uint16_t *norms_k_dev,
+                      const uint16_t *norms_v_dev, const int32_t *seq_lens_dev, int B, int Hq,
+                      int Hkv, int64_t Tmax, int d, int bits, int variant,
+                      const float *params_k_dev, float scale, void *workspace_dev,
+                      size_t workspace_bytes, isoq_stream_t stream) {
+  clear_error();
+  int st = decode::validate_common(dtype, B, Hq, Hkv, Tmax, d, variant, workspace_dev, workspace_bytes);
+  if (st) return st;
+  if (!supported_bits(bits)) return set_error(ISOQ_ERR_UNSUPPORTED, "bits=%d not supported", bits);
+  if (!q_dev || !packed_k_dev || !packed_v_dev || !norms_k_dev || !norms_v_dev || !seq_lens_dev || !params_k_dev)
+    return set_error(ISOQ_ERR_INVALID_ARG, "null pointer");
+  if (!decode::aligned(q_dev, 16) || !decode::aligned(packed_k_dev, 16) || !decode::aligned(packed_v_dev, 16) ||
+      !decode::aligned(params_k_dev, 16) || !decode::aligned(norms_k_dev, 2) || !decode::aligned(norms_v_dev, 2) ||
+      !decode::aligned(seq_lens_dev, 4))
+    return set_error(ISOQ_ERR_UNSUPPORTED, "misaligned pointer");
+  if (!std::isfinite(scale)) return set_error(ISOQ_ERR_INVALID_ARG, "scale is not finite");
+
+  decode::SplitArgs a;
+  a.q = q_dev;
+  a.packed_k = packed_k_dev;
+  a.packed_v = packed_v_dev;
+  a.norms_k = norms_k_dev;
+  a.norms_v = norms_v_dev;
+  a.seq_lens = seq_lens_dev;
+  a.params_k = params_k_dev;
+  a.batch = B;
+  a.hq = Hq;
+  a.hkv = Hkv;
+  a.group = Hq / Hkv;
+  a.tmax = Tmax;
+  a.chunk = decode_chunk_tokens(B, Hkv, Tmax, d);
+  a.n_splits = decode_num_splits(B, Hkv, Tmax, d);
+  a.scale = scale;
+  decode::workspace_views(workspace_dev, B, Hq, a.n_splits, d, &a.ws_acc, &a.ws_ml);
+  CodebookF32 cb;
+  codebook_f32(d, bits, &cb);
+  for (int j = 0; j < 16; ++j) a.centroid[j] = j < cb.levels ? cb.centroid[j] : 0.f;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (decode::mma_path_supported(dtype, d, bits, a)) return decode::run_split_mma(d, variant, a, s);
+  return decode::run_split_generic(dtype, d, bits, variant, a, s);
+}
+
+int isoq_decode_combine(int dtype, const int32_t *seq_lens_dev, int B, int Hq, int Hkv,
+                        int64_t Tmax, int d, int variant, const float *params_v_dev,
+                        void *out_dev, const void *workspace_dev, size_t workspace_bytes,
+                        isoq_stream_t stream) {
+  clear_error();
+  int st = decode::validate_common(dtype, B, Hq, Hkv, Tmax, d, variant, workspace_dev, workspace_bytes);
+  if (st) return st;
+  if (!params_v_dev || !out_dev || !seq_lens_dev) return set_error(ISOQ_ERR_INVALID_ARG, "null pointer");
+  if (!decode::aligned(params_v_dev, 16) || !decode::aligned(out_dev, 16))
+    return set_error(ISOQ_ERR_UNSUPPORTED, "misaligned pointer");
+  decode::CombineArgs a;
+  a.params_v = params_v_dev;
+  a.out = out_dev;
+  a.batch = B;
+  a.hq = Hq;
+  a.group = Hq / Hkv;
+  a.n_splits = decode_num_splits(B, Hkv, Tmax, d);
+  float *acc;
+  float2 *ml;
+  decode::workspace_views(const_cast<void *>(workspace_dev), B, Hq, a.n_splits, d, &acc, &ml);
+  a.ws_acc = acc;
+  a.ws_ml = ml;
+  return decode::run_combine(dtype, d, variant, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int isoq_decode_attention(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
+                          const uint8_t *packed_v_dev, const uint16_t *norms_k_dev,
+                          const uint16_t *norms_v_dev, const int32_t *seq_lens_dev, int B,
+                          int Hq, int Hkv, int64_t Tmax, int d, int bits, int variant,
+                          const float *params_k_dev, const float *params_v_dev, float scale,
+                          void *out_dev, void *workspace_dev, size_t workspace_bytes,
+                          isoq_stream_t stream) {
+  clear_error();
+  if (!params_v_dev || !out_dev) return set_error(ISOQ_ERR_INVALID_ARG, "null pointer");
+  if (!decode::aligned(params_v_dev, 16) || !decode::aligned(out_dev, 16))
+    return set_error(ISOQ_ERR_UNSUPPORTED, "misaligned pointer");
+  int st = isoq_decode_split(q_dev, dtype, packed_k_dev, packed_v_dev, norms_k_dev, norms_v_dev,
+                             seq_lens_dev, B, Hq, Hkv, Tmax, d, bits, variant, params_k_dev,
+                             scale, workspace_dev, workspace_bytes, stream);
+  if (st) return st;
+  return isoq_decode_combine(dtype, seq_lens_dev, B, Hq, Hkv, Tmax, d, variant, params_v_dev,
+                             out_dev, workspace_dev, workspace_bytes, stream);
+}
+
+__attribute__((visibility("hidden"))) int isoq_detail_take_decode_error(cudaStream_t stream, unsigned *out) {
+  unsigned zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, decode::g_decode_error, sizeof(unsigned), 0,
+                                            cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess && *out)
+    e = cudaMemcpyToSymbolAsync(decode::g_decode_error, &zero, sizeof(unsigned), 0,
+                                cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  return e == cudaSuccess ? ISOQ_OK : set_error(ISOQ_ERR_CUDA, "error word: %s", cudaGetErrorString(e));
+}
+
+}  // extern "C"

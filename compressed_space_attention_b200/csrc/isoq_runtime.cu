@@ -1,0 +1,22 @@
+// Device error word collection: each kernel translation unit owns one 32-bit
+// word per device that its bounded waits set when they give up.
+
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+extern "C" __attribute__((visibility("hidden"))) int isoq_detail_take_quant_error(cudaStream_t stream, unsigned *out);
+extern "C" __attribute__((visibility("hidden"))) int isoq_detail_take_decode_error(cudaStream_t stream, unsigned *out);
+
+extern "C" int isoq_check_device_error(isoq_stream_t stream) {
+  isoq::clear_error();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned q = 0, d = 0;
+  int st = isoq_detail_take_quant_error(s, &q);
+  if (st) return st;
+  st = isoq_detail_take_decode_error(s, &d);
+  if (st) return st;
+  if (q | d)
+    return isoq::set_error(ISOQ_ERR_TIMEOUT, "device wait timed out (quantize=%u, decode=%u)", q, d);
+  return ISOQ_OK;
+}

@@ -1,0 +1,137 @@
+"""The C-ABI library on the host: it loads, exports every entry point the
+header declares, and its host-only functions (parameter generator, codebook,
+split policy, argument validation) behave as specified.  No device work."""
+
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle as O
+from isoq_testlib import header_functions
+
+import compressed_space_attention_b200 as isoq
+from compressed_space_attention_b200 import binding
+
+
+def test_library_exports_every_header_function():
+    lib = isoq.lib()
+    declared = header_functions()
+    assert len(declared) >= 15
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in isoq.h but not exported"
+    bound = {n for n, _, _ in binding.SIGNATURES}
+    assert set(declared) == bound, "binding and header disagree"
+    assert isoq.isoq_abi_version() == 1
+
+
+def test_sizes():
+    assert isoq.isoq_params_size(128) == 256
+    assert isoq.isoq_params_size(256) == 512
+    assert isoq.isoq_params_size(100) < 0
+    assert isoq.isoq_packed_bytes(128, 3) == 48
+    assert isoq.isoq_packed_bytes(256, 3) == 96
+    assert isoq.isoq_packed_bytes(512, 4) == 256
+    assert isoq.isoq_packed_bytes(128, 5) == 0
+
+
+@pytest.mark.parametrize("variant", [isoq.ISOQ_FULL, isoq.ISOQ_FAST])
+@pytest.mark.parametrize("d", [128, 256, 512])
+def test_make_params_matches_oracle(variant, d):
+    got = isoq.isoq_make_params(d, variant, seed=1234, n_heads=3)
+    ref = O.make_params(d, variant, seed=1234, n_heads=3)
+    assert got.shape == ref.shape
+    # Same published generator on both sides; allow one float32 ulp for a
+    # last-bit difference in the host libm.
+    diff = np.abs(got.view(np.int32).astype(np.int64) - ref.view(np.int32).astype(np.int64))
+    assert diff.max() <= 1
+    assert (diff == 0).mean() > 0.99
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("d", [128, 256, 512])
+def test_make_codebook_matches_oracle(bits, d):
+    c, t = isoq.isoq_make_codebook(d, bits)
+    rc, rt = O.make_codebook(d, bits)
+    np.testing.assert_allclose(c, rc, rtol=0, atol=1e-14 / np.sqrt(d))
+    np.testing.assert_allclose(t, rt, rtol=0, atol=1e-14 / np.sqrt(d))
+    assert t[len(t) // 2] == 0.0
+    np.testing.assert_array_equal(c, -c[::-1])
+
+
+def test_split_policy_and_workspace():
+    for (B, hkv, tmax, d) in [(1, 4, 32768, 128), (16, 4, 8192, 128), (32, 8, 65536, 256),
+                              (1, 1, 4096, 128), (3, 2, 1, 512), (2, 2, 1001, 128)]:
+        n = isoq.isoq_decode_num_splits(B, hkv, tmax, d)
+        assert n >= 1
+        hq = 2 * hkv
+        ws = isoq.isoq_decode_workspace_size(B, hq, hkv, tmax, d)
+        assert ws >= B * hq * n * (d + 2) * 4 and ws % 256 == 0
+    assert isoq.isoq_decode_workspace_size(1, 3, 2, 100, 128) == 0  # Hq % Hkv != 0
+
+
+def _call_quantize(**kw):
+    args = dict(x=1, dtype=isoq.ISOQ_F16, n_heads=1, n_vec=10, d=128, bits=3,
+                variant=isoq.ISOQ_FULL, hs=1280, vs=128, params=16, codes=16, norms=16,
+                ohs=10, stream=None)
+    args.update(kw)
+    return isoq.lib().isoq_quantize(args["x"], args["dtype"], args["n_heads"], args["n_vec"],
+                                    args["d"], args["bits"], args["variant"], args["hs"],
+                                    args["vs"], args["params"], args["codes"], args["norms"],
+                                    args["ohs"], args["stream"])
+
+
+def test_quantize_validation_happens_on_host():
+    # Every case fails validation before any CUDA call, so no GPU is needed.
+    assert _call_quantize(d=100) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert _call_quantize(bits=5) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert _call_quantize(variant=7) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert _call_quantize(dtype=9) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert _call_quantize(n_vec=-1) == isoq.ISOQ_ERR_INVALID_ARG
+    assert _call_quantize(x=None, n_vec=10) == isoq.ISOQ_ERR_INVALID_ARG
+    assert _call_quantize(vs=64) == isoq.ISOQ_ERR_INVALID_ARG
+    assert _call_quantize(ohs=5) == isoq.ISOQ_ERR_INVALID_ARG
+    assert _call_quantize(x=0x1002) == isoq.ISOQ_ERR_UNSUPPORTED      # misaligned
+    assert _call_quantize(vs=132) == isoq.ISOQ_ERR_UNSUPPORTED        # 264-byte rows
+    assert _call_quantize(n_vec=0) == isoq.ISOQ_OK                    # empty is a no-op
+    assert "stride" in isoq.last_error() or isoq.last_error() == ""
+
+
+def test_decode_validation_happens_on_host():
+    lib = isoq.lib()
+    ws = isoq.isoq_decode_workspace_size(1, 8, 2, 64, 128)
+
+    def call(**kw):
+        a = dict(q=256, dtype=isoq.ISOQ_F16, pk=256, pv=256, nk=256, nv=256, sl=256, B=1, Hq=8,
+                 Hkv=2, Tmax=64, d=128, bits=3, variant=0, prk=256, prv=256, scale=0.088,
+                 out=256, ws=4096, wsb=ws)
+        a.update(kw)
+        return lib.isoq_decode_attention(a["q"], a["dtype"], a["pk"], a["pv"], a["nk"], a["nv"],
+                                         a["sl"], a["B"], a["Hq"], a["Hkv"], a["Tmax"], a["d"],
+                                         a["bits"], a["variant"], a["prk"], a["prv"], a["scale"],
+                                         a["out"], a["ws"], a["wsb"], None)
+
+    assert call(Hq=7) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(Hq=64, Hkv=2, wsb=1 << 30) == isoq.ISOQ_ERR_UNSUPPORTED   # group 32 > 16
+    assert call(d=64) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(bits=1) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(wsb=ws - 1) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(ws=4096 + 16) == isoq.ISOQ_ERR_INVALID_ARG               # not 256-aligned
+    assert call(q=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(B=0) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(out=None) == isoq.ISOQ_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for s in (0, -1, -2, -3, -4):
+        assert isoq.status_string(s)
+    assert isoq.status_string(-99) == "unknown status"
+
+
+def test_binding_rejects_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros((1, 4, 128), dtype=torch.float16)
+    p = torch.zeros((1, 32, 8))
+    with pytest.raises(ValueError, match="CUDA"):
+        isoq.isoq_quantize(x, p, 3, isoq.ISOQ_FULL)
