@@ -272,8 +272,9 @@ def run_reference(args):
     return 0
 
 
-def workload_config(workload, n_gpus):
+def workload_config(workload, n_gpus, batch=0):
     B, Hq, Hkv, T, d = WORKLOADS[workload]
+    B = batch or B
     return {
         "workload": workload + "+stage1_quantize_dequantize_d128_b3_f16_n1048576",
         "batch": B, "context": T, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d, "bits": 3,
@@ -281,6 +282,30 @@ def workload_config(workload, n_gpus):
         "l2": "inputs larger than L2: each step streams the whole packed K/V cache (no explicit flush)",
         "parallelism": f"replicas x{n_gpus} (weak; no data-path collective)",
     }
+
+
+# ---------------------------------------------------------------------------
+# Multi-rank helpers (weak-scaled replicas)
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    import torch
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_gbs(bytes_per_step_per_rank, steps, max_ms, n_ranks):
+    """Whole-job GB/s: bytes of all ranks over the slowest rank's time."""
+    return n_ranks * bytes_per_step_per_rank * steps / (max_ms * 1e-3) / 1e9
+
+
+def rank_seed(rank):
+    """Each replica draws its own data."""
+    return 1000 * rank
 
 
 # ---------------------------------------------------------------------------
@@ -310,9 +335,11 @@ def run_isoq(args):
     stream = torch.cuda.current_stream(dev)
 
     B, Hq, Hkv, T, d = WORKLOADS[args.workload]
+    if args.batch:
+        B = args.batch
     bits, variant = 3, isoq.ISOQ_FULL
     pb = d * bits // 8
-    seed0 = 1000 * rank
+    seed0 = rank_seed(rank)
 
     # ---- decode inputs: compress Student-t K/V into the packed cache ----
     prk = torch.from_numpy(np.tile(isoq.isoq_make_params(d, variant, 1, Hkv), (1, 1, 1))).to(dev)
@@ -401,8 +428,8 @@ def run_isoq(args):
     assert isoq.isoq_check_device_error() == 0
 
     # ---- end to end through the API with host buffers (decode half) ----
-    e2e_steps = max(1, min(args.steps, 3))
-    host = [t.cpu().pin_memory() for t in (q, pk, pv, nk, nv, lens)]
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 3))
+    host = [t.cpu().pin_memory() for t in (q, pk, pv, nk, nv, lens)] if e2e_steps else []
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host)
     d2h = out_host.numel() * out_host.element_size()
@@ -421,27 +448,25 @@ def run_isoq(args):
         out_host.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = e0.elapsed_time(e1) if e2e_steps else 0.0
     if dist:
         dist.barrier()
 
     # ---- reduce over ranks: max time, summed bytes ----
-    vals = torch.tensor([total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms = vals.tolist()
+    total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms = max_over_ranks(
+        [total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms], dist, dev)
     n_ranks = world
 
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
-    value = n_ranks * kv_bytes * args.steps / (t_decode * 1e-3) / 1e9
+    value = aggregate_gbs(kv_bytes, args.steps, t_decode, n_ranks)
     split_avg_s = t_split / args.steps * 1e-3
     achieved = kv_bytes / split_avg_s / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_ranks, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": workload_config(args.workload, n_ranks),
+        "config": workload_config(args.workload, n_ranks, args.batch),
         "frac_of_hbm_peak": value / n_ranks / hbm,
         "roofline": {"bound": "hbm", "kernel": "split_mma_kernel<256,Full> (decode split)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
@@ -455,7 +480,7 @@ def run_isoq(args):
                        "gbps": dq_bytes * args.steps / (t_deq * 1e-3) / 1e9},
         "step_ms": {"quantize": t_quant / args.steps, "dequantize": t_deq / args.steps,
                     "decode_split": t_split / args.steps, "decode_combine": t_comb / args.steps},
-        "e2e": {"value": n_ranks * kv_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        "e2e": {"value": (n_ranks * kv_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9) if e2e_steps else None, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "path": "pinned host cache -> device copy -> isoq_decode_attention -> host copy of the output"},
         "gpu_launches": 4 * args.steps,
@@ -481,7 +506,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["isoq", "reference"], default="isoq")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle CPU baseline (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end leg (profiling runs)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the decode batch size (smaller profiling cases)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -4,14 +4,20 @@
 //
 // Per CTA: one (b, kvh, token chunk).  One producer warp streams the chunk's
 // packed K/V rows and float16 norms into shared memory with CTA-local bulk
-// copies (64 tokens per stage, an mbarrier ring); four consumer warps each
-// take a 16-token slab of every stage.
+// copies (64 tokens per stage, an mbarrier ring) from the first cycle on;
+// four consumer warps rotate the queries, then each takes a 16-token slab of
+// every stage.
 //
-// QK (RotaryQuant Table 2 kernel A) runs as mma.sync m16n8k16 with
-// A = dequantised K~ [16 tokens x 16 dims] built in registers and
-// B = q~ [16 dims x 8 heads] (heads >= G are zero).  PV (kernel C) runs as
-// m16n8k16 with A = V~^T [16 dims x 16 tokens] and B = P [16 tokens x 8 heads].
+// QK (RotaryQuant Table 2 kernel A): mma.sync m16n8k16, A = K~ [16 tokens x
+// 16 dims] expanded from the codes in registers, B = q~ [16 dims x 8 columns].
+// q~ is split into float16 hi + lo parts so that its rounding does not reach
+// the scores: for G in {1, 2, 4} the lo parts take the spare columns G..2G-1
+// of the same MMA; otherwise a second MMA adds them.
 // The online softmax (kernel B) runs on the QK accumulator fragments.
+// PV (kernel C): mma.sync with M = 16 dim pairs, K = 8 tokens x 2 parities,
+// N = 4 heads x 2 parities:  D[u][(h, r)] = sum_j V~[j][2u + r] P[j][h], i.e.
+// B[(j, r')][(h, r)] = P[j][h] [r' = r].  Each A register then holds two
+// consecutive dims of one token, exactly what the code lookup produces.
 //
 // Fragment orders.  A fixed permutation of the rotated coordinates cancels in
 // q~.k~ and is undone when the accumulator is written out, and a permutation
@@ -19,12 +25,15 @@
 // chosen so that each lane expands whole 24-bit groups of 8 codes:
 //   QK: lane (g, t) owns tokens g and g+8 and dims [t d/4, (t+1) d/4); MMA kk
 //       uses its dims t d/4 + 4kk + {0,1} (k = 2t, 2t+1) and {2,3} (2t+8, 2t+9).
-//   PV: lane (g, t) owns dims [g d/8, (g+1) d/8) (row g of MMA mm is dim
-//       g d/8 + 2mm, row g+8 is the next dim) and tokens t, t+4, t+8, t+12
-//       (k = 2t, 2t+1, 2t+8, 2t+9).
+//   PV: lane (g, t) owns dims [g d/8, (g+1) d/8) and tokens t, t+4, t+8, t+12;
+//       M-block mb maps row g to dims g d/8 + 4mb + {0,1} and row g+8 to
+//       + {2,3}; K column 2j + r of a token half is token j (0..3 -> t, 4..7
+//       -> t+4 within the lane's pair) with parity r.
 // Code -> float16 centroid is a byte lookup with prmt: the low and high bytes
 // of the 8 centroids sit in two register pairs, a nibble-spread selector picks
 // four entries at once, and two more prmt interleave the bytes into half2.
+// The centroids are scaled by a host-chosen alpha that makes all of them
+// nearly exact in float16; alpha is divided out of the scores and the output.
 
 constexpr int kMmaConsumerWarps = 4;
 constexpr int kMmaThreads = 32 * (kMmaConsumerWarps + 1);
@@ -37,16 +46,17 @@ struct MmaCfg {
   static constexpr int CODES_BYTES = kMmaStageTokens * PB;
   static constexpr int NORM_BYTES = kMmaStageTokens * 2;
   static constexpr int STAGE_BYTES = 2 * CODES_BYTES + 2 * NORM_BYTES;
-  static constexpr int KK = D / 16;                         // MMAs along d (QK) / along dims (PV)
+  static constexpr int KK = D / 16;                         // QK MMAs along d
   static constexpr int QSEG = D / 4;                        // dims per lane in QK
   static constexpr int VSEG = D / 8;                        // dims per lane in PV
+  static constexpr int MB = D / 32;                         // PV M-blocks
   static constexpr int SCRATCH_FLOATS = 8 * D;              // q~ staging, then the warp merge
   static constexpr int SMEM = kMmaStages * STAGE_BYTES + SCRATCH_FLOATS * 4 +
                               2 * kMmaConsumerWarps * 8 * 4 + 2 * kMmaStages * 8 + 16 + 128;
 };
 
 struct MmaLut {
-  uint32_t lo0, lo1, hi0, hi1;  // low/high bytes of the 8 float16 centroids (unit variance)
+  uint32_t lo0, lo1, hi0, hi1;  // low/high bytes of the 8 float16 centroids (scaled)
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -72,13 +82,6 @@ __device__ __forceinline__ uint32_t spread3_to_nibbles(uint32_t w) {
   return x;
 }
 
-// 4 codes of 3 bits (bits 0..11) -> 4 bytes (code k at bits 8k..8k+2).
-__device__ __forceinline__ uint32_t spread3_to_bytes(uint32_t w) {
-  uint32_t x = (w & 0x3Fu) | ((w << 10) & 0x003F0000u);
-  x = (x & 0x00070007u) | ((x << 5) & 0x07000700u);
-  return x;
-}
-
 // Two half2 from a 4-nibble selector: (c[s0], c[s1]) and (c[s2], c[s3]).
 __device__ __forceinline__ void lut4(const MmaLut &l, uint32_t sel, uint32_t &h01, uint32_t &h23) {
   const uint32_t lo = prmt(l.lo0, l.lo1, sel);
@@ -91,7 +94,7 @@ __device__ __forceinline__ uint32_t lds32(const unsigned char *p) {
   return *reinterpret_cast<const uint32_t *>(p);
 }
 
-// Loads the 24-bit code group `grp` from a run of 32-bit words.
+// The 24-bit code group `grp` from a run of 32-bit words.
 template <int NW>
 __device__ __forceinline__ uint32_t group24(const uint32_t (&w)[NW], int grp) {
   const int bit = 24 * grp;
@@ -100,9 +103,16 @@ __device__ __forceinline__ uint32_t group24(const uint32_t (&w)[NW], int grp) {
   return __funnelshift_r(w[wi], (wi + 1 < NW) ? w[wi + 1] : 0u, sh);
 }
 
-template <int D, bool FULL>
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// QIN: q~'s lo parts ride in the spare B columns (G in {1, 2, 4}).
+// NT:  number of 4-head N tiles of the PV product (1 for G <= 4, else 2).
+template <int D, bool FULL, bool QIN, int NT>
 __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs a, const MmaLut lut,
-                                                                float qk_scale_log2) {
+                                                                float qk_scale_log2, float out_scale) {
   using C = MmaCfg<D>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -119,11 +129,11 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.group;
 
-  int T = a.seq_lens[b];
-  T = T < 0 ? 0 : (T > a.tmax ? static_cast<int>(a.tmax) : T);
+  int tlen = a.seq_lens[b];
+  tlen = tlen < 0 ? 0 : (tlen > a.tmax ? static_cast<int>(a.tmax) : tlen);
   const long long t0 = static_cast<long long>(split) * a.chunk;
   long long t1 = t0 + a.chunk;
-  if (t1 > T) t1 = T;
+  if (t1 > tlen) t1 = tlen;
   const int n_tok = t1 > t0 ? static_cast<int>(t1 - t0) : 0;
   const int n_stages = (n_tok + kMmaStageTokens - 1) / kMmaStageTokens;
 
@@ -135,22 +145,10 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
     *abort_flag = 0;
     mbar_fence_init();
   }
-  // Rotate the G queries of this KV head once: q~ = R_K q (all threads).
-  for (int i = tid; i < 8 * D; i += kMmaThreads) {
-    const int g = i / D;
-    float v = 0.f;
-    if (g < G) {
-      const __half *q = static_cast<const __half *>(a.q) +
-                        (static_cast<long long>(b) * a.hq + kvh * G + g) * D;
-      v = __half2float(q[i % D]);
-    }
-    scratch[i] = v;
-  }
   __syncthreads();
-  for (int g = 0; g < G; ++g)
-    rotate_forward_cta<D, FULL>(scratch + g * D, a.params_k + static_cast<size_t>(kvh) * 2 * D);
 
   const long long pair = static_cast<long long>(b) * a.hkv + kvh;
+  constexpr int kConsumers = 32 * kMmaConsumerWarps;
 
   if (warp == kMmaConsumerWarps) {
     // ---------------- bulk-copy producer ----------------
@@ -179,6 +177,7 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
         bulk_load(st + 2 * C::CODES_BYTES + C::NORM_BYTES, nvb + t, 2 * n8, &full_bar[s]);
         issued = i + 1;
       }
+      // Wait for every issued copy before the CTA may exit.
       for (int i = issued > kMmaStages ? issued - kMmaStages : 0; i < issued; ++i) {
         if (!mbar_wait_bounded(&full_bar[i % kMmaStages], (i / kMmaStages) & 1)) {
           atomicOr(&g_decode_error, kErrWaitTimeout);
@@ -186,29 +185,64 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
         }
       }
     }
-    // The producer warp joins the final merge barrier below.
   } else {
     // ---------------- consumers ----------------
+    // Rotate the G queries of this KV head once, q~ = R_K q, while the
+    // producer already streams the first stages.
+    for (int i = tid; i < 8 * D; i += kConsumers) {
+      const int gq = i / D;
+      float v = 0.f;
+      if (gq < G) {
+        const __half *qp = static_cast<const __half *>(a.q) +
+                           (static_cast<long long>(b) * a.hq + kvh * G + gq) * D;
+        v = __half2float(qp[i % D]);
+      }
+      scratch[i] = v;
+    }
+    named_barrier(2, kConsumers);
+    rotate_forward_smem<D, FULL>(scratch, G, a.params_k + static_cast<size_t>(kvh) * 2 * D, tid,
+                                 kConsumers, 2);
+
     const int g = lane >> 2, t = lane & 3;
 
-    // B fragments of q~ for QK: head g, dims t*QSEG + 4kk + {0..3}.
+    // B fragments of q~ (hi + lo float16 parts) for QK: column g, dims
+    // t*QSEG + 4kk + {0..3}.
     uint32_t qf[C::KK][2];
+    uint32_t qflo[QIN ? 1 : C::KK][2];
+    {
+      const int head = QIN ? (g < G ? g : g - G) : g;
+      const bool live = QIN ? (g < 2 * G) : (g < G);
+      const bool lo_col = QIN && g >= G;
 #pragma unroll
-    for (int kk = 0; kk < C::KK; ++kk) {
-      const float *src = scratch + g * D + t * C::QSEG + 4 * kk;
-      __half2 h0 = __floats2half2_rn(src[0], src[1]);
-      __half2 h1 = __floats2half2_rn(src[2], src[3]);
-      if (g >= G) h0 = h1 = __floats2half2_rn(0.f, 0.f);
-      qf[kk][0] = *reinterpret_cast<uint32_t *>(&h0);
-      qf[kk][1] = *reinterpret_cast<uint32_t *>(&h1);
+      for (int kk = 0; kk < C::KK; ++kk) {
+        float v[4], hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[j] = live ? scratch[head * D + t * C::QSEG + 4 * kk + j] : 0.f;
+          hi[j] = __half2float(__float2half_rn(v[j]));
+          lo[j] = v[j] - hi[j];
+        }
+        if (QIN) {
+          const float *src = lo_col ? lo : hi;
+          qf[kk][0] = pack_half2(src[0], src[1]);
+          qf[kk][1] = pack_half2(src[2], src[3]);
+        } else {
+          qf[kk][0] = pack_half2(hi[0], hi[1]);
+          qf[kk][1] = pack_half2(hi[2], hi[3]);
+          qflo[QIN ? 0 : kk][0] = pack_half2(lo[0], lo[1]);
+          qflo[QIN ? 0 : kk][1] = pack_half2(lo[2], lo[3]);
+        }
+      }
     }
 
-    float acc[C::KK][4];
+    float acc[NT][C::MB][4];
 #pragma unroll
-    for (int mm = 0; mm < C::KK; ++mm) acc[mm][0] = acc[mm][1] = acc[mm][2] = acc[mm][3] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int mb = 0; mb < C::MB; ++mb) acc[nt][mb][0] = acc[nt][mb][1] = acc[nt][mb][2] = acc[nt][mb][3] = 0.f;
+    // Online-softmax state in the QK layout: heads 2t, 2t+1 (log2 domain).
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    const uint32_t psel = (g & 1) ? 0x7632u : 0x5410u;
-    const int src1 = 4 * t + (g >> 1), src2 = 16 + 4 * t + (g >> 1);
+    const bool real0 = 2 * t < G, real1 = 2 * t + 1 < G;
 
     for (int i = 0; i < n_stages; ++i) {
       const int s = i % kMmaStages;
@@ -226,7 +260,7 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
         const __half *nk = reinterpret_cast<const __half *>(st + 2 * C::CODES_BYTES) + 16 * warp;
         const __half *nv = reinterpret_cast<const __half *>(st + 2 * C::CODES_BYTES + C::NORM_BYTES) + 16 * warp;
 
-        // ---- QK: S[16 tokens x 8 heads] ----
+        // ---- QK: S[16 tokens x 8 columns] ----
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
         {
           constexpr int NW = C::QSEG * 3 / 32;   // words per token segment (3 or 6)
@@ -246,9 +280,22 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
             lut4(lut, na, a0, a2);
             lut4(lut, nb, a1, a3);
             mma_16816(sc, a0, a1, a2, a3, qf[2 * grp][0], qf[2 * grp][1]);
+            if (!QIN) mma_16816(sc, a0, a1, a2, a3, qflo[QIN ? 0 : 2 * grp][0], qflo[QIN ? 0 : 2 * grp][1]);
             lut4(lut, na >> 16, a0, a2);
             lut4(lut, nb >> 16, a1, a3);
             mma_16816(sc, a0, a1, a2, a3, qf[2 * grp + 1][0], qf[2 * grp + 1][1]);
+            if (!QIN) mma_16816(sc, a0, a1, a2, a3, qflo[QIN ? 0 : 2 * grp + 1][0], qflo[QIN ? 0 : 2 * grp + 1][1]);
+          }
+        }
+        if (QIN) {
+          // Add the lo columns G..2G-1 onto the hi columns 0..G-1.
+          if (G == 1) {
+            sc[0] += sc[1];
+            sc[2] += sc[3];
+          } else {
+            const int o = G >> 1;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[e] += __shfl_xor_sync(0xffffffffu, sc[e], o);
           }
         }
 
@@ -256,10 +303,11 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
         const bool vg = g < nvalid, vg8 = g + 8 < nvalid;
         const float skg = vg ? __half2float(nk[g]) * qk_scale_log2 : 0.f;
         const float skg8 = vg8 ? __half2float(nk[g + 8]) * qk_scale_log2 : 0.f;
-        const float x0 = vg ? sc[0] * skg : -INFINITY;
-        const float x1 = vg ? sc[1] * skg : -INFINITY;
-        const float x2 = vg8 ? sc[2] * skg8 : -INFINITY;
-        const float x3 = vg8 ? sc[3] * skg8 : -INFINITY;
+        // Padded heads hold a constant 0 so that they never move the maximum.
+        const float x0 = real0 ? (vg ? sc[0] * skg : -INFINITY) : 0.f;
+        const float x1 = real1 ? (vg ? sc[1] * skg : -INFINITY) : 0.f;
+        const float x2 = real0 ? (vg8 ? sc[2] * skg8 : -INFINITY) : 0.f;
+        const float x3 = real1 ? (vg8 ? sc[3] * skg8 : -INFINITY) : 0.f;
         float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
@@ -270,17 +318,26 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
         if (__any_sync(0xffffffffu, (mn0 > m0) || (mn1 > m1))) {
           const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mn0);
           const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mn1);
-#pragma unroll
-          for (int mm = 0; mm < C::KK; ++mm) {
-            acc[mm][0] *= f0;
-            acc[mm][1] *= f1;
-            acc[mm][2] *= f0;
-            acc[mm][3] *= f1;
-          }
           l0 *= f0;
           l1 *= f1;
           m0 = mn0;
           m1 = mn1;
+          // The PV accumulator of lane (g, t) holds head nt*4 + t.
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const int h = nt * 4 + t;
+            const int src = 4 * g + (h >> 1);
+            const float F0 = __shfl_sync(0xffffffffu, f0, src);
+            const float F1 = __shfl_sync(0xffffffffu, f1, src);
+            const float f = (h & 1) ? F1 : F0;
+#pragma unroll
+            for (int mb = 0; mb < C::MB; ++mb) {
+              acc[nt][mb][0] *= f;
+              acc[nt][mb][1] *= f;
+              acc[nt][mb][2] *= f;
+              acc[nt][mb][3] *= f;
+            }
+          }
         }
         const float p0 = exp2f(x0 - m0), p1 = exp2f(x1 - m1);
         const float p2 = exp2f(x2 - m0), p3 = exp2f(x3 - m1);
@@ -288,51 +345,63 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
         l1 += p1 + p3;
         const float svg = vg ? __half2float(nv[g]) : 0.f;
         const float svg8 = vg8 ? __half2float(nv[g + 8]) : 0.f;
-        __half2 h01 = __floats2half2_rn(p0 * svg, p1 * svg);
-        __half2 h23 = __floats2half2_rn(p2 * svg8, p3 * svg8);
-        const uint32_t u01 = *reinterpret_cast<uint32_t *>(&h01);
-        const uint32_t u23 = *reinterpret_cast<uint32_t *>(&h23);
-        // P fragment for PV: lane (g, t) needs tokens t, t+4, t+8, t+12 of head g.
-        const uint32_t x_t = __shfl_sync(0xffffffffu, u01, src1);
-        const uint32_t x_t4 = __shfl_sync(0xffffffffu, u01, src2);
-        const uint32_t x_t8 = __shfl_sync(0xffffffffu, u23, src1);
-        const uint32_t x_t12 = __shfl_sync(0xffffffffu, u23, src2);
-        uint32_t pb0 = prmt(x_t, x_t4, psel);
-        uint32_t pb1 = prmt(x_t8, x_t12, psel);
-        if (g >= G) pb0 = pb1 = 0u;
+        const uint32_t u01 = pack_half2(p0 * svg, p1 * svg);      // token g, heads 2t, 2t+1
+        const uint32_t u23 = pack_half2(p2 * svg8, p3 * svg8);    // token g+8
 
-        // ---- PV: O^T[dims x 8 heads] += V~^T[dims x 16 tokens] P ----
+        // ---- PV: unpack this lane's 4 tokens once, reuse for the N tiles ----
+        constexpr int VB = C::VSEG * 3 / 8;     // bytes per token segment (6 or 12)
+        constexpr int NWV = (VB + 3) / 4 + 1;   // words loaded per token (room for alignment)
+        uint32_t w[4][NWV];
         {
-          constexpr int VB = C::VSEG * 3 / 8;     // bytes per token segment (6 or 12)
-          constexpr int NW = (VB + 3) / 4 + 1;    // words loaded per token (room for alignment)
           const int off = g * VB;
           const int off4 = off & ~3, sh = (off & 3) * 8;
-          uint32_t w[4][NW];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const unsigned char *row = vc + (t + 4 * r) * C::PB + off4;
 #pragma unroll
-            for (int k = 0; k < NW; ++k) w[r][k] = (4 * k < VB + (off & 3)) ? lds32(row + 4 * k) : 0u;
+            for (int k = 0; k < NWV; ++k) w[r][k] = (4 * k < VB + (off & 3)) ? lds32(row + 4 * k) : 0u;
             if (sh) {
 #pragma unroll
-              for (int k = 0; k + 1 < NW; ++k) w[r][k] = __funnelshift_r(w[r][k], w[r][k + 1], sh);
+              for (int k = 0; k + 1 < NWV; ++k) w[r][k] = __funnelshift_r(w[r][k], w[r][k + 1], sh);
             }
           }
+        }
+        // B fragments of P for each N tile: column g = (head nt*4 + g/2, parity g&1).
+        uint32_t pb[NT][4];
 #pragma unroll
-          for (int grp = 0; grp < C::VSEG / 8; ++grp) {
-            const uint32_t ga = group24(w[0], grp), gb = group24(w[1], grp);
-            const uint32_t gc = group24(w[2], grp), gd = group24(w[3], grp);
+        for (int nt = 0; nt < NT; ++nt) {
+          const int h = nt * 4 + (g >> 1);
+          const int src1 = 4 * t + (h >> 1), src2 = 16 + 4 * t + (h >> 1);
+          const uint32_t x_t = __shfl_sync(0xffffffffu, u01, src1);
+          const uint32_t x_t4 = __shfl_sync(0xffffffffu, u01, src2);
+          const uint32_t x_t8 = __shfl_sync(0xffffffffu, u23, src1);
+          const uint32_t x_t12 = __shfl_sync(0xffffffffu, u23, src2);
+          const uint32_t e2 = 2u * (h & 1);
+          const uint32_t sel = (g & 1) ? (0x44u | (e2 << 8) | ((e2 + 1u) << 12))
+                                       : (e2 | ((e2 + 1u) << 4) | 0x4400u);
+          const bool live = h < G;
+          pb[nt][0] = live ? prmt(x_t, 0u, sel) : 0u;
+          pb[nt][1] = live ? prmt(x_t4, 0u, sel) : 0u;
+          pb[nt][2] = live ? prmt(x_t8, 0u, sel) : 0u;
+          pb[nt][3] = live ? prmt(x_t12, 0u, sel) : 0u;
+        }
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {        // dims 0-3, then 4-7 of the group
-              const uint32_t sab = spread3_to_bytes(ga >> (12 * hh)) | (spread3_to_bytes(gb >> (12 * hh)) << 4);
-              const uint32_t scd = spread3_to_bytes(gc >> (12 * hh)) | (spread3_to_bytes(gd >> (12 * hh)) << 4);
+        for (int grp = 0; grp < C::VSEG / 8; ++grp) {
+          uint32_t n4[4];
 #pragma unroll
-              for (int j = 0; j < 2; ++j) {         // dim pairs (0,1), (2,3)
-                uint32_t a0, a1, a2, a3;
-                lut4(lut, sab >> (16 * j), a0, a1);
-                lut4(lut, scd >> (16 * j), a2, a3);
-                mma_16816(acc[4 * grp + 2 * hh + j], a0, a1, a2, a3, pb0, pb1);
-              }
+          for (int r = 0; r < 4; ++r) n4[r] = spread3_to_nibbles(group24(w[r], grp));
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {      // codes 0-3, then 4-7: M-block 2grp + half
+            const int mb = 2 * grp + half;
+            uint32_t ta0, ta1, tb0, tb1, tc0, tc1, td0, td1;
+            lut4(lut, n4[0] >> (16 * half), ta0, ta1);   // token t
+            lut4(lut, n4[1] >> (16 * half), tb0, tb1);   // token t+4
+            lut4(lut, n4[2] >> (16 * half), tc0, tc1);   // token t+8
+            lut4(lut, n4[3] >> (16 * half), td0, td1);   // token t+12
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_16816(acc[nt][mb], ta0, ta1, tb0, tb1, pb[nt][0], pb[nt][1]);
+              mma_16816(acc[nt][mb], tc0, tc1, td0, td1, pb[nt][2], pb[nt][3]);
             }
           }
         }
@@ -347,46 +416,53 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
       l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
-    named_barrier(1, 32 * kMmaConsumerWarps);   // all warps are done with the q~ scratch
-    for (int i = tid; i < 8 * D; i += 32 * kMmaConsumerWarps) scratch[i] = 0.f;
+    named_barrier(1, kConsumers);   // all warps are done with the q~ scratch
     if (g == 0) {
       wm[warp * 8 + 2 * t] = m0;
       wm[warp * 8 + 2 * t + 1] = m1;
       wl[warp * 8 + 2 * t] = l0;
       wl[warp * 8 + 2 * t + 1] = l1;
     }
-    named_barrier(1, 32 * kMmaConsumerWarps);
-    // Merge the warps' states into scratch[head][dim] (rotated domain).
-    float f[2];
+    named_barrier(1, kConsumers);
+    // Merge the warps' accumulators into scratch[head][dim] (rotated domain),
+    // one warp after the other so that the sum order is fixed.
+    float f[NT];
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int h = 2 * t + e;
+    for (int nt = 0; nt < NT; ++nt) {
+      const int h = nt * 4 + t;
       float mstar = -INFINITY;
       for (int w2 = 0; w2 < kMmaConsumerWarps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
       const float mine = wm[warp * 8 + h];
-      f[e] = (mine == -INFINITY) ? 0.f : exp2f(mine - mstar);
+      f[nt] = (mine == -INFINITY) ? 0.f : exp2f(mine - mstar);
     }
-    if (2 * t < G) {
+    for (int w2 = 0; w2 < kMmaConsumerWarps; ++w2) {
+      if (warp == w2) {
 #pragma unroll
-      for (int mm = 0; mm < C::KK; ++mm) {
-        const int dim = g * C::VSEG + 2 * mm;
-        atomicAdd(&scratch[(2 * t) * D + dim], acc[mm][0] * f[0]);
-        atomicAdd(&scratch[(2 * t) * D + dim + 1], acc[mm][2] * f[0]);
-        if (2 * t + 1 < G) {
-          atomicAdd(&scratch[(2 * t + 1) * D + dim], acc[mm][1] * f[1]);
-          atomicAdd(&scratch[(2 * t + 1) * D + dim + 1], acc[mm][3] * f[1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          const int h = nt * 4 + t;
+          if (h < G) {
+#pragma unroll
+            for (int mb = 0; mb < C::MB; ++mb) {
+              float *dst = scratch + h * D + g * C::VSEG + 4 * mb;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float v = acc[nt][mb][e] * f[nt];
+                dst[e] = (w2 == 0) ? v : dst[e] + v;
+              }
+            }
+          }
         }
       }
+      named_barrier(1, kConsumers);
     }
   }
   __syncthreads();
 
-  // Write one partial state per query head: natural-log max, sum, acc / sqrt(d).
-  const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+  // One partial state per query head: natural-log max, sum, acc (unscaled).
   for (int h = 0; h < G; ++h) {
     const long long slot = (static_cast<long long>(b) * a.hq + kvh * G + h) * a.n_splits + split;
     float *acc_out = a.ws_acc + slot * D;
-    for (int i = tid; i < D; i += kMmaThreads) acc_out[i] = scratch[h * D + i] * inv_sqrt_d;
+    for (int i = tid; i < D; i += kMmaThreads) acc_out[i] = scratch[h * D + i] * out_scale;
     if (tid == 0) {
       float mstar = -INFINITY, l = 0.f;
       for (int w2 = 0; w2 < kMmaConsumerWarps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
@@ -404,10 +480,46 @@ inline uint32_t half_bits(float v) {
   return static_cast<uint32_t>(*reinterpret_cast<unsigned short *>(&h));
 }
 
-template <int D, bool FULL>
+// Round-to-nearest-even to an 11-bit significand (float16, normal range).
+inline double round_f16(double x) {
+  int e;
+  const double m = std::frexp(x, &e);
+  return std::ldexp(std::nearbyint(std::ldexp(m, 11)), e - 11);
+}
+
+// Scale alpha in [1, 2) minimising the largest relative float16 rounding
+// error of alpha * c_k over the unit-variance 3-bit centroids (searched once).
+double centroid_scale_3bit() {
+  static double alpha = 0.0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    CodebookF32 cb;
+    codebook_f32(128, 3, &cb);
+    double mags[4];
+    for (int k = 0; k < 4; ++k) mags[k] = static_cast<double>(cb.centroid[4 + k]) * std::sqrt(128.0);
+    double best = 1.0, best_err = 1.0;
+    const int steps = 4000000;
+    for (int i = 0; i < steps; ++i) {
+      const double al = 1.0 + static_cast<double>(i) / steps;
+      double err = 0.0;
+      for (int k = 0; k < 4 && err < best_err; ++k) {
+        const double v = al * mags[k];
+        err = std::fmax(err, std::fabs(round_f16(v) - v) / v);
+      }
+      if (err < best_err) {
+        best_err = err;
+        best = al;
+      }
+    }
+    alpha = best;
+  });
+  return alpha;
+}
+
+template <int D, bool FULL, bool QIN, int NT>
 int launch_split_mma(const SplitArgs &a, cudaStream_t stream) {
   using C = MmaCfg<D>;
-  auto kernel = split_mma_kernel<D, FULL>;
+  auto kernel = split_mma_kernel<D, FULL, QIN, NT>;
   static bool configured = false;
   static std::mutex mu;
   {
@@ -418,19 +530,21 @@ int launch_split_mma(const SplitArgs &a, cudaStream_t stream) {
       configured = true;
     }
   }
-  // float16 centroids of the unit-variance codebook (the 1/sqrt(d) of the
-  // N(0, 1/d) codebook is folded into the score scale and the output).
+  // float16 centroids of the unit-variance codebook times alpha; the
+  // 1/(sqrt(d) alpha) is folded into the score scale and the output scale.
+  const double alpha = centroid_scale_3bit();
   const float sqrt_d = std::sqrt(static_cast<float>(D));
   uint32_t lo[2] = {0, 0}, hi[2] = {0, 0};
   for (int k = 0; k < 8; ++k) {
-    const uint32_t hb = half_bits(a.centroid[k] * sqrt_d);
+    const uint32_t hb = half_bits(static_cast<float>(a.centroid[k] * sqrt_d * alpha));
     lo[k / 4] |= (hb & 0xFFu) << (8 * (k % 4));
     hi[k / 4] |= (hb >> 8) << (8 * (k % 4));
   }
   MmaLut lut{lo[0], lo[1], hi[0], hi[1]};
-  const float qk_scale_log2 = a.scale / sqrt_d * 1.4426950408889634f;
+  const float inv = static_cast<float>(1.0 / (static_cast<double>(sqrt_d) * alpha));
+  const float qk_scale_log2 = a.scale * inv * 1.4426950408889634f;
   dim3 grid(a.n_splits, a.hkv, a.batch);
-  kernel<<<grid, kMmaThreads, C::SMEM, stream>>>(a, lut, qk_scale_log2);
+  kernel<<<grid, kMmaThreads, C::SMEM, stream>>>(a, lut, qk_scale_log2, inv);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode mma launch: %s", cudaGetErrorString(e));
   return ISOQ_OK;
@@ -443,8 +557,16 @@ bool mma_path_supported(int dtype, int d, int bits, const SplitArgs &a) {
          (reinterpret_cast<uintptr_t>(a.norms_v) & 15u) == 0;
 }
 
+template <int D, bool FULL>
+int run_split_mma_d(const SplitArgs &a, cudaStream_t st) {
+  const int G = a.group;
+  if (G == 1 || G == 2 || G == 4) return launch_split_mma<D, FULL, true, 1>(a, st);
+  if (G <= 4) return launch_split_mma<D, FULL, false, 1>(a, st);
+  return launch_split_mma<D, FULL, false, 2>(a, st);
+}
+
 int run_split_mma(int d, int variant, const SplitArgs &a, cudaStream_t st) {
   if (d == 128)
-    return variant == ISOQ_FULL ? launch_split_mma<128, true>(a, st) : launch_split_mma<128, false>(a, st);
-  return variant == ISOQ_FULL ? launch_split_mma<256, true>(a, st) : launch_split_mma<256, false>(a, st);
+    return variant == ISOQ_FULL ? run_split_mma_d<128, true>(a, st) : run_split_mma_d<128, false>(a, st);
+  return variant == ISOQ_FULL ? run_split_mma_d<256, true>(a, st) : run_split_mma_d<256, false>(a, st);
 }

@@ -37,32 +37,46 @@ using namespace isoq::dev;
 
 __device__ unsigned int g_decode_error = 0;
 
-// Forward rotation q~ = R q of one vector held in shared memory, by all
-// threads of the CTA: WHT butterflies (stride h = 1 ... d/2), 1/sqrt(d), then
-// the per-block quaternion map.
+// Barrier over the threads taking part in a shared-memory rotation: the whole
+// CTA (bar_id 0 -> __syncthreads) or a named barrier over `nthreads` threads.
+__device__ __forceinline__ void rotation_sync(int bar_id, int nthreads) {
+  if (bar_id == 0)
+    __syncthreads();
+  else
+    named_barrier(bar_id, nthreads);
+}
+
+// Forward rotation q~ = R q of `nvec` vectors v[nvec][D] held in shared
+// memory, all sharing one head's parameters, by threads [0, nthreads): WHT
+// butterflies (stride h = 1 ... d/2) for all vectors per barrier, 1/sqrt(d),
+// then the per-block quaternion map.
 template <int D, bool FULL>
-__device__ void rotate_forward_cta(float *v, const float *params_head) {
-  const int tid = threadIdx.x, nt = blockDim.x;
+__device__ void rotate_forward_smem(float *v, int nvec, const float *params_head, int tid,
+                                    int nthreads, int bar_id) {
 #pragma unroll 1
   for (int h = 1; h < D; h <<= 1) {
-    for (int p = tid; p < D / 2; p += nt) {
+    for (int idx = tid; idx < nvec * (D / 2); idx += nthreads) {
+      const int g = idx / (D / 2), p = idx % (D / 2);
+      float *w = v + g * D;
       const int i = (p / h) * 2 * h + (p % h);
-      const float a = v[i], b = v[i + h];
-      v[i] = a + b;
-      v[i + h] = a - b;
+      const float a = w[i], b = w[i + h];
+      w[i] = a + b;
+      w[i + h] = a - b;
     }
-    __syncthreads();
+    rotation_sync(bar_id, nthreads);
   }
   const float inv = rsqrtf(static_cast<float>(D));
-  for (int bi = tid; bi < D / 4; bi += nt) {
-    const Quat x{v[4 * bi] * inv, v[4 * bi + 1] * inv, v[4 * bi + 2] * inv, v[4 * bi + 3] * inv};
+  for (int idx = tid; idx < nvec * (D / 4); idx += nthreads) {
+    const int g = idx / (D / 4), bi = idx % (D / 4);
+    float *w = v + g * D + 4 * bi;
+    const Quat x{w[0] * inv, w[1] * inv, w[2] * inv, w[3] * inv};
     const Quat u = block_forward(load_quat(params_head + 8 * bi), load_quat(params_head + 8 * bi + 4), x, FULL);
-    v[4 * bi] = u.w;
-    v[4 * bi + 1] = u.x;
-    v[4 * bi + 2] = u.y;
-    v[4 * bi + 3] = u.z;
+    w[0] = u.w;
+    w[1] = u.x;
+    w[2] = u.y;
+    w[3] = u.z;
   }
-  __syncthreads();
+  rotation_sync(bar_id, nthreads);
 }
 
 // Inverse rotation x = H_d R_SO4^T u / sqrt(d) of one vector in shared memory.
@@ -144,7 +158,8 @@ __global__ void __launch_bounds__(kGenericThreads) split_generic_kernel(const Sp
     for (int i = tid; i < D; i += kGenericThreads) qrot[g * D + i] = to_f32<T>(q[i]);
   }
   __syncthreads();
-  for (int g = 0; g < G; ++g) rotate_forward_cta<D, FULL>(qrot + g * D, a.params_k + static_cast<size_t>(kvh) * 2 * D);
+  rotate_forward_smem<D, FULL>(qrot, G, a.params_k + static_cast<size_t>(kvh) * 2 * D, tid,
+                               kGenericThreads, 0);
 
   const long long pair = static_cast<long long>(b) * a.hkv + kvh;
   const uint8_t *kbase = a.packed_k + pair * a.tmax * PB;
