@@ -52,6 +52,9 @@ SIGNATURES = [
                                _F, _P, _SZ, _P]),
     ("isoq_decode_combine", _I, [_I, _P, _I, _I, _I, _I64, _I, _I, _P, _P, _P, _SZ, _P]),
     ("isoq_check_device_error", _I, [_P]),
+    ("isoq_decode_static_workspace_bytes", _SZ, []),
+    ("isoq_decode_attention_static", _I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I,
+                                          _I, _P, _P, _F, _P, _P]),
 ]
 
 _lib = None
@@ -310,3 +313,31 @@ def isoq_check_device_error(stream=None, device=None) -> int:
 
 def _torch_dtype_of(code: int):
     return _torch_dtype(code)
+
+
+def isoq_decode_attention_static(q, packed_k, packed_v, norms_k, norms_v, seq_lens, params_k,
+                                 params_v, bits: int, variant: int, scale: Optional[float] = None,
+                                 out=None, stream=None):
+    """isoq_decode_attention with the library's built-in device workspace.
+
+    For callers that cannot allocate device scratch; the output buffer may be
+    passed in (``out``) so that the call itself allocates nothing.
+    """
+    torch = _torch()
+    B, Hq, Hkv, Tmax, d = _decode_shapes(q, packed_k, bits)
+    dev = _require_cuda(q, packed_k, packed_v, norms_k, norms_v, seq_lens, params_k, params_v, out)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=q.dtype, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().isoq_decode_attention_static(
+            _ptr(q), _dtype_code(q), _ptr(packed_k), _ptr(packed_v), _ptr(norms_k), _ptr(norms_v),
+            _ptr(seq_lens), B, Hq, Hkv, Tmax, d, bits, variant, _ptr(params_k), _ptr(params_v),
+            float(scale), _ptr(out), _stream(dev, stream))
+    _check(st, "isoq_decode_attention_static")
+    return out
+
+
+def isoq_decode_static_workspace_bytes() -> int:
+    return lib().isoq_decode_static_workspace_bytes()

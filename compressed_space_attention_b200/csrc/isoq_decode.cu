@@ -486,3 +486,81 @@ __attribute__((visibility("hidden"))) int isoq_detail_take_decode_error(cudaStre
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention without caller-provided scratch.
+//
+// Some callers cannot allocate device memory: a host program whose device
+// memory belongs to another framework's allocator, a plugin that is handed
+// only its input and output buffers, or code on a path where cudaMalloc's
+// implicit device-wide synchronisation is not acceptable.  For them the
+// split-K partial states live in one file-scope device array of fixed size
+// (every GPU that loads this library holds it until the process exits), and
+// the entry point below allocates nothing.
+// ---------------------------------------------------------------------------
+
+namespace isoq {
+namespace decode {
+
+constexpr size_t kStaticWorkspaceBytes = size_t(16) << 20;  // 16 MiB per device
+
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+// Device address of g_static_workspace on the current device.  Host code
+// sees only a host-side stand-in for the array, so the device address is
+// looked up once per device, with that device current, and cached.
+int static_workspace_address(void **out) {
+  static std::mutex mu;
+  static void *addr[256] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 256) return set_error(ISOQ_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess || !p)
+      return set_error(ISOQ_ERR_CUDA, "cudaGetSymbolAddress(static workspace): %s", cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return ISOQ_OK;
+}
+
+}  // namespace decode
+}  // namespace isoq
+
+extern "C" size_t isoq_decode_static_workspace_bytes(void) { return isoq::decode::kStaticWorkspaceBytes; }
+
+extern "C" int isoq_decode_attention_static(const void *q_dev, int dtype,
+                                            const uint8_t *packed_k_dev,
+                                            const uint8_t *packed_v_dev,
+                                            const uint16_t *norms_k_dev,
+                                            const uint16_t *norms_v_dev,
+                                            const int32_t *seq_lens_dev, int B, int Hq, int Hkv,
+                                            int64_t Tmax, int d, int bits, int variant,
+                                            const float *params_k_dev,
+                                            const float *params_v_dev, float scale,
+                                            void *out_dev, isoq_stream_t stream) {
+  clear_error();
+  const size_t need = isoq_decode_workspace_size(B, Hq, Hkv, Tmax, d);
+  if (need == 0)  // invalid shapes: let the regular validation report which
+    return isoq_decode_attention(q_dev, dtype, packed_k_dev, packed_v_dev, norms_k_dev,
+                                 norms_v_dev, seq_lens_dev, B, Hq, Hkv, Tmax, d, bits, variant,
+                                 params_k_dev, params_v_dev, scale, out_dev, nullptr, 0, stream);
+  if (need > decode::kStaticWorkspaceBytes)
+    return set_error(ISOQ_ERR_UNSUPPORTED,
+                     "these shapes need %zu bytes of decode workspace; the built-in workspace "
+                     "holds %zu (use isoq_decode_attention with a caller-provided workspace)",
+                     need, decode::kStaticWorkspaceBytes);
+  void *ws = nullptr;
+  const int st = decode::static_workspace_address(&ws);
+  if (st) return st;
+  // The split kernel writes every partial slot the combine reads, so the
+  // array needs no clearing between calls.
+  return isoq_decode_attention(q_dev, dtype, packed_k_dev, packed_v_dev, norms_k_dev, norms_v_dev,
+                               seq_lens_dev, B, Hq, Hkv, Tmax, d, bits, variant, params_k_dev,
+                               params_v_dev, scale, out_dev, ws, decode::kStaticWorkspaceBytes,
+                               stream);
+}

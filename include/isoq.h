@@ -14,9 +14,10 @@
  *    never throws or aborts.  Arguments are validated on the host before any
  *    device work is queued; a call that fails validation writes nothing.
  *  - Pointers named *_dev are device pointers, *_host host pointers.  The
- *    caller owns every buffer; the library allocates no device memory and
- *    keeps no device state except one 32-bit device error word per device
- *    (see isoq_check_device_error).  Host state: a mutex-guarded cache of
+ *    caller owns every buffer; the library allocates no device memory.  Its
+ *    only device state is one 32-bit error word per device (see
+ *    isoq_check_device_error) and the fixed workspace array of
+ *    isoq_decode_attention_static.  Host state: a mutex-guarded cache of
  *    codebooks and a thread-local error message.
  *  - Device work is queued asynchronously on `stream` (a cudaStream_t; NULL
  *    is the legacy default stream).  Launch failures return ISOQ_ERR_CUDA
@@ -206,6 +207,38 @@ int isoq_decode_combine(int dtype, const int32_t *seq_lens_dev, int B, int Hq, i
                         int64_t Tmax, int d, int variant, const float *params_v_dev,
                         void *out_dev, const void *workspace_dev, size_t workspace_bytes,
                         isoq_stream_t stream);
+
+/*
+ * Decode attention for callers that cannot allocate device memory.  The
+ * method's pages have no counterpart to this entry point; it is a
+ * convenience of this library.
+ *
+ * Same computation, arguments and rules as isoq_decode_attention, without
+ * the workspace arguments: the split-K partial states go to one device array
+ * of isoq_decode_static_workspace_bytes() bytes (16 MiB) that the library
+ * defines at file scope, so every GPU that loads the library holds it until
+ * the process exits.  Intended for callers that have no device allocator of
+ * their own to hand (a host program whose device memory is owned by another
+ * framework, a plugin given only its input and output buffers, a path where
+ * cudaMalloc's implicit synchronisation is not acceptable).  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *   - Shapes whose workspace (isoq_decode_workspace_size) exceeds the array
+ *     are rejected with ISOQ_ERR_UNSUPPORTED before any launch.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress and caches it; make that first call before any
+ *     stream capture on that device.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (nothing in it needs clearing: each call writes every slot it reads).
+ *     Calls whose kernels overlap on the GPU, e.g. on two streams without an
+ *     ordering between them, race on it.
+ */
+size_t isoq_decode_static_workspace_bytes(void);
+int isoq_decode_attention_static(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
+                                 const uint8_t *packed_v_dev, const uint16_t *norms_k_dev,
+                                 const uint16_t *norms_v_dev, const int32_t *seq_lens_dev, int B,
+                                 int Hq, int Hkv, int64_t Tmax, int d, int bits, int variant,
+                                 const float *params_k_dev, const float *params_v_dev,
+                                 float scale, void *out_dev, isoq_stream_t stream);
 
 /*
  * Reads and clears the current device's error word after synchronising
