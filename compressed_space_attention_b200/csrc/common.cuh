@@ -171,5 +171,49 @@ __device__ __forceinline__ Quat h4_column(int c) {
               (__popc(c & 3) & 1) ? -1.0f : 1.0f};
 }
 
+// ---------------------------------------------------------------------------
+// Packed-code layout.  b = 2, 4: LSB-first bitstream (code i at bits
+// [b*i, b*i + b)).  b = 3: groups of 32 codes in three 32-bit words; code
+// 8r + j of a group sits in bits [4j, 4j+3) of word r, and bit r of code
+// 24 + j in bit 4j + 3 of word r, so that codes occupy 4-bit fields.
+// ---------------------------------------------------------------------------
+
+// ORs code number i (0 <= i < 64, compile-time after unrolling) of a 64-code
+// run into the run's packed words w.
+template <int BITS>
+__device__ __forceinline__ void pack_code(uint32_t *w, int i, uint32_t code) {
+  if constexpr (BITS == 3) {
+    const int grp = i >> 5, m = i & 31;
+    if (m < 24) {
+      w[3 * grp + (m >> 3)] += code << (4 * (m & 7));
+    } else {
+      const int j = m - 24;
+#pragma unroll
+      for (int r = 0; r < 3; ++r) w[3 * grp + r] |= ((code >> r) & 1u) << (4 * j + 3);
+    }
+  } else {
+    const int bp = BITS * i;
+    w[bp >> 5] |= code << (bp & 31);
+    if ((bp & 31) + BITS > 32) w[(bp >> 5) + 1] |= code >> (32 - (bp & 31));
+  }
+}
+
+// Code number i of a run of packed words (the inverse of pack_code).
+template <int BITS>
+__device__ __forceinline__ uint32_t unpack_code(const uint32_t *w, int i) {
+  if constexpr (BITS == 3) {
+    const int grp = i >> 5, m = i & 31;
+    if (m < 24) return (w[3 * grp + (m >> 3)] >> (4 * (m & 7))) & 7u;
+    const int sh = 4 * (m - 24) + 3;
+    return ((w[3 * grp] >> sh) & 1u) | (((w[3 * grp + 1] >> sh) & 1u) << 1) |
+           (((w[3 * grp + 2] >> sh) & 1u) << 2);
+  } else {
+    const int bp = BITS * i;
+    uint32_t c = w[bp >> 5] >> (bp & 31);
+    if ((bp & 31) + BITS > 32) c |= w[(bp >> 5) + 1] << (32 - (bp & 31));
+    return c & ((1u << BITS) - 1u);
+  }
+}
+
 }  // namespace dev
 }  // namespace isoq

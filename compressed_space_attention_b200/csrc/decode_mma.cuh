@@ -22,7 +22,8 @@
 // Fragment orders.  A fixed permutation of the rotated coordinates cancels in
 // q~.k~ and is undone when the accumulator is written out, and a permutation
 // of the tokens inside a slab is applied identically to P and V~; both are
-// chosen so that each lane expands whole 24-bit groups of 8 codes:
+// chosen so that each lane expands whole 32-code groups (three words in the
+// layout of common.cuh, codes in 4-bit fields):
 //   QK: lane (g, t) owns tokens g and g+8 and dims [t d/4, (t+1) d/4); MMA kk
 //       uses its dims t d/4 + 4kk + {0,1} (k = 2t, 2t+1) and {2,3} (2t+8, 2t+9).
 //   PV: lane (g, t) owns dims [g d/8, (g+1) d/8) and tokens t, t+4, t+8, t+12;
@@ -30,8 +31,9 @@
 //       + {2,3}; K column 2j + r of a token half is token j (0..3 -> t, 4..7
 //       -> t+4 within the lane's pair) with parity r.
 // Code -> float16 centroid is a byte lookup with prmt: the low and high bytes
-// of the 8 centroids sit in two register pairs, a nibble-spread selector picks
-// four entries at once, and two more prmt interleave the bytes into half2.
+// of the 8 centroids sit in two register pairs, a selector made of four code
+// nibbles picks four entries at once, and two more prmt interleave the bytes
+// into half2.
 // The centroids are scaled by a host-chosen alpha that makes all of them
 // nearly exact in float16; alpha is divided out of the scores and the output.
 
@@ -74,12 +76,26 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// 8 codes of 3 bits (bits 0..23) -> 8 nibbles (code k at bits 4k..4k+2).
-__device__ __forceinline__ uint32_t spread3_to_nibbles(uint32_t w) {
-  uint32_t x = (w & 0xFFFu) | ((w << 4) & 0x0FFF0000u);
-  x = (x & 0x003F003Fu) | ((x << 2) & 0x3F003F00u);
-  x = (x & 0x07070707u) | ((x << 1) & 0x70707070u);
-  return x;
+// prmt selectors of one 32-code group (three words in the layout of
+// common.cuh): m_r = codes 8r..8r+7 with the spare bits cleared, and e =
+// codes 24..31 gathered from the spare bits.  Quad q (codes 4q..4q+3) is the
+// low or high half of one of them.
+struct GroupSel {
+  uint32_t m0, m1, m2, e;
+};
+
+__device__ __forceinline__ GroupSel group_selectors(uint32_t w0, uint32_t w1, uint32_t w2) {
+  GroupSel s;
+  s.m0 = w0 & 0x77777777u;
+  s.m1 = w1 & 0x77777777u;
+  s.m2 = w2 & 0x77777777u;
+  s.e = ((w0 >> 3) & 0x11111111u) | ((w1 >> 2) & 0x22222222u) | ((w2 >> 1) & 0x44444444u);
+  return s;
+}
+
+__device__ __forceinline__ uint32_t quad_selector(const GroupSel &s, int q) {
+  const uint32_t x = q < 2 ? s.m0 : (q < 4 ? s.m1 : (q < 6 ? s.m2 : s.e));
+  return (q & 1) ? (x >> 16) : x;
 }
 
 // Two half2 from a 4-nibble selector: (c[s0], c[s1]) and (c[s2], c[s3]).
@@ -92,15 +108,6 @@ __device__ __forceinline__ void lut4(const MmaLut &l, uint32_t sel, uint32_t &h0
 
 __device__ __forceinline__ uint32_t lds32(const unsigned char *p) {
   return *reinterpret_cast<const uint32_t *>(p);
-}
-
-// The 24-bit code group `grp` from a run of 32-bit words.
-template <int NW>
-__device__ __forceinline__ uint32_t group24(const uint32_t (&w)[NW], int grp) {
-  const int bit = 24 * grp;
-  const int wi = bit >> 5, sh = bit & 31;
-  if (sh == 0) return w[wi];
-  return __funnelshift_r(w[wi], (wi + 1 < NW) ? w[wi + 1] : 0u, sh);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -273,18 +280,18 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
             wg8[k] = lds32(rg8 + 4 * k);
           }
 #pragma unroll
-          for (int grp = 0; grp < C::QSEG / 8; ++grp) {
-            const uint32_t na = spread3_to_nibbles(group24(wg, grp));
-            const uint32_t nb = spread3_to_nibbles(group24(wg8, grp));
-            uint32_t a0, a1, a2, a3;
-            lut4(lut, na, a0, a2);
-            lut4(lut, nb, a1, a3);
-            mma_16816(sc, a0, a1, a2, a3, qf[2 * grp][0], qf[2 * grp][1]);
-            if (!QIN) mma_16816(sc, a0, a1, a2, a3, qflo[QIN ? 0 : 2 * grp][0], qflo[QIN ? 0 : 2 * grp][1]);
-            lut4(lut, na >> 16, a0, a2);
-            lut4(lut, nb >> 16, a1, a3);
-            mma_16816(sc, a0, a1, a2, a3, qf[2 * grp + 1][0], qf[2 * grp + 1][1]);
-            if (!QIN) mma_16816(sc, a0, a1, a2, a3, qflo[QIN ? 0 : 2 * grp + 1][0], qflo[QIN ? 0 : 2 * grp + 1][1]);
+          for (int gq = 0; gq < C::QSEG / 32; ++gq) {
+            const GroupSel sa = group_selectors(wg[3 * gq], wg[3 * gq + 1], wg[3 * gq + 2]);
+            const GroupSel sb = group_selectors(wg8[3 * gq], wg8[3 * gq + 1], wg8[3 * gq + 2]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int kk = 8 * gq + q;
+              uint32_t a0, a1, a2, a3;
+              lut4(lut, quad_selector(sa, q), a0, a2);
+              lut4(lut, quad_selector(sb, q), a1, a3);
+              mma_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+              if (!QIN) mma_16816(sc, a0, a1, a2, a3, qflo[QIN ? 0 : kk][0], qflo[QIN ? 0 : kk][1]);
+            }
           }
         }
         if (QIN) {
@@ -348,21 +355,18 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
         const uint32_t u01 = pack_half2(p0 * svg, p1 * svg);      // token g, heads 2t, 2t+1
         const uint32_t u23 = pack_half2(p2 * svg8, p3 * svg8);    // token g+8
 
-        // ---- PV: unpack this lane's 4 tokens once, reuse for the N tiles ----
-        constexpr int VB = C::VSEG * 3 / 8;     // bytes per token segment (6 or 12)
-        constexpr int NWV = (VB + 3) / 4 + 1;   // words loaded per token (room for alignment)
-        uint32_t w[4][NWV];
+        // ---- PV: this lane's 4 tokens, one 32-code group each (d=256) or
+        // half a group (d=128: lanes 2m, 2m+1 share group m) ----
+        GroupSel vs[4];
         {
-          const int off = g * VB;
-          const int off4 = off & ~3, sh = (off & 3) * 8;
+          const int goff = (D == 256 ? g : (g >> 1)) * 12;
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const unsigned char *row = vc + (t + 4 * r) * C::PB + off4;
-#pragma unroll
-            for (int k = 0; k < NWV; ++k) w[r][k] = (4 * k < VB + (off & 3)) ? lds32(row + 4 * k) : 0u;
-            if (sh) {
-#pragma unroll
-              for (int k = 0; k + 1 < NWV; ++k) w[r][k] = __funnelshift_r(w[r][k], w[r][k + 1], sh);
+            const unsigned char *row = vc + (t + 4 * r) * C::PB + goff;
+            vs[r] = group_selectors(lds32(row), lds32(row + 4), lds32(row + 8));
+            if (D == 128 && (g & 1)) {   // codes 16..31 of the group
+              vs[r].m0 = vs[r].m2;
+              vs[r].m1 = vs[r].e;
             }
           }
         }
@@ -386,23 +390,16 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
           pb[nt][3] = live ? prmt(x_t12, 0u, sel) : 0u;
         }
 #pragma unroll
-        for (int grp = 0; grp < C::VSEG / 8; ++grp) {
-          uint32_t n4[4];
+        for (int mb = 0; mb < C::MB; ++mb) {          // M-block mb = codes 4mb..4mb+3
+          uint32_t ta0, ta1, tb0, tb1, tc0, tc1, td0, td1;
+          lut4(lut, quad_selector(vs[0], mb), ta0, ta1);   // token t
+          lut4(lut, quad_selector(vs[1], mb), tb0, tb1);   // token t+4
+          lut4(lut, quad_selector(vs[2], mb), tc0, tc1);   // token t+8
+          lut4(lut, quad_selector(vs[3], mb), td0, td1);   // token t+12
 #pragma unroll
-          for (int r = 0; r < 4; ++r) n4[r] = spread3_to_nibbles(group24(w[r], grp));
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {      // codes 0-3, then 4-7: M-block 2grp + half
-            const int mb = 2 * grp + half;
-            uint32_t ta0, ta1, tb0, tb1, tc0, tc1, td0, td1;
-            lut4(lut, n4[0] >> (16 * half), ta0, ta1);   // token t
-            lut4(lut, n4[1] >> (16 * half), tb0, tb1);   // token t+4
-            lut4(lut, n4[2] >> (16 * half), tc0, tc1);   // token t+8
-            lut4(lut, n4[3] >> (16 * half), td0, td1);   // token t+12
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              mma_16816(acc[nt][mb], ta0, ta1, tb0, tb1, pb[nt][0], pb[nt][1]);
-              mma_16816(acc[nt][mb], tc0, tc1, td0, td1, pb[nt][2], pb[nt][3]);
-            }
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_16816(acc[nt][mb], ta0, ta1, tb0, tb1, pb[nt][0], pb[nt][1]);
+            mma_16816(acc[nt][mb], tc0, tc1, td0, td1, pb[nt][2], pb[nt][3]);
           }
         }
       }

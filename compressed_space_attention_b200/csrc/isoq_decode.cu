@@ -118,14 +118,24 @@ __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <>
 __device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
 
-// Code of dimension i from a packed row read as 32-bit words.
+// Code of dimension i from a packed row read as 32-bit words (layout in
+// common.cuh).
 template <int BITS>
 __device__ __forceinline__ uint32_t code_at(const uint32_t *row, int i) {
-  const int bp = BITS * i;
-  const uint32_t lo = __ldg(row + (bp >> 5));
-  uint32_t c = lo >> (bp & 31);
-  if ((bp & 31) + BITS > 32) c |= __ldg(row + (bp >> 5) + 1) << (32 - (bp & 31));
-  return c & ((1u << BITS) - 1u);
+  if constexpr (BITS == 3) {
+    const int grp = i >> 5, m = i & 31;
+    const uint32_t *gw = row + 3 * grp;
+    if (m < 24) return (__ldg(gw + (m >> 3)) >> (4 * (m & 7))) & 7u;
+    const int sh = 4 * (m - 24) + 3;
+    return ((__ldg(gw) >> sh) & 1u) | (((__ldg(gw + 1) >> sh) & 1u) << 1) |
+           (((__ldg(gw + 2) >> sh) & 1u) << 2);
+  } else {
+    const int bp = BITS * i;
+    const uint32_t lo = __ldg(row + (bp >> 5));
+    uint32_t c = lo >> (bp & 31);
+    if ((bp & 31) + BITS > 32) c |= __ldg(row + (bp >> 5) + 1) << (32 - (bp & 31));
+    return c & ((1u << BITS) - 1u);
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -313,10 +313,8 @@ __global__ void __launch_bounds__(kQuantThreads)
       for (int j = 0; j < C::NPOS; ++j) m += (a > ts[j]) ? 1 : 0;
       const uint32_t code = (y > 0.f) ? static_cast<uint32_t>(C::L / 2 + m)
                                       : static_cast<uint32_t>(C::L / 2 - 1 - m);
-      // Step 4: LSB-first bit-pack.
-      const int bp = BITS * i;
-      w[bp >> 5] |= code << (bp & 31);
-      if ((bp & 31) + BITS > 32) w[(bp >> 5) + 1] |= code >> (32 - (bp & 31));
+      // Step 4: bit-pack (layout in common.cuh).
+      pack_code<BITS>(w, i, code);
     }
 
     if (v < args.n_vec) {
@@ -406,12 +404,7 @@ __global__ void __launch_bounds__(kDequantThreads) dequantize_kernel(const Dequa
 
     float x[kE];
 #pragma unroll
-    for (int i = 0; i < kE; ++i) {
-      const int bp = BITS * i;
-      uint32_t code = w[bp >> 5] >> (bp & 31);
-      if ((bp & 31) + BITS > 32) code |= w[(bp >> 5) + 1] << (32 - (bp & 31));
-      x[i] = cent[code & (L - 1)];
-    }
+    for (int i = 0; i < kE; ++i) x[i] = cent[unpack_code<BITS>(w, i)];
     apply_block_matrices(x, mat + part * (kE / 4) * 16);
     wht_inlane_h4_to_32(x);
     wht_crosslane<P, VPW>(x, part);

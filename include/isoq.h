@@ -24,9 +24,14 @@
  *    with the CUDA error text in isoq_last_error().
  *  - Rotation parameters are float32 arrays [n_heads][d/4][8]: for each
  *    4-dim block the unit quaternions q_L then q_R, each (w, x, y, z).
- *  - Packed codes: d*bits/8 bytes per vector, an LSB-first little-endian
- *    bitstream (code i at bits [bits*i, bits*i + bits)); norms are IEEE
- *    float16 bit patterns (uint16).
+ *  - Packed codes: d*bits/8 bytes per vector ([RQ] §3.2 Step 4; the pages
+ *    fix the size, not the bit order).  bits = 2, 4: an LSB-first
+ *    little-endian bitstream (code i at bits [bits*i, bits*i + bits)).
+ *    bits = 3: groups of 32 codes in 12 bytes, read as three little-endian
+ *    32-bit words w0, w1, w2: bits [4j, 4j+3) of w_r hold code 8r + j of the
+ *    group, and bit 4j + 3 of w_r holds bit r of code 24 + j, so that every
+ *    code sits in a 4-bit field.  Norms are IEEE float16 bit patterns
+ *    (uint16).
  *  - Supported: d in {128, 256, 512}, bits in {2, 3, 4}, variant
  *    ISOQ_FULL or ISOQ_FAST, element dtype ISOQ_F16 or ISOQ_F32.  Anything
  *    else returns ISOQ_ERR_UNSUPPORTED.

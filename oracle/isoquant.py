@@ -36,8 +36,10 @@ the repository's design notes):
     ``make_params``), rounded to float32.
   * Codebook: Lloyd-Max for N(0, 1/d), 2^b levels, the same for K and V and
     all heads; code = #{k : y > t_k} (ties go to the lower code).
-  * Bit-pack: LSB-first little-endian bitstream per vector, code i at bits
-    [b*i, b*i + b); vectors are contiguous with no padding.
+  * Bit-pack: b = 2, 4: LSB-first little-endian bitstream per vector, code
+    i at bits [b*i, b*i + b).  b = 3: 32-code groups of three little-endian
+    32-bit words; codes 32k+8r+j in bits [4j, 4j+3) of word r, bit r of code
+    32k+24+j in bit 4j+3 of word r.  Vectors are contiguous with no padding.
   * Scale: s = ||x||_2 is stored as float16 (round to nearest even); the
     vector is normalised by the unrounded s; dequantisation multiplies by the
     stored float16 s.  s = 0 gives x_hat = 0.
@@ -340,13 +342,7 @@ def packed_bytes(d: int, bits: int) -> int:
     return d * bits // 8
 
 
-def bitpack(codes, bits: int):
-    """BitPack_b ([RQ] Algorithm 1): LSB-first bitstream, code i at bit b*i.
-
-    codes: integer array [..., d]; returns uint8 [..., d*b/8].  Written bit by
-    bit: bit k of code i goes to stream position b*i + k, which is bit
-    (b*i + k) % 8 of byte (b*i + k) // 8.
-    """
+def _bitpack_lsb_first(codes, bits: int):
     codes = np.asarray(codes, dtype=np.int64)
     d = codes.shape[-1]
     out = np.zeros(codes.shape[:-1] + (packed_bytes(d, bits),), dtype=np.int64)
@@ -357,8 +353,7 @@ def bitpack(codes, bits: int):
     return out.astype(np.uint8)
 
 
-def bitunpack(packed, bits: int, d: int):
-    """Inverse of ``bitpack``: uint8 [..., d*b/8] -> int64 codes [..., d]."""
+def _bitunpack_lsb_first(packed, bits: int, d: int):
     packed = np.asarray(packed, dtype=np.int64)
     codes = np.zeros(packed.shape[:-1] + (d,), dtype=np.int64)
     for i in range(d):
@@ -366,6 +361,76 @@ def bitunpack(packed, bits: int, d: int):
             pos = bits * i + k
             codes[..., i] |= ((packed[..., pos // 8] >> (pos % 8)) & 1) << k
     return codes
+
+
+def _words_to_bytes(words):
+    """Little-endian bytes of a list of 32-bit word arrays."""
+    out = []
+    for w in words:
+        for byte in range(4):
+            out.append((w >> (8 * byte)) & 0xFF)
+    return np.stack(out, axis=-1)
+
+
+def _bitpack3_groups(codes):
+    """BitPack_3 in 32-code groups of three little-endian 32-bit words.
+
+    Group k holds codes 32k .. 32k+31 at bytes 12k .. 12k+11 (words w0, w1,
+    w2).  For r in {0, 1, 2} and j in 0..7: bits [4j, 4j+3) of w_r hold code
+    32k + 8r + j, and bit 4j+3 of w_r holds bit r of code 32k + 24 + j.
+    """
+    codes = np.asarray(codes, dtype=np.int64)
+    d = codes.shape[-1]
+    if d % 32:
+        raise ValueError("3-bit packing needs d to be a multiple of 32")
+    groups = []
+    for k in range(d // 32):
+        words = [np.zeros(codes.shape[:-1], dtype=np.int64) for _ in range(3)]
+        for r in range(3):
+            for j in range(8):
+                words[r] |= (codes[..., 32 * k + 8 * r + j] & 7) << (4 * j)
+                words[r] |= ((codes[..., 32 * k + 24 + j] >> r) & 1) << (4 * j + 3)
+        groups.append(_words_to_bytes(words))
+    return np.concatenate(groups, axis=-1).astype(np.uint8)
+
+
+def _bitunpack3_groups(packed, d: int):
+    packed = np.asarray(packed, dtype=np.int64)
+    codes = np.zeros(packed.shape[:-1] + (d,), dtype=np.int64)
+    for k in range(d // 32):
+        words = []
+        for r in range(3):
+            base = 12 * k + 4 * r
+            words.append(packed[..., base] | (packed[..., base + 1] << 8) |
+                         (packed[..., base + 2] << 16) | (packed[..., base + 3] << 24))
+        for r in range(3):
+            for j in range(8):
+                codes[..., 32 * k + 8 * r + j] = (words[r] >> (4 * j)) & 7
+        for j in range(8):
+            codes[..., 32 * k + 24 + j] = sum(((words[r] >> (4 * j + 3)) & 1) << r for r in range(3))
+    return codes
+
+
+def bitpack(codes, bits: int):
+    """BitPack_b ([RQ] Algorithm 1): d codes of b bits in d*b/8 bytes.
+
+    b = 2 and b = 4: LSB-first bitstream, code i at bits [b*i, b*i + b)
+    (written bit by bit: bit k of code i goes to stream position b*i + k).
+    b = 3: 32-code groups of three 32-bit words (``_bitpack3_groups``), a bit
+    order chosen so that the codes sit in 4-bit fields.  The pages fix only
+    the size (48 bytes at d = 128); the order within a vector is a reading.
+    codes: integer array [..., d]; returns uint8 [..., d*b/8].
+    """
+    if bits == 3:
+        return _bitpack3_groups(codes)
+    return _bitpack_lsb_first(codes, bits)
+
+
+def bitunpack(packed, bits: int, d: int):
+    """Inverse of ``bitpack``: uint8 [..., d*b/8] -> int64 codes [..., d]."""
+    if bits == 3:
+        return _bitunpack3_groups(packed, d)
+    return _bitunpack_lsb_first(packed, bits, d)
 
 
 # ---------------------------------------------------------------------------

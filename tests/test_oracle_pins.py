@@ -336,7 +336,7 @@ def test_one_bit_closed_form_and_scaling():
 
 def _read_bitpack_golden():
     rows = []
-    with open(os.path.join(GOLDEN, "bitpack_lsb_first.txt")) as f:
+    with open(os.path.join(GOLDEN, "bitpack_examples.txt")) as f:
         for line in f:
             if line.startswith("#") or not line.strip():
                 continue
@@ -363,9 +363,20 @@ def test_bitpack_roundtrip_and_size(bits, d):
     packed = O.bitpack(codes, bits)
     assert packed.shape == (7, d * bits // 8)
     np.testing.assert_array_equal(O.bitunpack(packed, bits, d), codes)
-    # LSB-first as one little-endian integer per vector
-    as_int = int.from_bytes(bytes(packed[0]), "little")
-    assert as_int == sum(int(c) << (bits * i) for i, c in enumerate(codes[0]))
+    if bits != 3:
+        # LSB-first as one little-endian integer per vector
+        as_int = int.from_bytes(bytes(packed[0]), "little")
+        assert as_int == sum(int(c) << (bits * i) for i, c in enumerate(codes[0]))
+    else:
+        # 32-code groups of three words: code 32k+8r+j in nibble j of word
+        # 3k+r (low 3 bits); bit r of code 32k+24+j in bit 3 of that nibble
+        words = np.frombuffer(bytes(packed[0]), dtype="<u4").astype(np.int64)
+        for k in range(d // 32):
+            for r in range(3):
+                for j in range(8):
+                    nib = (words[3 * k + r] >> (4 * j)) & 15
+                    assert nib & 7 == codes[0, 32 * k + 8 * r + j]
+                    assert nib >> 3 == (codes[0, 32 * k + 24 + j] >> r) & 1
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4])
