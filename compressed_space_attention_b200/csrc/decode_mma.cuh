@@ -2,11 +2,13 @@
 // 3-bit codes, d in {128, 256}, up to 8 query heads per KV head.
 // Included by isoq_decode.cu inside namespace isoq::decode.
 //
-// Per CTA: one (b, kvh, token chunk).  One producer warp streams the chunk's
-// packed K/V rows and float16 norms into shared memory with CTA-local bulk
-// copies (64 tokens per stage, an mbarrier ring) from the first cycle on;
-// four consumer warps rotate the queries, then each takes a 16-token slab of
-// every stage.
+// Per CTA: one (b, kvh, token chunk) and all G query heads of the KV head.
+// The chunk is cut into 16-token slabs; warp w takes slabs w, w+4, w+8, ...
+// and streams them through its own 3-deep ring of shared-memory stages with
+// CTA-local bulk copies (packed K/V rows and float16 norms; mbarrier
+// completion), issuing the copy for slab i+3 as soon as it is done with slab
+// i.  There is no producer warp and no cross-warp handshake until the final
+// merge, so four CTAs (16 warps) fit on an SM.
 //
 // QK (RotaryQuant Table 2 kernel A): mma.sync m16n8k16, A = K~ [16 tokens x
 // 16 dims] expanded from the codes in registers, B = q~ [16 dims x 8 columns].
@@ -37,24 +39,26 @@
 // The centroids are scaled by a host-chosen alpha that makes all of them
 // nearly exact in float16; alpha is divided out of the scores and the output.
 
-constexpr int kMmaConsumerWarps = 4;
-constexpr int kMmaThreads = 32 * (kMmaConsumerWarps + 1);
-constexpr int kMmaStageTokens = 16 * kMmaConsumerWarps;
-constexpr int kMmaStages = 4;
+constexpr int kMmaWarps = 4;
+constexpr int kMmaThreads = 32 * kMmaWarps;
+constexpr int kSlab = 16;          // tokens per slab (the M of one QK tile)
+constexpr int kWarpStages = 3;     // per-warp ring depth
+constexpr int kChunkQuantum = kSlab * kMmaWarps;
 
 template <int D>
 struct MmaCfg {
   static constexpr int PB = D * 3 / 8;                      // packed bytes per token
-  static constexpr int CODES_BYTES = kMmaStageTokens * PB;
-  static constexpr int NORM_BYTES = kMmaStageTokens * 2;
-  static constexpr int STAGE_BYTES = 2 * CODES_BYTES + 2 * NORM_BYTES;
+  static constexpr int SLAB_CODES = kSlab * PB;
+  static constexpr int SLAB_NORMS = kSlab * 2;
+  static constexpr int STAGE_BYTES = 2 * SLAB_CODES + 2 * SLAB_NORMS;
+  static constexpr int RING_BYTES = kWarpStages * STAGE_BYTES;
   static constexpr int KK = D / 16;                         // QK MMAs along d
   static constexpr int QSEG = D / 4;                        // dims per lane in QK
   static constexpr int VSEG = D / 8;                        // dims per lane in PV
   static constexpr int MB = D / 32;                         // PV M-blocks
   static constexpr int SCRATCH_FLOATS = 8 * D;              // q~ staging, then the warp merge
-  static constexpr int SMEM = kMmaStages * STAGE_BYTES + SCRATCH_FLOATS * 4 +
-                              2 * kMmaConsumerWarps * 8 * 4 + 2 * kMmaStages * 8 + 16 + 128;
+  static constexpr int SMEM = kMmaWarps * RING_BYTES + SCRATCH_FLOATS * 4 +
+                              2 * kMmaWarps * 8 * 4 + kMmaWarps * kWarpStages * 8 + 128;
 };
 
 struct MmaLut {
@@ -110,6 +114,10 @@ __device__ __forceinline__ uint32_t lds32(const unsigned char *p) {
   return *reinterpret_cast<const uint32_t *>(p);
 }
 
+__device__ __forceinline__ uint2 lds64(const unsigned char *p) {
+  return *reinterpret_cast<const uint2 *>(p);
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
@@ -118,23 +126,22 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 // QIN: q~'s lo parts ride in the spare B columns (G in {1, 2, 4}).
 // NT:  number of 4-head N tiles of the PV product (1 for G <= 4, else 2).
 template <int D, bool FULL, bool QIN, int NT>
-__global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs a, const MmaLut lut,
-                                                                float qk_scale_log2, float out_scale) {
+__global__ void __launch_bounds__(kMmaThreads, D == 256 && NT == 2 ? 2 : (D == 256 && !QIN ? 3 : 4))
+    split_mma_kernel(const SplitArgs a, const MmaLut lut,
+                                                                   float qk_scale_log2, float out_scale) {
   using C = MmaCfg<D>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
-  unsigned char *stages = smem;
-  float *scratch = reinterpret_cast<float *>(smem + kMmaStages * C::STAGE_BYTES);
-  float *wm = scratch + C::SCRATCH_FLOATS;          // [warps][8]
-  float *wl = wm + kMmaConsumerWarps * 8;           // [warps][8]
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(wl + kMmaConsumerWarps * 8);
-  uint64_t *empty_bar = full_bar + kMmaStages;
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty_bar + kMmaStages);
-
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.group;
+
+  unsigned char *ring = smem + warp * C::RING_BYTES;
+  float *scratch = reinterpret_cast<float *>(smem + kMmaWarps * C::RING_BYTES);
+  float *wm = scratch + C::SCRATCH_FLOATS;          // [warps][8]
+  float *wl = wm + kMmaWarps * 8;                   // [warps][8]
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(wl + kMmaWarps * 8) + warp * kWarpStages;
 
   int tlen = a.seq_lens[b];
   tlen = tlen < 0 ? 0 : (tlen > a.tmax ? static_cast<int>(a.tmax) : tlen);
@@ -142,130 +149,113 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
   long long t1 = t0 + a.chunk;
   if (t1 > tlen) t1 = tlen;
   const int n_tok = t1 > t0 ? static_cast<int>(t1 - t0) : 0;
-  const int n_stages = (n_tok + kMmaStageTokens - 1) / kMmaStageTokens;
-
-  if (tid == 0) {
-    for (int s = 0; s < kMmaStages; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kMmaConsumerWarps);
-    }
-    *abort_flag = 0;
-    mbar_fence_init();
-  }
-  __syncthreads();
+  const int n_slabs = (n_tok + kSlab - 1) / kSlab;
+  const int n_mine = n_slabs > warp ? (n_slabs - warp + kMmaWarps - 1) / kMmaWarps : 0;
 
   const long long pair = static_cast<long long>(b) * a.hkv + kvh;
-  constexpr int kConsumers = 32 * kMmaConsumerWarps;
+  const uint8_t *kb = a.packed_k + pair * a.tmax * C::PB;
+  const uint8_t *vb = a.packed_v + pair * a.tmax * C::PB;
+  const uint16_t *nkb = a.norms_k + pair * a.tmax;
+  const uint16_t *nvb = a.norms_v + pair * a.tmax;
 
-  if (warp == kMmaConsumerWarps) {
-    // ---------------- bulk-copy producer ----------------
-    if (lane == 0) {
-      const uint8_t *kb = a.packed_k + pair * a.tmax * C::PB;
-      const uint8_t *vb = a.packed_v + pair * a.tmax * C::PB;
-      const uint16_t *nkb = a.norms_k + pair * a.tmax;
-      const uint16_t *nvb = a.norms_v + pair * a.tmax;
-      int issued = 0;
-      for (int i = 0; i < n_stages; ++i) {
-        const int s = i % kMmaStages;
-        if (!mbar_wait_bounded(&empty_bar[s], ((i / kMmaStages) & 1) ^ 1) || *abort_flag) {
-          atomicOr(&g_decode_error, kErrWaitTimeout);
-          *abort_flag = 1;
-          break;
-        }
-        const long long t = t0 + static_cast<long long>(i) * kMmaStageTokens;
-        int n = n_tok - i * kMmaStageTokens;
-        if (n > kMmaStageTokens) n = kMmaStageTokens;
-        const int n8 = (n + 7) & ~7;
-        unsigned char *st = stages + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full_bar[s], 2u * n * C::PB + 4u * n8);
-        bulk_load(st, kb + t * C::PB, n * C::PB, &full_bar[s]);
-        bulk_load(st + C::CODES_BYTES, vb + t * C::PB, n * C::PB, &full_bar[s]);
-        bulk_load(st + 2 * C::CODES_BYTES, nkb + t, 2 * n8, &full_bar[s]);
-        bulk_load(st + 2 * C::CODES_BYTES + C::NORM_BYTES, nvb + t, 2 * n8, &full_bar[s]);
-        issued = i + 1;
+  // Lane 0 of each warp issues the copies of the warp's i-th slab into ring
+  // stage i % kWarpStages.
+  auto issue = [&](int i) {
+    const int j = warp + kMmaWarps * i;                 // slab index within the chunk
+    const long long t = t0 + static_cast<long long>(j) * kSlab;
+    int n = n_tok - j * kSlab;
+    if (n > kSlab) n = kSlab;
+    const int n8 = (n + 7) & ~7;
+    const int s = i % kWarpStages;
+    unsigned char *st = ring + s * C::STAGE_BYTES;
+    mbar_arrive_expect_tx(&full_bar[s], 2u * n * C::PB + 4u * n8);
+    bulk_load(st, kb + t * C::PB, n * C::PB, &full_bar[s]);
+    bulk_load(st + C::SLAB_CODES, vb + t * C::PB, n * C::PB, &full_bar[s]);
+    bulk_load(st + 2 * C::SLAB_CODES, nkb + t, 2 * n8, &full_bar[s]);
+    bulk_load(st + 2 * C::SLAB_CODES + C::SLAB_NORMS, nvb + t, 2 * n8, &full_bar[s]);
+  };
+  int issued = 0;
+  if (lane == 0) {
+    for (int s = 0; s < kWarpStages; ++s) mbar_init(&full_bar[s], 1);
+    mbar_fence_init();
+    for (; issued < kWarpStages && issued < n_mine; ++issued) issue(issued);
+  }
+
+  // Rotate the G queries of this KV head once, q~ = R_K q, while the first
+  // slabs stream in.
+  for (int i = tid; i < 8 * D; i += kMmaThreads) {
+    const int gq = i / D;
+    float v = 0.f;
+    if (gq < G) {
+      const __half *qp = static_cast<const __half *>(a.q) +
+                         (static_cast<long long>(b) * a.hq + kvh * G + gq) * D;
+      v = __half2float(qp[i % D]);
+    }
+    scratch[i] = v;
+  }
+  __syncthreads();
+  rotate_forward_smem<D, FULL>(scratch, G, a.params_k + static_cast<size_t>(kvh) * 2 * D, tid,
+                               kMmaThreads, 0);
+
+  const int g = lane >> 2, t = lane & 3;
+
+  // B fragments of q~ (hi + lo float16 parts) for QK: column g, dims
+  // t*QSEG + 4kk + {0..3}.
+  uint32_t qf[C::KK][2];
+  uint32_t qflo[QIN ? 1 : C::KK][2];
+  {
+    const int head = QIN ? (g < G ? g : g - G) : g;
+    const bool live = QIN ? (g < 2 * G) : (g < G);
+    const bool lo_col = QIN && g >= G;
+#pragma unroll
+    for (int kk = 0; kk < C::KK; ++kk) {
+      float v[4], hi[4], lo[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[j] = live ? scratch[head * D + t * C::QSEG + 4 * kk + j] : 0.f;
+        hi[j] = __half2float(__float2half_rn(v[j]));
+        lo[j] = v[j] - hi[j];
       }
-      // Wait for every issued copy before the CTA may exit.
-      for (int i = issued > kMmaStages ? issued - kMmaStages : 0; i < issued; ++i) {
-        if (!mbar_wait_bounded(&full_bar[i % kMmaStages], (i / kMmaStages) & 1)) {
-          atomicOr(&g_decode_error, kErrWaitTimeout);
-          break;
-        }
+      if (QIN) {
+        const float *src = lo_col ? lo : hi;
+        qf[kk][0] = pack_half2(src[0], src[1]);
+        qf[kk][1] = pack_half2(src[2], src[3]);
+      } else {
+        qf[kk][0] = pack_half2(hi[0], hi[1]);
+        qf[kk][1] = pack_half2(hi[2], hi[3]);
+        qflo[QIN ? 0 : kk][0] = pack_half2(lo[0], lo[1]);
+        qflo[QIN ? 0 : kk][1] = pack_half2(lo[2], lo[3]);
       }
     }
-  } else {
-    // ---------------- consumers ----------------
-    // Rotate the G queries of this KV head once, q~ = R_K q, while the
-    // producer already streams the first stages.
-    for (int i = tid; i < 8 * D; i += kConsumers) {
-      const int gq = i / D;
-      float v = 0.f;
-      if (gq < G) {
-        const __half *qp = static_cast<const __half *>(a.q) +
-                           (static_cast<long long>(b) * a.hq + kvh * G + gq) * D;
-        v = __half2float(qp[i % D]);
-      }
-      scratch[i] = v;
+  }
+
+  float acc[NT][C::MB][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int mb = 0; mb < C::MB; ++mb) acc[nt][mb][0] = acc[nt][mb][1] = acc[nt][mb][2] = acc[nt][mb][3] = 0.f;
+  // Online-softmax state in the QK layout: heads 2t, 2t+1 (log2 domain).
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const bool real0 = 2 * t < G, real1 = 2 * t + 1 < G;
+
+  int consumed = 0;
+  bool failed = false;
+  for (int i = 0; i < n_mine; ++i) {
+    const int s = i % kWarpStages;
+    if (!mbar_wait_bounded(&full_bar[s], (i / kWarpStages) & 1)) {
+      atomicOr(&g_decode_error, kErrWaitTimeout);
+      failed = true;
+      break;
     }
-    named_barrier(2, kConsumers);
-    rotate_forward_smem<D, FULL>(scratch, G, a.params_k + static_cast<size_t>(kvh) * 2 * D, tid,
-                                 kConsumers, 2);
-
-    const int g = lane >> 2, t = lane & 3;
-
-    // B fragments of q~ (hi + lo float16 parts) for QK: column g, dims
-    // t*QSEG + 4kk + {0..3}.
-    uint32_t qf[C::KK][2];
-    uint32_t qflo[QIN ? 1 : C::KK][2];
     {
-      const int head = QIN ? (g < G ? g : g - G) : g;
-      const bool live = QIN ? (g < 2 * G) : (g < G);
-      const bool lo_col = QIN && g >= G;
-#pragma unroll
-      for (int kk = 0; kk < C::KK; ++kk) {
-        float v[4], hi[4], lo[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          v[j] = live ? scratch[head * D + t * C::QSEG + 4 * kk + j] : 0.f;
-          hi[j] = __half2float(__float2half_rn(v[j]));
-          lo[j] = v[j] - hi[j];
-        }
-        if (QIN) {
-          const float *src = lo_col ? lo : hi;
-          qf[kk][0] = pack_half2(src[0], src[1]);
-          qf[kk][1] = pack_half2(src[2], src[3]);
-        } else {
-          qf[kk][0] = pack_half2(hi[0], hi[1]);
-          qf[kk][1] = pack_half2(hi[2], hi[3]);
-          qflo[QIN ? 0 : kk][0] = pack_half2(lo[0], lo[1]);
-          qflo[QIN ? 0 : kk][1] = pack_half2(lo[2], lo[3]);
-        }
-      }
-    }
-
-    float acc[NT][C::MB][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int mb = 0; mb < C::MB; ++mb) acc[nt][mb][0] = acc[nt][mb][1] = acc[nt][mb][2] = acc[nt][mb][3] = 0.f;
-    // Online-softmax state in the QK layout: heads 2t, 2t+1 (log2 domain).
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    const bool real0 = 2 * t < G, real1 = 2 * t + 1 < G;
-
-    for (int i = 0; i < n_stages; ++i) {
-      const int s = i % kMmaStages;
-      if (!mbar_wait_bounded(&full_bar[s], (i / kMmaStages) & 1) || *abort_flag) {
-        atomicOr(&g_decode_error, kErrWaitTimeout);
-        *abort_flag = 1;
-        break;
-      }
-      int nvalid = n_tok - i * kMmaStageTokens - 16 * warp;
-      nvalid = nvalid > 16 ? 16 : nvalid;
-      if (nvalid > 0) {
-        const unsigned char *st = stages + s * C::STAGE_BYTES;
-        const unsigned char *kc = st + (16 * warp) * C::PB;
-        const unsigned char *vc = st + C::CODES_BYTES + (16 * warp) * C::PB;
-        const __half *nk = reinterpret_cast<const __half *>(st + 2 * C::CODES_BYTES) + 16 * warp;
-        const __half *nv = reinterpret_cast<const __half *>(st + 2 * C::CODES_BYTES + C::NORM_BYTES) + 16 * warp;
+      int nvalid = n_tok - (warp + kMmaWarps * i) * kSlab;
+      nvalid = nvalid > kSlab ? kSlab : nvalid;
+      {
+        const unsigned char *st = ring + s * C::STAGE_BYTES;
+        const unsigned char *kc = st;
+        const unsigned char *vc = st + C::SLAB_CODES;
+        const __half *nk = reinterpret_cast<const __half *>(st + 2 * C::SLAB_CODES);
+        const __half *nv = reinterpret_cast<const __half *>(st + 2 * C::SLAB_CODES + C::SLAB_NORMS);
 
         // ---- QK: S[16 tokens x 8 columns] ----
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -274,10 +264,21 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
           uint32_t wg[NW], wg8[NW];
           const unsigned char *rg = kc + g * C::PB + t * (C::QSEG * 3 / 8);
           const unsigned char *rg8 = rg + 8 * C::PB;
+          if constexpr (NW % 2 == 0) {   // 8-byte aligned segments: 64-bit loads
 #pragma unroll
-          for (int k = 0; k < NW; ++k) {
-            wg[k] = lds32(rg + 4 * k);
-            wg8[k] = lds32(rg8 + 4 * k);
+            for (int k = 0; k < NW / 2; ++k) {
+              const uint2 x = lds64(rg + 8 * k), y = lds64(rg8 + 8 * k);
+              wg[2 * k] = x.x;
+              wg[2 * k + 1] = x.y;
+              wg8[2 * k] = y.x;
+              wg8[2 * k + 1] = y.y;
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < NW; ++k) {
+              wg[k] = lds32(rg + 4 * k);
+              wg8[k] = lds32(rg8 + 4 * k);
+            }
           }
 #pragma unroll
           for (int gq = 0; gq < C::QSEG / 32; ++gq) {
@@ -321,29 +322,28 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
           mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
           mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
         }
+        // Rescale unconditionally (the factors are 1 when the maximum holds):
+        // a few multiplies on the otherwise idle FMA pipe instead of a branch.
         const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        if (__any_sync(0xffffffffu, (mn0 > m0) || (mn1 > m1))) {
-          const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mn0);
-          const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mn1);
-          l0 *= f0;
-          l1 *= f1;
-          m0 = mn0;
-          m1 = mn1;
-          // The PV accumulator of lane (g, t) holds head nt*4 + t.
+        const float f0 = exp2f(m0 - mn0), f1 = exp2f(m1 - mn1);   // 0 on the first slab
+        l0 *= f0;
+        l1 *= f1;
+        m0 = mn0;
+        m1 = mn1;
+        // The PV accumulator of lane (g, t) holds head nt*4 + t.
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const int h = nt * 4 + t;
-            const int src = 4 * g + (h >> 1);
-            const float F0 = __shfl_sync(0xffffffffu, f0, src);
-            const float F1 = __shfl_sync(0xffffffffu, f1, src);
-            const float f = (h & 1) ? F1 : F0;
+        for (int nt = 0; nt < NT; ++nt) {
+          const int h = nt * 4 + t;
+          const int src = 4 * g + (h >> 1);
+          const float F0 = __shfl_sync(0xffffffffu, f0, src);
+          const float F1 = __shfl_sync(0xffffffffu, f1, src);
+          const float f = (h & 1) ? F1 : F0;
 #pragma unroll
-            for (int mb = 0; mb < C::MB; ++mb) {
-              acc[nt][mb][0] *= f;
-              acc[nt][mb][1] *= f;
-              acc[nt][mb][2] *= f;
-              acc[nt][mb][3] *= f;
-            }
+          for (int mb = 0; mb < C::MB; ++mb) {
+            acc[nt][mb][0] *= f;
+            acc[nt][mb][1] *= f;
+            acc[nt][mb][2] *= f;
+            acc[nt][mb][3] *= f;
           }
         }
         const float p0 = exp2f(x0 - m0), p1 = exp2f(x1 - m1);
@@ -403,36 +403,49 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
     }
+    __syncwarp();
+    consumed = i + 1;
+    // The warp is done reading stage s: refill it with the slab kWarpStages on.
+    if (lane == 0 && issued < n_mine) {
+      fence_proxy_async_smem();
+      issue(issued);
+      ++issued;
+    }
+  }
+  if (failed && lane == 0) {
+    // Let every copy still in flight land before the CTA may exit.
+    for (int k = consumed; k < issued; ++k)
+      if (!mbar_wait_bounded(&full_bar[k % kWarpStages], (k / kWarpStages) & 1)) break;
+  }
 
-    // Per-warp totals over the 8 lanes sharing t.
+  // Per-warp totals over the 8 lanes sharing t.
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    }
-    named_barrier(1, kConsumers);   // all warps are done with the q~ scratch
-    if (g == 0) {
-      wm[warp * 8 + 2 * t] = m0;
-      wm[warp * 8 + 2 * t + 1] = m1;
-      wl[warp * 8 + 2 * t] = l0;
-      wl[warp * 8 + 2 * t + 1] = l1;
-    }
-    named_barrier(1, kConsumers);
-    // Merge the warps' accumulators into scratch[head][dim] (rotated domain),
-    // one warp after the other so that the sum order is fixed.
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  __syncthreads();   // all warps are done with the q~ scratch
+  if (g == 0) {
+    wm[warp * 8 + 2 * t] = m0;
+    wm[warp * 8 + 2 * t + 1] = m1;
+    wl[warp * 8 + 2 * t] = l0;
+    wl[warp * 8 + 2 * t + 1] = l1;
+  }
+  __syncthreads();
+  // Merge the warps' accumulators into scratch[head][dim] (rotated domain),
+  // one warp after the other so that the sum order is fixed.
+  {
     float f[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int h = nt * 4 + t;
       float mstar = -INFINITY;
-      for (int w2 = 0; w2 < kMmaConsumerWarps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
+      for (int w2 = 0; w2 < kMmaWarps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
       const float mine = wm[warp * 8 + h];
       f[nt] = (mine == -INFINITY) ? 0.f : exp2f(mine - mstar);
     }
-    for (int w2 = 0; w2 < kMmaConsumerWarps; ++w2) {
+    for (int w2 = 0; w2 < kMmaWarps; ++w2) {
       if (warp == w2) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -450,10 +463,9 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
           }
         }
       }
-      named_barrier(1, kConsumers);
+      __syncthreads();
     }
   }
-  __syncthreads();
 
   // One partial state per query head: natural-log max, sum, acc (unscaled).
   for (int h = 0; h < G; ++h) {
@@ -462,8 +474,8 @@ __global__ void __launch_bounds__(kMmaThreads) split_mma_kernel(const SplitArgs 
     for (int i = tid; i < D; i += kMmaThreads) acc_out[i] = scratch[h * D + i] * out_scale;
     if (tid == 0) {
       float mstar = -INFINITY, l = 0.f;
-      for (int w2 = 0; w2 < kMmaConsumerWarps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
-      for (int w2 = 0; w2 < kMmaConsumerWarps; ++w2) {
+      for (int w2 = 0; w2 < kMmaWarps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
+      for (int w2 = 0; w2 < kMmaWarps; ++w2) {
         const float mw = wm[w2 * 8 + h];
         if (mw != -INFINITY) l += wl[w2 * 8 + h] * exp2f(mw - mstar);
       }
@@ -549,7 +561,7 @@ int launch_split_mma(const SplitArgs &a, cudaStream_t stream) {
 
 bool mma_path_supported(int dtype, int d, int bits, const SplitArgs &a) {
   return dtype == ISOQ_F16 && bits == 3 && (d == 128 || d == 256) && a.group <= 8 &&
-         a.tmax % 8 == 0 && a.chunk % kMmaStageTokens == 0 &&
+         a.tmax % 8 == 0 && a.chunk % kChunkQuantum == 0 &&
          (reinterpret_cast<uintptr_t>(a.norms_k) & 15u) == 0 &&
          (reinterpret_cast<uintptr_t>(a.norms_v) & 15u) == 0;
 }
