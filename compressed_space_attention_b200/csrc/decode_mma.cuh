@@ -110,12 +110,23 @@ __device__ __forceinline__ void lut4(const MmaLut &l, uint32_t sel, uint32_t &h0
   h23 = prmt(lo, hi, 0x7362u);
 }
 
+// Shared-memory loads by explicit shared-window address (no generic LD).
 __device__ __forceinline__ uint32_t lds32(const unsigned char *p) {
-  return *reinterpret_cast<const uint32_t *>(p);
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+  return v;
 }
 
 __device__ __forceinline__ uint2 lds64(const unsigned char *p) {
-  return *reinterpret_cast<const uint2 *>(p);
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
+  return v;
+}
+
+__device__ __forceinline__ float lds_half(const unsigned char *p) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_u32(p)));
+  return __half2float(__ushort_as_half(v));
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -254,8 +265,8 @@ __global__ void __launch_bounds__(kMmaThreads, D == 256 && NT == 2 ? 2 : (D == 2
         const unsigned char *st = ring + s * C::STAGE_BYTES;
         const unsigned char *kc = st;
         const unsigned char *vc = st + C::SLAB_CODES;
-        const __half *nk = reinterpret_cast<const __half *>(st + 2 * C::SLAB_CODES);
-        const __half *nv = reinterpret_cast<const __half *>(st + 2 * C::SLAB_CODES + C::SLAB_NORMS);
+        const unsigned char *nk = st + 2 * C::SLAB_CODES;                 // float16 [16]
+        const unsigned char *nv = st + 2 * C::SLAB_CODES + C::SLAB_NORMS;
 
         // ---- QK: S[16 tokens x 8 columns] ----
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -309,8 +320,8 @@ __global__ void __launch_bounds__(kMmaThreads, D == 256 && NT == 2 ? 2 : (D == 2
 
         // ---- online softmax on the fragments (log2 domain) ----
         const bool vg = g < nvalid, vg8 = g + 8 < nvalid;
-        const float skg = vg ? __half2float(nk[g]) * qk_scale_log2 : 0.f;
-        const float skg8 = vg8 ? __half2float(nk[g + 8]) * qk_scale_log2 : 0.f;
+        const float skg = vg ? lds_half(nk + 2 * g) * qk_scale_log2 : 0.f;
+        const float skg8 = vg8 ? lds_half(nk + 2 * (g + 8)) * qk_scale_log2 : 0.f;
         // Padded heads hold a constant 0 so that they never move the maximum.
         const float x0 = real0 ? (vg ? sc[0] * skg : -INFINITY) : 0.f;
         const float x1 = real1 ? (vg ? sc[1] * skg : -INFINITY) : 0.f;
@@ -350,8 +361,8 @@ __global__ void __launch_bounds__(kMmaThreads, D == 256 && NT == 2 ? 2 : (D == 2
         const float p2 = exp2f(x2 - m0), p3 = exp2f(x3 - m1);
         l0 += p0 + p2;
         l1 += p1 + p3;
-        const float svg = vg ? __half2float(nv[g]) : 0.f;
-        const float svg8 = vg8 ? __half2float(nv[g + 8]) : 0.f;
+        const float svg = vg ? lds_half(nv + 2 * g) : 0.f;
+        const float svg8 = vg8 ? lds_half(nv + 2 * (g + 8)) : 0.f;
         const uint32_t u01 = pack_half2(p0 * svg, p1 * svg);      // token g, heads 2t, 2t+1
         const uint32_t u23 = pack_half2(p2 * svg8, p3 * svg8);    // token g+8
 

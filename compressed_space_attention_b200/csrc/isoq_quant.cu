@@ -103,23 +103,30 @@ __device__ void build_block_matrices(const float *params_head, float *mat, int t
         m[3][c] = u.w - u.x - u.y + u.z;
       }
     }
-    float4 *out = reinterpret_cast<float4 *>(mat + 16 * b);
-    for (int r = 0; r < 4; ++r)
-      out[r] = make_float4(m[r][0] * inv_sqrt_d, m[r][1] * inv_sqrt_d, m[r][2] * inv_sqrt_d,
-                           m[r][3] * inv_sqrt_d);
+    // Pair order for the packed block product (see apply_block_matrices):
+    // (y0, y1) uses (M00,M11) (M01,M10) (M02,M13) (M03,M12) and
+    // (y2, y3) uses (M22,M33) (M23,M32) (M20,M31) (M21,M30).
+    const int order[16][2] = {{0, 0}, {1, 1}, {0, 1}, {1, 0}, {0, 2}, {1, 3}, {0, 3}, {1, 2},
+                              {2, 2}, {3, 3}, {2, 3}, {3, 2}, {2, 0}, {3, 1}, {2, 1}, {3, 0}};
+    float *out = mat + 16 * b;
+    for (int k = 0; k < 16; ++k) out[k] = m[order[k][0]][order[k][1]] * inv_sqrt_d;
   }
 }
 
-// In-lane Walsh-Hadamard butterflies for the strides 4 <= h < 64.
-__device__ __forceinline__ void wht_inlane_h4_to_32(float (&x)[kE]) {
+// The 64 elements of a lane are held as 32 packed float pairs
+// xp[k] = (x[2k], x[2k+1]).
+
+// In-lane Walsh-Hadamard butterflies for the strides 4 <= h < 64 (pair
+// strides 2..16): both elements of a pair move together.
+__device__ __forceinline__ void wht_inlane_h4_to_32(uint64_t (&xp)[kE / 2]) {
 #pragma unroll
-  for (int h = 4; h < kE; h <<= 1) {
+  for (int hp = 2; hp < kE / 2; hp <<= 1) {
 #pragma unroll
-    for (int i = 0; i < kE; ++i) {
-      if (!(i & h)) {
-        const float a = x[i], b = x[i + h];
-        x[i] = a + b;
-        x[i + h] = a - b;
+    for (int k = 0; k < kE / 2; ++k) {
+      if (!(k & hp)) {
+        const uint64_t a = xp[k], b = xp[k + hp];
+        xp[k] = f2_add(a, b);
+        xp[k + hp] = f2_sub(a, b);
       }
     }
   }
@@ -128,29 +135,40 @@ __device__ __forceinline__ void wht_inlane_h4_to_32(float (&x)[kE]) {
 // Cross-lane butterflies for h = 64, 128, ..., D/2: the partner part of a
 // vector sits VPW lanes away per doubling.
 template <int P, int VPW>
-__device__ __forceinline__ void wht_crosslane(float (&x)[kE], int part) {
+__device__ __forceinline__ void wht_crosslane(uint64_t (&xp)[kE / 2], int part) {
 #pragma unroll
   for (int k = 1; k < P; k <<= 1) {
     const float sgn = (part & k) ? -1.f : 1.f;
+    const uint64_t sgn2 = f2_pack(sgn, sgn);
 #pragma unroll
-    for (int i = 0; i < kE; ++i) {
-      const float o = __shfl_xor_sync(0xffffffffu, x[i], k * VPW);
-      x[i] = fmaf(sgn, x[i], o);
+    for (int i = 0; i < kE / 2; ++i) {
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, xp[i], k * VPW);
+      xp[i] = f2_fma(sgn2, xp[i], o);
     }
   }
 }
 
 // Applies the 16 per-block 4x4 matrices of this lane's blocks, in place.
-__device__ __forceinline__ void apply_block_matrices(float (&x)[kE], const float *mat_lane) {
+// With z = (z0..z3), Z01 = (z0, z1), Z10 = (z1, z0) and so on:
+//   (y0, y1) = (M00,M11) Z01 + (M01,M10) Z10 + (M02,M13) Z23 + (M03,M12) Z32
+//   (y2, y3) = (M22,M33) Z23 + (M23,M32) Z32 + (M20,M31) Z01 + (M21,M30) Z10
+__device__ __forceinline__ void apply_block_matrices(uint64_t (&xp)[kE / 2], const float *mat_lane) {
 #pragma unroll
   for (int lb = 0; lb < kE / 4; ++lb) {
     const float4 *m = reinterpret_cast<const float4 *>(mat_lane + 16 * lb);
-    const float z0 = x[4 * lb], z1 = x[4 * lb + 1], z2 = x[4 * lb + 2], z3 = x[4 * lb + 3];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float4 row = m[r];
-      x[4 * lb + r] = fmaf(row.x, z0, fmaf(row.y, z1, fmaf(row.z, z2, row.w * z3)));
-    }
+    const float4 m0 = m[0], m1 = m[1], m2 = m[2], m3 = m[3];
+    const uint64_t z01 = xp[2 * lb], z23 = xp[2 * lb + 1];
+    const uint64_t z10 = f2_swap(z01), z32 = f2_swap(z23);
+    uint64_t y01 = f2_mul(f2_pack(m0.x, m0.y), z01);
+    y01 = f2_fma(f2_pack(m0.z, m0.w), z10, y01);
+    y01 = f2_fma(f2_pack(m1.x, m1.y), z23, y01);
+    y01 = f2_fma(f2_pack(m1.z, m1.w), z32, y01);
+    uint64_t y23 = f2_mul(f2_pack(m2.x, m2.y), z23);
+    y23 = f2_fma(f2_pack(m2.z, m2.w), z32, y23);
+    y23 = f2_fma(f2_pack(m3.x, m3.y), z01, y23);
+    y23 = f2_fma(f2_pack(m3.z, m3.w), z10, y23);
+    xp[2 * lb] = y01;
+    xp[2 * lb + 1] = y23;
   }
 }
 
@@ -251,8 +269,8 @@ __global__ void __launch_bounds__(kQuantThreads)
       return;
     }
 
-    // Load this lane's 64 elements from the swizzled tile.
-    float x[kE];
+    // Load this lane's 64 elements from the swizzled tile as float pairs.
+    uint64_t xp[kE / 2];
     const unsigned char *stage = stages + s * C::STAGE_BYTES;
     if constexpr (C::ES == 2) {
       const unsigned char *box = stage + part * C::BOX_BYTES + vt * 128;
@@ -263,8 +281,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f = __half22float2(h[j]);
-          x[8 * c + 2 * j] = f.x;
-          x[8 * c + 2 * j + 1] = f.y;
+          xp[4 * c + j] = f2_pack(f.x, f.y);
         }
       }
     } else {
@@ -274,10 +291,8 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const float4 f = *reinterpret_cast<const float4 *>(box + ((c ^ (vt & 7)) << 4));
-          x[32 * bx + 4 * c] = f.x;
-          x[32 * bx + 4 * c + 1] = f.y;
-          x[32 * bx + 4 * c + 2] = f.z;
-          x[32 * bx + 4 * c + 3] = f.w;
+          xp[16 * bx + 2 * c] = f2_pack(f.x, f.y);
+          xp[16 * bx + 2 * c + 1] = f2_pack(f.z, f.w);
         }
       }
     }
@@ -285,17 +300,23 @@ __global__ void __launch_bounds__(kQuantThreads)
     if (lane == 0) mbar_arrive(&empty_bar[s]);  // the stage may be refilled
 
     // Step 1: norm (float32 accumulation, reduced over the P lanes).
-    float ss = 0.f;
+    uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < kE; ++i) ss = fmaf(x[i], x[i], ss);
+    for (int k = 0; k < kE / 2; ++k) acc2 = f2_fma(xp[k], xp[k], acc2);
+    float ss_lo, ss_hi;
+    f2_unpack(acc2, ss_lo, ss_hi);
+    float ss = ss_lo + ss_hi;
 #pragma unroll
     for (int k = 1; k < P; k <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, k * VPW);
     const float norm = sqrtf(ss);
 
     // Step 2: WHT stages h >= 4, then the folded (H_4, SO(4), 1/sqrt d) blocks.
-    wht_inlane_h4_to_32(x);
-    wht_crosslane<P, VPW>(x, part);
-    apply_block_matrices(x, mat + part * (kE / 4) * 16);
+    wht_inlane_h4_to_32(xp);
+    wht_crosslane<P, VPW>(xp, part);
+    apply_block_matrices(xp, mat + part * (kE / 4) * 16);
+    float x[kE];
+#pragma unroll
+    for (int k = 0; k < kE / 2; ++k) f2_unpack(xp[k], x[2 * k], x[2 * k + 1]);
 
     // Step 3: Lloyd-Max codes against thresholds scaled by the norm.
     float ts[C::NPOS > 0 ? C::NPOS : 1];
@@ -402,12 +423,19 @@ __global__ void __launch_bounds__(kDequantThreads) dequantize_kernel(const Dequa
     }
     const float s16 = __half2float(__ushort_as_half(args.norms[idx]));
 
+    uint64_t xp[kE / 2];
+#pragma unroll
+    for (int k = 0; k < kE / 2; ++k)
+      xp[k] = f2_pack(cent[unpack_code<BITS>(w, 2 * k)], cent[unpack_code<BITS>(w, 2 * k + 1)]);
+    apply_block_matrices(xp, mat + part * (kE / 4) * 16);
+    wht_inlane_h4_to_32(xp);
+    wht_crosslane<P, VPW>(xp, part);
+    const uint64_t s2 = f2_pack(s16, s16);
+#pragma unroll
+    for (int k = 0; k < kE / 2; ++k) xp[k] = f2_mul(xp[k], s2);
     float x[kE];
 #pragma unroll
-    for (int i = 0; i < kE; ++i) x[i] = cent[unpack_code<BITS>(w, i)];
-    apply_block_matrices(x, mat + part * (kE / 4) * 16);
-    wht_inlane_h4_to_32(x);
-    wht_crosslane<P, VPW>(x, part);
+    for (int k = 0; k < kE / 2; ++k) f2_unpack(xp[k], x[2 * k], x[2 * k + 1]);
 
     if (valid) {
       T *dst = static_cast<T *>(args.out) + static_cast<long long>(head) * args.head_stride +
@@ -419,14 +447,14 @@ __global__ void __launch_bounds__(kDequantThreads) dequantize_kernel(const Dequa
           __half2 *h = reinterpret_cast<__half2 *>(&u);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            h[j] = __floats2half2_rn(x[8 * c + 2 * j] * s16, x[8 * c + 2 * j + 1] * s16);
+            h[j] = __floats2half2_rn(x[8 * c + 2 * j], x[8 * c + 2 * j + 1]);
           reinterpret_cast<uint4 *>(dst)[c] = u;
         }
       } else {
 #pragma unroll
         for (int c = 0; c < kE / 4; ++c)
-          reinterpret_cast<float4 *>(dst)[c] = make_float4(x[4 * c] * s16, x[4 * c + 1] * s16,
-                                                           x[4 * c + 2] * s16, x[4 * c + 3] * s16);
+          reinterpret_cast<float4 *>(dst)[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2],
+                                                           x[4 * c + 3]);
       }
     }
   }
