@@ -8,21 +8,38 @@
 //   x = s16 * H_d(R_SO4^T c[codes]) / sqrt d.
 //
 // Mapping.  A vector of d elements is held by P = d/64 lanes of one warp,
-// 64 consecutive elements per lane, in registers.  The Walsh-Hadamard stages
-// with h >= 4 run as butterflies (in-lane for h < 64, by warp shuffle for
-// h >= 64).  The stages h = 1, 2 act inside each 4-block and commute with the
-// others, so they are folded into one 4x4 matrix per block together with the
-// SO(4) map and the 1/sqrt(d) normalisation:
-//   quantize:   M_i = R_i H_4 / sqrt(d)   applied after the h >= 4 stages,
+// 64 elements per lane, as two groups of 32 (the 32-code groups of the packed
+// layout).  Inside a group the elements are held as 16 packed float pairs
+// (e, e + 16), so every butterfly or block product that acts on whole pairs
+// is one f32x2 instruction for two elements.
+//
+// The Walsh-Hadamard stages commute, so they run in whatever order suits the
+// registers:
+//   h = 16       inside a pair (for float16 input, fused with the conversion),
+//   h = 4, 8     between pairs of a group,
+//   h = 32       between the two groups of a lane,
+//   h = 64 .. d/4  by warp shuffle, every pair exchanged,
+//   h = d/2      by a half exchange: each lane sends one group and keeps one,
+//                so the stage moves half the data of a full exchange.
+// The stages h = 1, 2 act inside each 4-block and are folded into one 4x4
+// matrix per block together with the SO(4) map and 1/sqrt(d):
+//   quantize:   M_i = R_i H_4 / sqrt(d)   applied after the other stages,
 //   dequantize: N_i = H_4 R_i^T / sqrt(d) applied before them.
+// The block pairs (i, i + 4) of a group share registers, so the matrices are
+// stored interleaved (M_i[j][c], M_{i+4}[j][c]).
+//
+// After the half exchange, the lane whose part has the exchange bit clear
+// holds the lower 32 elements of its own 64 and of its partner's, and the
+// lane with the bit set holds the upper 32 of both, the latter negated; the
+// negation is folded into that group's block matrices.
+//
 // The quantiser compares the unnormalised R x with s * t_k (no division per
 // element) using the symmetry of the codebook: the sign picks the half, and
 // the magnitude is counted against the positive thresholds.
 //
-// Data movement.  quantize stages its input through 128B-swizzled TMA tiles
-// (one producer warp, four consumer warps, an mbarrier ring); each lane then
-// reads its own 128-byte row segments conflict-free.  Outputs are written with
-// 8/16-byte stores that cover whole sectors per warp.
+// Data movement.  Each warp of a quantize CTA streams its own rows through a
+// ring of 128B-swizzled TMA tiles (no producer warp); each lane reads its own
+// 128-byte row segments conflict-free.  Each lane writes whole 32-code groups.
 
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -42,29 +59,42 @@ namespace quant {
 using namespace isoq::dev;
 
 constexpr int kE = 64;              // elements per lane
-constexpr int kConsumerWarps = 4;
-constexpr int kConsumers = 32 * kConsumerWarps;
-constexpr int kQuantThreads = kConsumers + 32;  // + one TMA producer warp
+constexpr int kPairs = kE / 2;      // packed pairs per lane
+constexpr int kGP = 16;             // packed pairs per 32-element group
+constexpr int kQuantWarps = 4;
+constexpr int kQuantThreads = 32 * kQuantWarps;
+constexpr int kDequantThreads = 128;
 
 __device__ unsigned int g_quant_error = 0;
 
+// Lane geometry shared by both directions.
+template <int D>
+struct Lanes {
+  static constexpr int P = D / kE;      // lanes per vector
+  static constexpr int VPW = 32 / P;    // vectors per warp
+  static constexpr int KH = P / 2;      // part bit of the half-exchange stage
+};
+
 template <typename T, int D, int BITS>
-struct Cfg {
-  static constexpr int P = D / kE;              // lanes per vector
-  static constexpr int VPW = 32 / P;            // vectors per warp
-  static constexpr int NV = kConsumers / P;     // vectors per tile
+struct Cfg : Lanes<D> {
+  using Lanes<D>::P;
+  using Lanes<D>::VPW;
+  static constexpr int NV = kQuantWarps * VPW;  // vectors per CTA tile
   static constexpr int ES = sizeof(T);
   static constexpr int BOX_ELEMS = 128 / ES;    // elements in one 128-byte box row
-  static constexpr int NBOX = D * ES / 128;     // boxes per tile
-  static constexpr int BOX_BYTES = NV * 128;
-  static constexpr int STAGE_BYTES = NBOX * BOX_BYTES;
-  static constexpr int STAGES = ES == 2 ? 4 : 3;
+  static constexpr int NBOX = D * ES / 128;     // boxes per row
+  static constexpr int BOX_BYTES = VPW * 128;   // one warp's rows of one box
+  // 128B-swizzled boxes start on 1024-byte boundaries.
+  static constexpr int BOX_STRIDE = BOX_BYTES < 1024 ? 1024 : BOX_BYTES;
+  static constexpr int STAGE_BYTES = NBOX * BOX_STRIDE;
+  static constexpr int STAGES = STAGE_BYTES >= 8192 ? 2 : 3;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int L = 1 << BITS;
   static constexpr int NPOS = L / 2 - 1;        // positive thresholds
   static constexpr int PB = D * BITS / 8;       // packed bytes per vector
-  static constexpr int TB = kE * BITS / 8;      // packed bytes per lane
-  static constexpr int MAT_BYTES = (D / 4) * 16 * 4;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + MAT_BYTES + 2 * STAGES * 8 + 16 + 1024;
+  static constexpr int GB = 32 * BITS / 8;      // packed bytes per 32-code group
+  static constexpr int MAT_BYTES = D * 16;      // D/4 blocks of 16 floats
+  static constexpr int SMEM = kQuantWarps * RING_BYTES + MAT_BYTES + kQuantWarps * STAGES * 8 + 1024;
 };
 
 struct QuantArgs {
@@ -79,8 +109,46 @@ struct QuantArgs {
   float tau[7];             // positive thresholds t_{L/2}, ..., t_{L-2}
 };
 
-// Builds the per-block 4x4 matrices of one head into shared memory, row-major.
-// forward: M_i = R_i H_4 / sqrt(d); inverse: N_i = H_4 R_i^T / sqrt(d).
+// ---------------------------------------------------------------------------
+// Register-level pieces
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void lds2x64(uint32_t addr, uint64_t &a, uint64_t &b) {
+  asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr));
+}
+
+// Groups of the final layout held by a lane (see the file comment): g[0] and
+// g[1] are 32-element group indices within the vector.
+template <int D>
+__device__ __forceinline__ void lane_groups(int part, int (&g)[2]) {
+  constexpr int KH = Lanes<D>::KH;
+  if (part & KH) {
+    g[0] = 2 * (part - KH) + 1;
+    g[1] = 2 * part + 1;
+  } else {
+    g[0] = 2 * part;
+    g[1] = 2 * (part + KH);
+  }
+}
+
+// True for the groups a lane holds negated after the half exchange.
+template <int D>
+__host__ __device__ constexpr bool group_negated(int g) {
+  return (g & 1) && (((g >> 1) & Lanes<D>::KH) != 0);
+}
+
+// Per-block 4x4 matrices of one head, stored for the packed product:
+// group g, block pair beta (blocks 8g + beta and 8g + beta + 4), entry
+// (j, c) -> float pair at mat[128 g + 32 beta + 2 (4 j + c) + {0, 1}].
+//   forward: M_i = R_i H_4 / sqrt(d); inverse: N_i = H_4 R_i^T / sqrt(d).
 template <int D, bool FULL, bool FORWARD>
 __device__ void build_block_matrices(const float *params_head, float *mat, int tid, int nthreads) {
   const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
@@ -103,26 +171,41 @@ __device__ void build_block_matrices(const float *params_head, float *mat, int t
         m[3][c] = u.w - u.x - u.y + u.z;
       }
     }
-    // Pair order for the packed block product (see apply_block_matrices):
-    // (y0, y1) uses (M00,M11) (M01,M10) (M02,M13) (M03,M12) and
-    // (y2, y3) uses (M22,M33) (M23,M32) (M20,M31) (M21,M30).
-    const int order[16][2] = {{0, 0}, {1, 1}, {0, 1}, {1, 0}, {0, 2}, {1, 3}, {0, 3}, {1, 2},
-                              {2, 2}, {3, 3}, {2, 3}, {3, 2}, {2, 0}, {3, 1}, {2, 1}, {3, 0}};
-    float *out = mat + 16 * b;
-    for (int k = 0; k < 16; ++k) out[k] = m[order[k][0]][order[k][1]] * inv_sqrt_d;
+    const int g = b >> 3, r = b & 7, beta = r & 3, half = r >> 2;
+    const float sc = group_negated<D>(g) ? -inv_sqrt_d : inv_sqrt_d;
+    float *out = mat + 128 * g + 32 * beta + half;
+    for (int j = 0; j < 4; ++j)
+      for (int c = 0; c < 4; ++c) out[2 * (4 * j + c)] = m[j][c] * sc;
   }
 }
 
-// The 64 elements of a lane are held as 32 packed float pairs
-// xp[k] = (x[2k], x[2k+1]).
+// Applies the block matrices of one group (16 pairs starting at xp[base]).
+__device__ __forceinline__ void apply_group_matrices(uint64_t (&xp)[kPairs], int base, uint32_t mat_g) {
+#pragma unroll
+  for (int beta = 0; beta < 4; ++beta) {
+    const uint64_t z0 = xp[base + 4 * beta], z1 = xp[base + 4 * beta + 1];
+    const uint64_t z2 = xp[base + 4 * beta + 2], z3 = xp[base + 4 * beta + 3];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint64_t m0, m1, m2, m3;
+      lds2x64(mat_g + 128 * beta + 32 * j, m0, m1);
+      lds2x64(mat_g + 128 * beta + 32 * j + 16, m2, m3);
+      uint64_t y = f2_mul(m0, z0);
+      y = f2_fma(m1, z1, y);
+      y = f2_fma(m2, z2, y);
+      y = f2_fma(m3, z3, y);
+      xp[base + 4 * beta + j] = y;
+    }
+  }
+}
 
-// In-lane Walsh-Hadamard butterflies for the strides 4 <= h < 64 (pair
-// strides 2..16): both elements of a pair move together.
-__device__ __forceinline__ void wht_inlane_h4_to_32(uint64_t (&xp)[kE / 2]) {
+// Butterflies between pairs of each group, strides h = 4 and 8 (pair
+// distance 4 and 8).
+__device__ __forceinline__ void wht_pairs_h4_h8(uint64_t (&xp)[kPairs]) {
 #pragma unroll
-  for (int hp = 2; hp < kE / 2; hp <<= 1) {
+  for (int hp = 4; hp <= 8; hp <<= 1) {
 #pragma unroll
-    for (int k = 0; k < kE / 2; ++k) {
+    for (int k = 0; k < kPairs; ++k) {
       if (!(k & hp)) {
         const uint64_t a = xp[k], b = xp[k + hp];
         xp[k] = f2_add(a, b);
@@ -132,226 +215,282 @@ __device__ __forceinline__ void wht_inlane_h4_to_32(uint64_t (&xp)[kE / 2]) {
   }
 }
 
-// Cross-lane butterflies for h = 64, 128, ..., D/2: the partner part of a
-// vector sits VPW lanes away per doubling.
-template <int P, int VPW>
-__device__ __forceinline__ void wht_crosslane(uint64_t (&xp)[kE / 2], int part) {
+// Butterfly inside each pair (h = 16): (a, b) -> (a + b, a - b).
+__device__ __forceinline__ void wht_in_pair(uint64_t (&xp)[kPairs]) {
 #pragma unroll
-  for (int k = 1; k < P; k <<= 1) {
+  for (int k = 0; k < kPairs; ++k) {
+    float a, b;
+    f2_unpack(xp[k], a, b);
+    xp[k] = f2_pack(a + b, a - b);
+  }
+}
+
+// Full-exchange stages h = 64 .. d/4 (part bits below KH).
+template <int D>
+__device__ __forceinline__ void wht_cross_full(uint64_t (&xp)[kPairs], int part) {
+  constexpr int KH = Lanes<D>::KH, VPW = Lanes<D>::VPW;
+#pragma unroll
+  for (int k = 1; k < KH; k <<= 1) {
     const float sgn = (part & k) ? -1.f : 1.f;
     const uint64_t sgn2 = f2_pack(sgn, sgn);
 #pragma unroll
-    for (int i = 0; i < kE / 2; ++i) {
+    for (int i = 0; i < kPairs; ++i) {
       const uint64_t o = __shfl_xor_sync(0xffffffffu, xp[i], k * VPW);
       xp[i] = f2_fma(sgn2, xp[i], o);
     }
   }
 }
 
-// Applies the 16 per-block 4x4 matrices of this lane's blocks, in place.
-// With z = (z0..z3), Z01 = (z0, z1), Z10 = (z1, z0) and so on:
-//   (y0, y1) = (M00,M11) Z01 + (M01,M10) Z10 + (M02,M13) Z23 + (M03,M12) Z32
-//   (y2, y3) = (M22,M33) Z23 + (M23,M32) Z32 + (M20,M31) Z01 + (M21,M30) Z10
-__device__ __forceinline__ void apply_block_matrices(uint64_t (&xp)[kE / 2], const float *mat_lane) {
+// Lloyd-Max code of one coordinate against thresholds scaled by the norm.
+template <int BITS>
+__device__ __forceinline__ uint32_t quant_code(float y, const float *ts) {
+  constexpr int L = 1 << BITS, NPOS = L / 2 - 1;
+  const float a = fabsf(y);
+  uint32_t m = 0;
 #pragma unroll
-  for (int lb = 0; lb < kE / 4; ++lb) {
-    const float4 *m = reinterpret_cast<const float4 *>(mat_lane + 16 * lb);
-    const float4 m0 = m[0], m1 = m[1], m2 = m[2], m3 = m[3];
-    const uint64_t z01 = xp[2 * lb], z23 = xp[2 * lb + 1];
-    const uint64_t z10 = f2_swap(z01), z32 = f2_swap(z23);
-    uint64_t y01 = f2_mul(f2_pack(m0.x, m0.y), z01);
-    y01 = f2_fma(f2_pack(m0.z, m0.w), z10, y01);
-    y01 = f2_fma(f2_pack(m1.x, m1.y), z23, y01);
-    y01 = f2_fma(f2_pack(m1.z, m1.w), z32, y01);
-    uint64_t y23 = f2_mul(f2_pack(m2.x, m2.y), z23);
-    y23 = f2_fma(f2_pack(m2.z, m2.w), z32, y23);
-    y23 = f2_fma(f2_pack(m3.x, m3.y), z01, y23);
-    y23 = f2_fma(f2_pack(m3.z, m3.w), z10, y23);
-    xp[2 * lb] = y01;
-    xp[2 * lb + 1] = y23;
+  for (int j = 0; j < NPOS; ++j) m += (a > ts[j]) ? 1u : 0u;
+  return (y > 0.f) ? static_cast<uint32_t>(L / 2) + m : static_cast<uint32_t>(L / 2 - 1) - m;
+}
+
+// Codes of one group (16 pairs from xp[base]) packed into its GB/4 words
+// (layout in common.cuh).
+template <int BITS>
+__device__ __forceinline__ void quantize_group(const uint64_t (&xp)[kPairs], int base,
+                                               const float *ts, uint32_t *w) {
+  uint32_t code[32];
+#pragma unroll
+  for (int p = 0; p < kGP; ++p) {
+    float lo, hi;
+    f2_unpack(xp[base + p], lo, hi);
+    code[p] = quant_code<BITS>(lo, ts);
+    code[p + 16] = quant_code<BITS>(hi, ts);
+  }
+  if constexpr (BITS == 3) {
+    uint32_t x = 0;
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v += code[8 * r + j] << (4 * j);
+      w[r] = v;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x += code[24 + j] << (4 * j);
+    w[0] |= (x & 0x11111111u) << 3;
+    w[1] |= (x & 0x22222222u) << 2;
+    w[2] |= (x & 0x44444444u) << 1;
+  } else {
+    constexpr int PER = 32 / BITS;  // codes per word
+#pragma unroll
+    for (int r = 0; r < 32 / PER; ++r) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int j = 0; j < PER; ++j) v += code[PER * r + j] << (BITS * j);
+      w[r] = v;
+    }
   }
 }
 
+// ---------------------------------------------------------------------------
+// Quantize
+// ---------------------------------------------------------------------------
+
 template <typename T, int D, int BITS, bool FULL>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 4)
     quantize_kernel(const __grid_constant__ CUtensorMap xmap, const QuantArgs args) {
   using C = Cfg<T, D, BITS>;
+  constexpr int P = C::P, VPW = C::VPW, KH = C::KH;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char *stages = smem;
-  float *mat = reinterpret_cast<float *>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES + C::MAT_BYTES);
-  uint64_t *empty_bar = full_bar + C::STAGES;
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty_bar + C::STAGES);
-
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  unsigned char *ring = smem + warp * C::RING_BYTES;
+  float *mat = reinterpret_cast<float *>(smem + kQuantWarps * C::RING_BYTES);
+  uint64_t *full_bar =
+      reinterpret_cast<uint64_t *>(smem + kQuantWarps * C::RING_BYTES + C::MAT_BYTES) + warp * C::STAGES;
 
-  // Contiguous range of tiles for this CTA (few head changes per CTA).
+  // Contiguous range of CTA tiles (few head changes per CTA).  Every warp
+  // walks the same tiles, taking rows [warp * VPW, warp * VPW + VPW) of each.
   const long long per_cta = (args.total_tiles + gridDim.x - 1) / gridDim.x;
   const long long tile_begin = static_cast<long long>(blockIdx.x) * per_cta;
   long long tile_end = tile_begin + per_cta;
   if (tile_end > args.total_tiles) tile_end = args.total_tiles;
+  const int n_mine = tile_end > tile_begin ? static_cast<int>(tile_end - tile_begin) : 0;
 
-  if (tid == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kConsumerWarps);
-    }
-    *abort_flag = 0;
+  if (lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(&full_bar[s], 1);
     mbar_fence_init();
+  }
+  __syncwarp();
+
+  auto issue = [&](int i) {
+    const long long t = tile_begin + i;
+    const int head = static_cast<int>(t / args.tiles_per_head);
+    const int v0 = static_cast<int>((t % args.tiles_per_head) * C::NV) + warp * VPW;
+    const int s = i % C::STAGES;
+    unsigned char *st = ring + s * C::STAGE_BYTES;
+    mbar_arrive_expect_tx(&full_bar[s], C::NBOX * C::BOX_BYTES);
+    for (int b = 0; b < C::NBOX; ++b)
+      tma_load_3d(st + b * C::BOX_STRIDE, &xmap, &full_bar[s], b * C::BOX_ELEMS, v0, head);
+  };
+  int issued = 0;
+  if (lane == 0)
+    for (; issued < n_mine && issued < C::STAGES; ++issued) issue(issued);
+
+  int cur_head = -1;
+  if (n_mine > 0) {
+    cur_head = static_cast<int>(tile_begin / args.tiles_per_head);
+    build_block_matrices<D, FULL, true>(args.params + static_cast<size_t>(cur_head) * 2 * D, mat,
+                                        tid, kQuantThreads);
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      int issued_any = 0;
-      for (long long t = tile_begin; t < tile_end; ++t) {
-        const long long it = t - tile_begin;
-        const int s = static_cast<int>(it % C::STAGES);
-        const uint32_t round = static_cast<uint32_t>(it / C::STAGES);
-        if (!mbar_wait_bounded(&empty_bar[s], (round & 1u) ^ 1u) || *abort_flag) {
-          atomicOr(&g_quant_error, kErrWaitTimeout);
-          *abort_flag = 1;
-          break;
-        }
-        const int head = static_cast<int>(t / args.tiles_per_head);
-        const int v0 = static_cast<int>((t % args.tiles_per_head) * C::NV);
-        mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
-        for (int b = 0; b < C::NBOX; ++b)
-          tma_load_3d(stages + s * C::STAGE_BYTES + b * C::BOX_BYTES, &xmap, &full_bar[s],
-                      b * C::BOX_ELEMS, v0, head);
-        issued_any = 1;
-      }
-      // Drain: wait until every issued load has landed before the CTA may exit.
-      if (issued_any) {
-        const long long n = tile_end - tile_begin;
-        const long long first = n > C::STAGES ? n - C::STAGES : 0;
-        for (long long it = first; it < n; ++it) {
-          const int s = static_cast<int>(it % C::STAGES);
-          if (!mbar_wait_bounded(&full_bar[s], static_cast<uint32_t>(it / C::STAGES) & 1u)) {
-            atomicOr(&g_quant_error, kErrWaitTimeout);
-            break;
-          }
-        }
-      }
-    }
-    return;
-  }
-
-  // ---------------- consumers ----------------
-  constexpr int P = C::P, VPW = C::VPW;
-  const int part = lane / VPW;                 // which 64-element slice
+  const int part = lane / VPW;
   const int vl = lane % VPW;
-  const int vt = warp * VPW + vl;              // row of this vector within the tile
-  int cur_head = -1;
+  const bool hb = (part & KH) != 0;
+  int grp[2];
+  lane_groups<D>(part, grp);
+  const uint32_t mat_s = smem_u32(mat);
+  const float sg = hb ? -1.f : 1.f;
+  const uint64_t sig2 = f2_pack(sg, sg), nsig2 = f2_pack(-sg, -sg);
+  bool failed = false;
+  int consumed = 0;
 
-  for (long long t = tile_begin; t < tile_end; ++t) {
-    const long long it = t - tile_begin;
-    const int s = static_cast<int>(it % C::STAGES);
+  for (int i = 0; i < n_mine; ++i) {
+    const long long t = tile_begin + i;
     const int head = static_cast<int>(t / args.tiles_per_head);
-    const long long v = (t % args.tiles_per_head) * C::NV + vt;
-
     if (head != cur_head) {
-      named_barrier(1, kConsumers);
+      // Every warp walks the same tiles, so all of them meet here.
+      named_barrier(1, kQuantThreads);
       build_block_matrices<D, FULL, true>(args.params + static_cast<size_t>(head) * 2 * D, mat,
-                                          tid, kConsumers);
-      named_barrier(1, kConsumers);
+                                          tid, kQuantThreads);
+      named_barrier(1, kQuantThreads);
       cur_head = head;
     }
-
-    if (!mbar_wait_bounded(&full_bar[s], static_cast<uint32_t>(it / C::STAGES) & 1u) ||
-        *abort_flag) {
-      atomicOr(&g_quant_error, kErrWaitTimeout);
-      *abort_flag = 1;
-      return;
+    if (failed) continue;
+    const int s = i % C::STAGES;
+    const bool ok = mbar_wait_bounded(&full_bar[s], static_cast<uint32_t>(i / C::STAGES) & 1u);
+    if (__any_sync(0xffffffffu, !ok)) {
+      if (lane == 0) atomicOr(&g_quant_error, kErrWaitTimeout);
+      failed = true;
+      continue;
     }
 
-    // Load this lane's 64 elements from the swizzled tile as float pairs.
-    uint64_t xp[kE / 2];
-    const unsigned char *stage = stages + s * C::STAGE_BYTES;
+    // Load this lane's 64 elements (two groups of 16 pairs (e, e + 16)),
+    // doing the h = 16 butterfly on the way.
+    uint64_t xp[kPairs];
+    const uint32_t stage = smem_u32(ring + s * C::STAGE_BYTES);
+    const uint32_t sw = static_cast<uint32_t>(vl & 7);
     if constexpr (C::ES == 2) {
-      const unsigned char *box = stage + part * C::BOX_BYTES + vt * 128;
+      const uint32_t row = stage + part * C::BOX_STRIDE + vl * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(box + ((c ^ (vt & 7)) << 4));
-        const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+      for (int G = 0; G < 2; ++G) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = __half22float2(h[j]);
-          xp[4 * c + j] = f2_pack(f.x, f.y);
+        for (int c = 0; c < 2; ++c) {
+          const uint4 ulo = lds128(row + (((4 * G + c) ^ sw) << 4));
+          const uint4 uhi = lds128(row + (((4 * G + 2 + c) ^ sw) << 4));
+          const __half2 *hl = reinterpret_cast<const __half2 *>(&ulo);
+          const __half2 *hh = reinterpret_cast<const __half2 *>(&uhi);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 a = __half22float2(hl[j]);
+            const float2 b = __half22float2(hh[j]);
+            xp[kGP * G + 8 * c + 2 * j] = f2_pack(a.x + b.x, a.x - b.x);
+            xp[kGP * G + 8 * c + 2 * j + 1] = f2_pack(a.y + b.y, a.y - b.y);
+          }
         }
       }
     } else {
 #pragma unroll
-      for (int bx = 0; bx < 2; ++bx) {
-        const unsigned char *box = stage + (2 * part + bx) * C::BOX_BYTES + vt * 128;
+      for (int G = 0; G < 2; ++G) {
+        const uint32_t row = stage + (2 * part + G) * C::BOX_STRIDE + vl * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 f = *reinterpret_cast<const float4 *>(box + ((c ^ (vt & 7)) << 4));
-          xp[16 * bx + 2 * c] = f2_pack(f.x, f.y);
-          xp[16 * bx + 2 * c + 1] = f2_pack(f.z, f.w);
+        for (int c = 0; c < 4; ++c) {
+          const uint4 ulo = lds128(row + ((c ^ sw) << 4));
+          const uint4 uhi = lds128(row + (((4 + c) ^ sw) << 4));
+          const float a0 = __uint_as_float(ulo.x), a1 = __uint_as_float(ulo.y);
+          const float a2 = __uint_as_float(ulo.z), a3 = __uint_as_float(ulo.w);
+          const float b0 = __uint_as_float(uhi.x), b1 = __uint_as_float(uhi.y);
+          const float b2 = __uint_as_float(uhi.z), b3 = __uint_as_float(uhi.w);
+          xp[kGP * G + 4 * c] = f2_pack(a0 + b0, a0 - b0);
+          xp[kGP * G + 4 * c + 1] = f2_pack(a1 + b1, a1 - b1);
+          xp[kGP * G + 4 * c + 2] = f2_pack(a2 + b2, a2 - b2);
+          xp[kGP * G + 4 * c + 3] = f2_pack(a3 + b3, a3 - b3);
         }
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[s]);  // the stage may be refilled
+    consumed = i + 1;
+    // The warp is done reading stage s: refill it STAGES tiles ahead.
+    if (lane == 0 && issued < n_mine) {
+      fence_proxy_async_smem();
+      issue(issued);
+      ++issued;
+    }
 
-    // Step 1: norm (float32 accumulation, reduced over the P lanes).
+    // Step 1: norm.  The pairs hold (a + b, a - b), whose squares sum to
+    // twice a^2 + b^2.
     uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
-    for (int k = 0; k < kE / 2; ++k) acc2 = f2_fma(xp[k], xp[k], acc2);
+    for (int k = 0; k < kPairs; ++k) acc2 = f2_fma(xp[k], xp[k], acc2);
     float ss_lo, ss_hi;
     f2_unpack(acc2, ss_lo, ss_hi);
-    float ss = ss_lo + ss_hi;
+    float ss = 0.5f * (ss_lo + ss_hi);
 #pragma unroll
     for (int k = 1; k < P; k <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, k * VPW);
     const float norm = sqrtf(ss);
 
-    // Step 2: WHT stages h >= 4, then the folded (H_4, SO(4), 1/sqrt d) blocks.
-    wht_inlane_h4_to_32(xp);
-    wht_crosslane<P, VPW>(xp, part);
-    apply_block_matrices(xp, mat + part * (kE / 4) * 16);
-    float x[kE];
+    // Step 2: the remaining WHT stages, then the folded block matrices.
+    wht_pairs_h4_h8(xp);
+    // h = 32, arranged so that group 0 holds what this lane keeps in the
+    // half exchange: (G0, G1) <- (G0 + sg G1, G0 - sg G1).
 #pragma unroll
-    for (int k = 0; k < kE / 2; ++k) f2_unpack(xp[k], x[2 * k], x[2 * k + 1]);
+    for (int p = 0; p < kGP; ++p) {
+      const uint64_t a = xp[p], b = xp[kGP + p];
+      xp[p] = f2_fma(sig2, b, a);
+      xp[kGP + p] = f2_fma(nsig2, b, a);
+    }
+    wht_cross_full<D>(xp, part);
+#pragma unroll
+    for (int p = 0; p < kGP; ++p) {
+      const uint64_t r = __shfl_xor_sync(0xffffffffu, xp[kGP + p], KH * VPW);
+      const uint64_t k = xp[p];
+      xp[p] = f2_add(k, r);
+      xp[kGP + p] = f2_sub(k, r);
+    }
+    apply_group_matrices(xp, 0, mat_s + 512 * grp[0]);
+    apply_group_matrices(xp, kGP, mat_s + 512 * grp[1]);
 
-    // Step 3: Lloyd-Max codes against thresholds scaled by the norm.
-    float ts[C::NPOS > 0 ? C::NPOS : 1];
+    // Steps 3-4: Lloyd-Max codes and bit-packing, one 32-code group at a time.
+    float ts[C::NPOS];
 #pragma unroll
     for (int j = 0; j < C::NPOS; ++j) ts[j] = args.tau[j] * norm;
-    uint32_t w[C::TB / 4];
-#pragma unroll
-    for (int k = 0; k < C::TB / 4; ++k) w[k] = 0u;
-#pragma unroll
-    for (int i = 0; i < kE; ++i) {
-      const float y = x[i];
-      const float a = fabsf(y);
-      int m = 0;
-#pragma unroll
-      for (int j = 0; j < C::NPOS; ++j) m += (a > ts[j]) ? 1 : 0;
-      const uint32_t code = (y > 0.f) ? static_cast<uint32_t>(C::L / 2 + m)
-                                      : static_cast<uint32_t>(C::L / 2 - 1 - m);
-      // Step 4: bit-pack (layout in common.cuh).
-      pack_code<BITS>(w, i, code);
-    }
-
+    const long long v = (t % args.tiles_per_head) * C::NV + warp * VPW + vl;
     if (v < args.n_vec) {
       const long long idx = static_cast<long long>(head) * args.out_head_stride + v;
-      uint8_t *dst = args.codes + idx * C::PB + part * C::TB;
-      if constexpr (C::TB % 16 == 0) {
+      uint8_t *dst = args.codes + idx * C::PB;
 #pragma unroll
-        for (int k = 0; k < C::TB / 16; ++k)
-          reinterpret_cast<uint4 *>(dst)[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-      } else {
+      for (int G = 0; G < 2; ++G) {
+        uint32_t w[C::GB / 4];
+        quantize_group<BITS>(xp, kGP * G, ts, w);
+        uint8_t *gd = dst + grp[G] * C::GB;
+        if constexpr (C::GB == 16) {
+          *reinterpret_cast<uint4 *>(gd) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else if constexpr (C::GB == 8) {
+          *reinterpret_cast<uint2 *>(gd) = make_uint2(w[0], w[1]);
+        } else {
 #pragma unroll
-        for (int k = 0; k < C::TB / 8; ++k)
-          reinterpret_cast<uint2 *>(dst)[k] = make_uint2(w[2 * k], w[2 * k + 1]);
+          for (int k = 0; k < C::GB / 4; ++k) reinterpret_cast<uint32_t *>(gd)[k] = w[k];
+        }
       }
       if (part == 0) args.norms[idx] = __half_as_ushort(__float2half_rn(norm));
     }
+  }
+  if (failed && lane == 0) {
+    // Let every copy still in flight land before the CTA may exit.
+    for (int k = consumed; k < issued; ++k)
+      if (!mbar_wait_bounded(&full_bar[k % C::STAGES], static_cast<uint32_t>(k / C::STAGES) & 1u)) break;
   }
 }
 
@@ -374,18 +513,23 @@ struct DequantArgs {
   float centroid[16];
 };
 
-constexpr int kDequantThreads = 128;
-
 template <typename T, int D, int BITS, bool FULL>
 __global__ void __launch_bounds__(kDequantThreads) dequantize_kernel(const DequantArgs args) {
-  constexpr int P = D / kE, VPW = 32 / P, NV = kDequantThreads / P;
-  constexpr int L = 1 << BITS, PB = D * BITS / 8, TB = kE * BITS / 8;
-  __shared__ __align__(16) float mat[(D / 4) * 16];
+  constexpr int P = Lanes<D>::P, VPW = Lanes<D>::VPW, KH = Lanes<D>::KH;
+  constexpr int NV = kDequantThreads / P;
+  constexpr int PB = D * BITS / 8, GB = 32 * BITS / 8;
+  constexpr int L = 1 << BITS;
+  __shared__ __align__(16) float mat[D * 4];
   __shared__ float cent[16];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int part = lane / VPW, vl = lane % VPW, vt = warp * VPW + vl;
+  const int part = lane / VPW, vl = lane % VPW;
+  const int vt = warp * VPW + vl;
+  const bool hb = (part & KH) != 0;
+  int grp[2];
+  lane_groups<D>(part, grp);
   if (tid < L) cent[tid] = args.centroid[tid];
+  const uint32_t mat_s = smem_u32(mat);
 
   const long long per_cta = (args.total_tiles + gridDim.x - 1) / gridDim.x;
   const long long tile_begin = static_cast<long long>(blockIdx.x) * per_cta;
@@ -405,56 +549,86 @@ __global__ void __launch_bounds__(kDequantThreads) dequantize_kernel(const Dequa
     }
     const bool valid = v < args.n_vec;
     const long long idx = static_cast<long long>(head) * args.in_head_stride + (valid ? v : 0);
+    const uint8_t *src = args.codes + idx * PB;
 
-    uint32_t w[TB / 4];
-    const uint8_t *src = args.codes + idx * PB + part * TB;
-    if constexpr (TB % 16 == 0) {
+    // Centroids of this lane's two groups as pairs (e, e + 16).
+    uint64_t xp[kPairs];
 #pragma unroll
-      for (int k = 0; k < TB / 16; ++k) {
-        const uint4 u = reinterpret_cast<const uint4 *>(src)[k];
-        w[4 * k] = u.x; w[4 * k + 1] = u.y; w[4 * k + 2] = u.z; w[4 * k + 3] = u.w;
-      }
-    } else {
+    for (int G = 0; G < 2; ++G) {
+      uint32_t w[GB / 4];
+      const uint8_t *gs = src + grp[G] * GB;
+      if constexpr (GB == 16) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(gs);
+        w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+      } else if constexpr (GB == 8) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(gs);
+        w[0] = u.x; w[1] = u.y;
+      } else {
 #pragma unroll
-      for (int k = 0; k < TB / 8; ++k) {
-        const uint2 u = reinterpret_cast<const uint2 *>(src)[k];
-        w[2 * k] = u.x; w[2 * k + 1] = u.y;
+        for (int k = 0; k < GB / 4; ++k) w[k] = reinterpret_cast<const uint32_t *>(gs)[k];
       }
+#pragma unroll
+      for (int p = 0; p < kGP; ++p)
+        xp[kGP * G + p] = f2_pack(cent[unpack_code<BITS>(w, p)], cent[unpack_code<BITS>(w, p + 16)]);
     }
     const float s16 = __half2float(__ushort_as_half(args.norms[idx]));
 
-    uint64_t xp[kE / 2];
+    apply_group_matrices(xp, 0, mat_s + 512 * grp[0]);
+    apply_group_matrices(xp, kGP, mat_s + 512 * grp[1]);
+    // Half exchange (h = d/2): keep G0 + G1, send G0 - G1.
 #pragma unroll
-    for (int k = 0; k < kE / 2; ++k)
-      xp[k] = f2_pack(cent[unpack_code<BITS>(w, 2 * k)], cent[unpack_code<BITS>(w, 2 * k + 1)]);
-    apply_block_matrices(xp, mat + part * (kE / 4) * 16);
-    wht_inlane_h4_to_32(xp);
-    wht_crosslane<P, VPW>(xp, part);
-    const uint64_t s2 = f2_pack(s16, s16);
+    for (int p = 0; p < kGP; ++p) {
+      const uint64_t a = xp[p], b = xp[kGP + p];
+      const uint64_t dsend = f2_sub(a, b);
+      xp[p] = f2_add(a, b);
+      xp[kGP + p] = __shfl_xor_sync(0xffffffffu, dsend, KH * VPW);
+    }
+    wht_cross_full<D>(xp, part);
+    // h = 32: afterwards G0 holds this lane's lower 32 elements and G1 its
+    // upper 32, the latter negated on lanes with the exchange bit set.
 #pragma unroll
-    for (int k = 0; k < kE / 2; ++k) xp[k] = f2_mul(xp[k], s2);
-    float x[kE];
+    for (int p = 0; p < kGP; ++p) {
+      const uint64_t a = xp[p], b = xp[kGP + p];
+      xp[p] = f2_add(a, b);
+      xp[kGP + p] = f2_sub(a, b);
+    }
+    wht_pairs_h4_h8(xp);
+    wht_in_pair(xp);
+    const uint64_t sc0 = f2_pack(s16, s16);
+    const float s1 = hb ? -s16 : s16;
+    const uint64_t sc1 = f2_pack(s1, s1);
 #pragma unroll
-    for (int k = 0; k < kE / 2; ++k) f2_unpack(xp[k], x[2 * k], x[2 * k + 1]);
+    for (int p = 0; p < kGP; ++p) {
+      xp[p] = f2_mul(xp[p], sc0);
+      xp[kGP + p] = f2_mul(xp[kGP + p], sc1);
+    }
 
     if (valid) {
       T *dst = static_cast<T *>(args.out) + static_cast<long long>(head) * args.head_stride +
                v * args.vec_stride + part * kE;
-      if constexpr (sizeof(T) == 2) {
 #pragma unroll
-        for (int c = 0; c < kE / 8; ++c) {
-          uint4 u;
-          __half2 *h = reinterpret_cast<__half2 *>(&u);
+      for (int G = 0; G < 2; ++G) {
+        float lo[kGP], hi[kGP];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            h[j] = __floats2half2_rn(x[8 * c + 2 * j], x[8 * c + 2 * j + 1]);
-          reinterpret_cast<uint4 *>(dst)[c] = u;
+        for (int p = 0; p < kGP; ++p) f2_unpack(xp[kGP * G + p], lo[p], hi[p]);
+        T *gd = dst + 32 * G;
+        if constexpr (sizeof(T) == 2) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float *e = c < 2 ? lo + 8 * c : hi + 8 * (c - 2);
+            uint4 u;
+            __half2 *h = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(e[2 * j], e[2 * j + 1]);
+            reinterpret_cast<uint4 *>(gd)[c] = u;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float *e = c < 4 ? lo + 4 * c : hi + 4 * (c - 4);
+            reinterpret_cast<float4 *>(gd)[c] = make_float4(e[0], e[1], e[2], e[3]);
+          }
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kE / 4; ++c)
-          reinterpret_cast<float4 *>(dst)[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2],
-                                                           x[4 * c + 3]);
       }
     }
   }
@@ -520,7 +694,7 @@ int launch_quantize(const void *x, int n_heads, long long n_vec, long long head_
   const long long hs = n_heads > 1 ? head_stride : vec_stride * n_vec;
   const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(vec_stride * C::ES),
                                  static_cast<cuuint64_t>(hs * C::ES)};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(C::BOX_ELEMS), static_cast<cuuint32_t>(C::NV), 1u};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(C::BOX_ELEMS), static_cast<cuuint32_t>(C::VPW), 1u};
   const cuuint32_t estride[3] = {1u, 1u, 1u};
   CUresult r = encode(&map, C::ES == 2 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                       3, const_cast<void *>(x), gdim, gstride, box, estride,
@@ -553,7 +727,7 @@ template <typename T, int D, int BITS, bool FULL>
 int launch_dequantize(const uint8_t *codes, const uint16_t *norms, int n_heads, long long n_vec,
                       long long in_head_stride, const float *params, void *out,
                       long long head_stride, long long vec_stride, cudaStream_t stream) {
-  constexpr int NV = kDequantThreads / (D / kE);
+  constexpr int NV = kDequantThreads / Lanes<D>::P;
   auto kernel = dequantize_kernel<T, D, BITS, FULL>;
   static int max_ctas_per_sm = -1;
   static std::mutex mu;
