@@ -36,6 +36,8 @@ struct CombineArgs {
 
 bool mma_path_supported(int dtype, int d, int bits, const SplitArgs &a);
 int run_split_mma(int d, int variant, const SplitArgs &a, cudaStream_t stream);
+bool i8_path_supported(const SplitArgs &a);
+int run_split_i8(int d, int variant, const SplitArgs &a, cudaStream_t stream);
 
 }  // namespace decode
 }  // namespace isoq

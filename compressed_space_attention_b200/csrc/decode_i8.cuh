@@ -1,0 +1,732 @@
+// Integer tensor-core split kernel of the compressed-space decode: float16
+// queries, 3-bit codes, d in {128, 256}, up to 8 query heads per KV head.
+// Included by isoq_decode.cu inside namespace isoq::decode, after
+// decode_mma.cuh (whose slab ring, shared-memory loads and selectors it uses).
+//
+// The work per token is RotaryQuant Table 2 kernels A-C on the packed codes:
+// z_j = s^K_j <q~, c[K_j]> scale, online softmax, acc += p_j s^V_j c[V_j], all
+// in the rotated domain.  What makes this kernel different from the float16
+// one is how a code becomes a tensor-core operand.
+//
+// Exact integer centroids.  The unit-variance centroids are scaled by a
+// host-chosen S (about 7,500) so that every C_k = round(S c_k) is within a few
+// hundredths of S c_k; |C_k| <= 16319 is split as C = 128 Ch + Cl with
+// Ch in [-128, 127] and Cl in [-64, 63].  Each part is an int8 table of 8
+// entries held in two registers, so one prmt turns four codes (a 4-nibble
+// selector) into a full int8 MMA register: half a prmt per code per part,
+// against one prmt per code for a float16 operand, whose two bytes need a
+// lookup each plus an interleave.
+//
+// QK (kernel A): mma.sync m16n8k32 s8 x s8 -> s32.  A = Ch or Cl of 16 tokens
+// x 32 dims; B = the rotated query in 22-bit fixed point,
+// Q = 2^14 Qh + 2^7 Qm + Ql (per-head step max|q~| / 2088000), the three
+// parts in separate columns (or N tiles).  Each part's two products give
+// sum C Q_part exactly in int32; only their conversion to float32 and the
+// final 2^14 / 2^7 weighting round.
+//
+// Softmax (kernel B): float32, log2 domain, on the accumulator fragments.
+//
+// PV (kernel C): mma.sync m16n8k32 s8 x u8 -> s32 with M = 16 dim quads,
+// K = 8 tokens x 4 parities, N = 2 heads x 4 parities:
+//   D[u][(h, r)] = sum_(j, r') A[u][(j, r')] B[(j, r')][(h, r)],
+//   A[u][(j, r')] = V~[j][4u + r'],   B[(j, r')][(h, r)] = W[j][h] [r' = r],
+// so every A register is four consecutive codes of one token, exactly what
+// one prmt lookup produces.  W = p s^V is block-scaled per 16-token slab and
+// head to 16 bits, W = 256 Wh + Wl (u8 parts); C W = 2^15 Ch Wh +
+// 2^7 (Ch Wl + 2 Cl Wh) + Cl Wl, of which the last term (below 2^-15 of one
+// token's largest contribution) is dropped.  W is fixed-point against a
+// per-warp reference, W_q = rint(p s^V 32000 / s_ref) with p = 2^(x - m_ref)
+// <= 2 and s^V <= s_ref, so the two int32 sums accumulate across the whole
+// chunk; they are rescaled only when a block's maximum score
+// passes m_ref + 1 or a V norm passes s_ref, which after the first block is
+// rare.  The pair (m_ref, l) it leaves is a valid partial state: l and acc
+// are both relative to 2^m_ref.
+//
+// Fragment orders.  A fixed permutation of the rotated coordinates cancels in
+// q~.k~ and is undone when the accumulator is written out:
+//   QK: per 16-token tile, lane (g, t) owns tokens g, g+8 and dims
+//       [t d/4, (t+1) d/4) (one or two 32-code groups); k-step kk uses quads
+//       2kk, 2kk+1 of that range.
+//   PV: per 16-token half, lane (g, t) owns tokens t, t+4, t+8, t+12 and the
+//       32-code group g (d = 256) or half of group g/2 (d = 128); M-block mb
+//       maps row g to the lane's quad 2mb and row g+8 to quad 2mb+1.
+//
+// Staging: each warp streams 32-token blocks (packed K and V rows, float16
+// norms) through its own 2-deep ring with CTA-local bulk copies and mbarrier
+// completion, refilling a stage as soon as it has consumed it.
+//
+// Selectors.  A prmt selector is four 3-bit codes in the low nibbles of its
+// low 16 bits.  The 32-code group layout (codes in 4-bit fields, codes
+// 24..31 spread over the spare bits) needs a mask per word and a shift per
+// high half on the integer pipe; the lookups themselves (half a prmt per code
+// per part) are the rest of that pipe's work, which bounds the kernel.
+
+constexpr int kI8Warps = 4;
+constexpr int kI8Threads = 32 * kI8Warps;
+constexpr int kBlk = 32;                 // tokens per ring stage (two 16-token MMA tiles)
+constexpr int kI8Stages = 2;             // per-warp ring depth
+constexpr int kCentroidIntMax = 16319;   // |C_k| bound that keeps Ch, 2 Cl in int8
+constexpr int kQueryIntMax = 2088000;    // |Q| bound that keeps Qh, Qm, Ql in int8
+constexpr float kWScale = 32000.f;       // W_q = rint(p s^V kWScale / s_ref), p <= 2
+constexpr float kNormHeadroom = 1.25f;   // s_ref = 1.25 x the largest V norm seen
+
+template <int D, int GP>
+struct I8Cfg {
+  static constexpr int PB = D * 3 / 8;                      // packed bytes per token
+  static constexpr int BLK_CODES = kBlk * PB;
+  static constexpr int BLK_NORMS = kBlk * 2;
+  static constexpr int STAGE_BYTES = 2 * BLK_CODES + 2 * BLK_NORMS;
+  static constexpr int RING_BYTES = kI8Stages * STAGE_BYTES;
+  static constexpr int KK = D / 32;                         // QK k-steps (8 codes per lane-row each)
+  static constexpr int GRP_QK = D / 128;                    // 32-code groups per QK lane segment
+  static constexpr int MB = D / 64;                         // PV M-blocks (64 dims each)
+  static constexpr int NQ = GP <= 2 ? 1 : (GP == 4 ? 2 : 3);  // QK N tiles (3 parts x GP columns)
+  static constexpr int NV = (GP + 1) / 2;                   // PV N tiles (2 heads each)
+  static constexpr int SCRATCH_FLOATS = GP * D;             // q~, then the warp merge
+  static constexpr int SMEM = kI8Warps * RING_BYTES + SCRATCH_FLOATS * 4 + 8 * 4 +
+                              2 * kI8Warps * 8 * 4 + kI8Warps * kI8Stages * 8 + 128;
+  static constexpr int MIN_BLOCKS = (D == 256 && GP == 8) ? 2 : ((D == 256 && GP == 4) || GP == 8 ? 3 : 4);
+};
+
+// int8 tables of the centroid parts, four entries per register: kh/kl =
+// (Ch, Cl) for the K side, vh/vl = (Ch, 2 Cl) for the V side.
+struct I8Lut {
+  uint32_t kh0, kh1, kl0, kl1, vh0, vh1, vl0, vl1;
+};
+
+__device__ __forceinline__ float ex2f(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// c += A B (s8 x s8), and the same with a zero accumulator.
+__device__ __forceinline__ void mma_s8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_s8s8_z(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                           uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{0,0,0,0};"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// c += A B (s8 x u8).
+__device__ __forceinline__ void mma_s8u8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// prmt selectors of the eight quads of one 32-code group (three words in the
+// layout of common.cuh); quad q = codes 4q..4q+3, in the low 16 bits of s[q].
+__device__ __forceinline__ void group_sel8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t (&s)[8]) {
+  const uint32_t m0 = w0 & 0x77777777u, m1 = w1 & 0x77777777u, m2 = w2 & 0x77777777u;
+  // The spare bits x_r = w_r - m_r (bit 4j+3 = bit r of code 24+j) gathered
+  // into nibbles: the three shifted planes are disjoint, so their sum (integer
+  // adds, which the compiler may place on the FMA pipe) is their union.
+  const uint32_t x0 = w0 - m0, x1 = w1 - m1, x2 = w2 - m2;
+  const uint32_t sum = (x0 >> 2) + (x1 >> 1) + x2;   // code 24+j at bits 4j+1 .. 4j+3
+  s[0] = m0;
+  s[1] = m0 >> 16;
+  s[2] = m1;
+  s[3] = m1 >> 16;
+  s[4] = m2;
+  s[5] = m2 >> 16;
+  s[6] = sum >> 1;
+  s[7] = sum >> 17;
+}
+
+// Packs the low 16 bits of two words into one (a in bits 0-15, b in 16-31).
+__device__ __forceinline__ uint32_t pack_lo16(uint32_t a, uint32_t b) { return prmt(a, b, 0x5410u); }
+
+// Four int8 values into one register, byte i = v[i].
+__device__ __forceinline__ uint32_t pack_s8x4(int v0, int v1, int v2, int v3) {
+  return (static_cast<uint32_t>(v0) & 0xFFu) | ((static_cast<uint32_t>(v1) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(v2) & 0xFFu) << 16) | ((static_cast<uint32_t>(v3) & 0xFFu) << 24);
+}
+
+// E <- rint(E F) for one pair of int32 sums representing 256 E1 + E2 (F <= 1;
+// the fraction of E1 F that is dropped is below 2^-15 of one token's largest
+// contribution).
+__device__ __forceinline__ void rescale_pair(int &e1, int &e2, float f) {
+  e1 = __float2int_rn(static_cast<float>(e1) * f);
+  e2 = __float2int_rn(static_cast<float>(e2) * f);
+}
+
+// GP: query heads per KV head rounded up to 1, 2, 4 or 8 (padded heads carry
+// zero queries and zero weights).
+template <int D, bool FULL, int GP>
+__global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
+    split_i8_kernel(const SplitArgs a, const I8Lut lut, float score_unit, float out_scale) {
+  using C = I8Cfg<D, GP>;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.group;
+
+  unsigned char *ring = smem + warp * C::RING_BYTES;
+  float *scratch = reinterpret_cast<float *>(smem + kI8Warps * C::RING_BYTES);
+  float *qinv = scratch + C::SCRATCH_FLOATS;        // [8] max|q~_h| / kQueryIntMax
+  float *wm = qinv + 8;                             // [warps][8]
+  float *wl = wm + kI8Warps * 8;                    // [warps][8]
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(wl + kI8Warps * 8) + warp * kI8Stages;
+
+  int tlen = a.seq_lens[b];
+  tlen = tlen < 0 ? 0 : (tlen > a.tmax ? static_cast<int>(a.tmax) : tlen);
+  const long long t0 = static_cast<long long>(split) * a.chunk;
+  long long t1 = t0 + a.chunk;
+  if (t1 > tlen) t1 = tlen;
+  const int n_tok = t1 > t0 ? static_cast<int>(t1 - t0) : 0;
+  const int n_blk = (n_tok + kBlk - 1) / kBlk;
+  const int n_mine = n_blk > warp ? (n_blk - warp + kI8Warps - 1) / kI8Warps : 0;
+
+  const long long pair = static_cast<long long>(b) * a.hkv + kvh;
+  const uint8_t *kb = a.packed_k + pair * a.tmax * C::PB;
+  const uint8_t *vb = a.packed_v + pair * a.tmax * C::PB;
+  const uint16_t *nkb = a.norms_k + pair * a.tmax;
+  const uint16_t *nvb = a.norms_v + pair * a.tmax;
+
+  // Lane 0 of each warp issues the copies of the warp's i-th block into ring
+  // stage i % kI8Stages.
+  auto issue = [&](int i) {
+    const int j = warp + kI8Warps * i;
+    const long long t = t0 + static_cast<long long>(j) * kBlk;
+    int n = n_tok - j * kBlk;
+    if (n > kBlk) n = kBlk;
+    const int n8 = (n + 7) & ~7;
+    const int s = i % kI8Stages;
+    unsigned char *st = ring + s * C::STAGE_BYTES;
+    mbar_arrive_expect_tx(&full_bar[s], 2u * n * C::PB + 4u * n8);
+    bulk_load(st, kb + t * C::PB, n * C::PB, &full_bar[s]);
+    bulk_load(st + C::BLK_CODES, vb + t * C::PB, n * C::PB, &full_bar[s]);
+    bulk_load(st + 2 * C::BLK_CODES, nkb + t, 2 * n8, &full_bar[s]);
+    bulk_load(st + 2 * C::BLK_CODES + C::BLK_NORMS, nvb + t, 2 * n8, &full_bar[s]);
+  };
+  int issued = 0;
+  if (lane == 0) {
+    for (int s = 0; s < kI8Stages; ++s) mbar_init(&full_bar[s], 1);
+    mbar_fence_init();
+    for (; issued < kI8Stages && issued < n_mine; ++issued) issue(issued);
+  }
+
+  // Rotate the G queries of this KV head once, q~ = R_K q, while the first
+  // blocks stream in; padded heads stay zero.
+  for (int i = tid; i < GP * D; i += kI8Threads) {
+    const int gq = i / D;
+    float v = 0.f;
+    if (gq < G) {
+      const __half *qp = static_cast<const __half *>(a.q) +
+                         (static_cast<long long>(b) * a.hq + kvh * G + gq) * D;
+      v = __half2float(qp[i % D]);
+    }
+    scratch[i] = v;
+  }
+  __syncthreads();
+  rotate_forward_smem<D, FULL>(scratch, G, a.params_k + static_cast<size_t>(kvh) * 2 * D, tid,
+                               kI8Threads, 0);
+  // Per-head fixed-point step of the query: max|q~_h| / kQueryIntMax.
+  for (int h = warp; h < 8; h += kI8Warps) {
+    float mx = 0.f;
+    if (h < G)
+      for (int i = lane; i < D; i += 32) mx = fmaxf(mx, fabsf(scratch[h * D + i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) qinv[h] = mx / static_cast<float>(kQueryIntMax);
+  }
+  __syncthreads();
+
+  const int g = lane >> 2, t = lane & 3;
+
+  // B fragments of the fixed-point query Q = rint(q~ / qinv) =
+  // 2^14 Qh + 2^7 Qm + Ql: tile nq, column g = (head, part), dims of quads
+  // 2kk, 2kk+1 of lane t.  Part p of head h sits in tile 0, column p GP + h
+  // (GP <= 2); tile 0, column 4p + h for p < 2 and tile 1, column h for p = 2
+  // (GP = 4); tile p, column h (GP = 8).
+  uint32_t qb[C::NQ][C::KK][2];
+#pragma unroll
+  for (int nq = 0; nq < C::NQ; ++nq) {
+    int head, part;
+    if constexpr (GP <= 2) {
+      part = g / GP;
+      head = g % GP;
+    } else if constexpr (GP == 4) {
+      part = nq == 0 ? (g >> 2) : (g < 4 ? 2 : 3);
+      head = g & 3;
+    } else {
+      part = nq;
+      head = g;
+    }
+    const bool live = part < 3 && head < G;
+    const float qi = live ? qinv[head] : 0.f;
+    const float qs = qi > 0.f ? 1.f / qi : 0.f;
+#pragma unroll
+    for (int kk = 0; kk < C::KK; ++kk) {
+      const int grp = (D == 256 ? 2 * t : t) + kk / 4;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int base = 32 * grp + 4 * (2 * (kk & 3) + half);
+        int v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int q = live ? __float2int_rn(scratch[head * D + base + i] * qs) : 0;
+          q = q > kQueryIntMax ? kQueryIntMax : (q < -kQueryIntMax ? -kQueryIntMax : q);
+          const int r1 = (q + 64) >> 7, ql = q - 128 * r1;     // arithmetic shifts: floor
+          const int r2 = (r1 + 64) >> 7, qm = r1 - 128 * r2;
+          v[i] = part == 0 ? r2 : (part == 1 ? qm : ql);
+        }
+        qb[nq][kk][half] = pack_s8x4(v[0], v[1], v[2], v[3]);
+      }
+    }
+  }
+  const bool real0 = 2 * t < G, real1 = 2 * t + 1 < G;
+  const float qk0 = real0 ? qinv[2 * t] * score_unit : 0.f;
+  const float qk1 = real1 ? qinv[2 * t + 1] * score_unit : 0.f;
+
+  // prmt selectors that move byte k of a packed (W_a, W_b) word to byte g&3
+  // of a PV B register (zeros elsewhere): lo / hi byte of head parity g>>2.
+  const uint32_t r4 = 4u * static_cast<uint32_t>(g & 3);
+  const uint32_t hpb = 2u * static_cast<uint32_t>(g >> 2);
+  const uint32_t sel_lo = (0x4444u & ~(0xFu << r4)) | (hpb << r4);
+  const uint32_t sel_hi = (0x4444u & ~(0xFu << r4)) | ((hpb + 1u) << r4);
+
+  // PV sums 256 E1 + E2 (int32, whole chunk) in the PV layout: head
+  // 2nv + (t >> 1).
+  int e1[C::NV][C::MB][4], e2[C::NV][C::MB][4];
+#pragma unroll
+  for (int nvt = 0; nvt < C::NV; ++nvt)
+#pragma unroll
+    for (int mb = 0; mb < C::MB; ++mb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) e1[nvt][mb][e] = e2[nvt][mb][e] = 0;
+  // Softmax state in the QK layout (heads 2t, 2t+1; log2 domain): reference
+  // maximum and sum; the V-norm reference is warp-uniform.
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float s_ref = 0.f, wsc = 0.f;
+
+  int consumed = 0;
+  bool failed = false;
+  for (int i = 0; i < n_mine; ++i) {
+    const int s = i % kI8Stages;
+    if (!mbar_wait_bounded(&full_bar[s], (i / kI8Stages) & 1)) {
+      atomicOr(&g_decode_error, kErrWaitTimeout);
+      failed = true;
+      break;
+    }
+    int nvalid = n_tok - (warp + kI8Warps * i) * kBlk;
+    nvalid = nvalid > kBlk ? kBlk : nvalid;
+    const unsigned char *st = ring + s * C::STAGE_BYTES;
+    const unsigned char *kc = st;
+    const unsigned char *vc = st + C::BLK_CODES;
+    const unsigned char *nk = st + 2 * C::BLK_CODES;                 // float16 [32]
+    const unsigned char *nv = st + 2 * C::BLK_CODES + C::BLK_NORMS;
+
+    // ---- QK: exact int32 sums of C * Q_part over the lane's dims, per tile ----
+    // sc[T][e]: token 16T + g + 8 (e >> 1), head 2t + (e & 1).
+    float sc[2][4];
+#pragma unroll
+    for (int T = 0; T < 2; ++T) {
+      int d1[C::NQ][4], d2[C::NQ][4];
+      constexpr int NW = D * 3 / 128;   // words per token segment (6 or 3)
+      uint32_t wg[NW], wg8[NW];
+      const unsigned char *rg = kc + (16 * T + g) * C::PB + t * (NW * 4);
+      const unsigned char *rg8 = rg + 8 * C::PB;
+      if constexpr (NW % 2 == 0) {
+#pragma unroll
+        for (int k = 0; k < NW / 2; ++k) {
+          const uint2 x = lds64(rg + 8 * k), y = lds64(rg8 + 8 * k);
+          wg[2 * k] = x.x;
+          wg[2 * k + 1] = x.y;
+          wg8[2 * k] = y.x;
+          wg8[2 * k + 1] = y.y;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < NW; ++k) {
+          wg[k] = lds32(rg + 4 * k);
+          wg8[k] = lds32(rg8 + 4 * k);
+        }
+      }
+#pragma unroll
+      for (int gq = 0; gq < C::GRP_QK; ++gq) {
+        uint32_t sa[8], sb[8];
+        group_sel8(wg[3 * gq], wg[3 * gq + 1], wg[3 * gq + 2], sa);
+        group_sel8(wg8[3 * gq], wg8[3 * gq + 1], wg8[3 * gq + 2], sb);
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          const int kk = 4 * gq + kq;
+          const uint32_t sa0 = sa[2 * kq], sa1 = sa[2 * kq + 1], sb0 = sb[2 * kq], sb1 = sb[2 * kq + 1];
+          {
+            const uint32_t a0 = prmt(lut.kh0, lut.kh1, sa0), a1 = prmt(lut.kh0, lut.kh1, sb0);
+            const uint32_t a2 = prmt(lut.kh0, lut.kh1, sa1), a3 = prmt(lut.kh0, lut.kh1, sb1);
+#pragma unroll
+            for (int nq = 0; nq < C::NQ; ++nq) {
+              if (kk == 0)
+                mma_s8s8_z(d1[nq], a0, a1, a2, a3, qb[nq][kk][0], qb[nq][kk][1]);
+              else
+                mma_s8s8(d1[nq], a0, a1, a2, a3, qb[nq][kk][0], qb[nq][kk][1]);
+            }
+          }
+          {
+            const uint32_t a0 = prmt(lut.kl0, lut.kl1, sa0), a1 = prmt(lut.kl0, lut.kl1, sb0);
+            const uint32_t a2 = prmt(lut.kl0, lut.kl1, sa1), a3 = prmt(lut.kl0, lut.kl1, sb1);
+#pragma unroll
+            for (int nq = 0; nq < C::NQ; ++nq) {
+              if (kk == 0)
+                mma_s8s8_z(d2[nq], a0, a1, a2, a3, qb[nq][kk][0], qb[nq][kk][1]);
+              else
+                mma_s8s8(d2[nq], a0, a1, a2, a3, qb[nq][kk][0], qb[nq][kk][1]);
+            }
+          }
+        }
+      }
+      // sum C Q = 2^14 X_h + 2^7 X_m + X_l with X_p = 128 (sum Ch Q_p) + sum Cl Q_p;
+      // c0 = (g, 2t), c1 = (g, 2t+1), c2 = (g+8, 2t), c3 = (g+8, 2t+1).
+      float f[C::NQ][4];
+#pragma unroll
+      for (int nq = 0; nq < C::NQ; ++nq)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f[nq][e] = static_cast<float>(128 * d1[nq][e] + d2[nq][e]);
+      if constexpr (GP == 1) {
+        // columns (hi, mid, lo): hi and mid in lane t = 0, lo in lane t = 1
+        const float lo0 = __shfl_xor_sync(0xffffffffu, f[0][0], 1);
+        const float lo2 = __shfl_xor_sync(0xffffffffu, f[0][2], 1);
+        sc[T][0] = fmaf(f[0][0], 16384.f, fmaf(f[0][1], 128.f, lo0));
+        sc[T][2] = fmaf(f[0][2], 16384.f, fmaf(f[0][3], 128.f, lo2));
+        sc[T][1] = sc[T][3] = 0.f;
+      } else if constexpr (GP == 2) {
+        // lane t = 0: hi, t = 1: mid, t = 2: lo of heads 0, 1
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          sc[T][e] = fmaf(f[0][e], 16384.f, fmaf(__shfl_xor_sync(0xffffffffu, f[0][e], 1), 128.f,
+                                                 __shfl_xor_sync(0xffffffffu, f[0][e], 2)));
+      } else if constexpr (GP == 4) {
+        // tile 0: lanes t = 0, 1 hi, t = 2, 3 mid; tile 1: lanes t = 0, 1 lo
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          sc[T][e] = fmaf(f[0][e], 16384.f, fmaf(__shfl_xor_sync(0xffffffffu, f[0][e], 2), 128.f, f[1][e]));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[T][e] = fmaf(f[0][e], 16384.f, fmaf(f[1][e], 128.f, f[2][e]));
+      }
+    }
+
+    // ---- softmax bookkeeping (log2 domain) ----
+    float x[2][4], sv[2][2];
+    float mx0 = -INFINITY, mx1 = -INFINITY, vmx = 0.f;
+#pragma unroll
+    for (int T = 0; T < 2; ++T) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int j = 16 * T + 8 * hh + g;
+        const bool ok = j < nvalid;
+        const float sk = lds_half(nk + 2 * j);
+        const float svr = lds_half(nv + 2 * j);
+        sv[T][hh] = ok ? svr : 0.f;
+        vmx = fmaxf(vmx, sv[T][hh]);
+        // Padded heads hold a constant 0 so that they never move the maximum.
+        x[T][2 * hh] = real0 ? (ok ? sc[T][2 * hh] * sk * qk0 : -INFINITY) : 0.f;
+        x[T][2 * hh + 1] = real1 ? (ok ? sc[T][2 * hh + 1] * sk * qk1 : -INFINITY) : 0.f;
+        mx0 = fmaxf(mx0, x[T][2 * hh]);
+        mx1 = fmaxf(mx1, x[T][2 * hh + 1]);
+      }
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
+    }
+    // Move the references only when this block would leave the fixed-point
+    // range: a score above m_ref + 1 or a V norm above s_ref.
+    const bool ev0 = mx0 > m0 + 1.f, ev1 = mx1 > m1 + 1.f, evs = vmx > s_ref;
+    if (__any_sync(0xffffffffu, ev0 || ev1 || evs)) {
+      const float mn0 = ev0 ? mx0 : m0, mn1 = ev1 ? mx1 : m1;
+      const float f0 = ex2f(m0 - mn0), f1 = ex2f(m1 - mn1);   // 0 on the first block
+      const float sn = evs ? vmx * kNormHeadroom : s_ref;
+      const float ratio = sn > 0.f ? s_ref / sn : 0.f;
+      l0 *= f0;
+      l1 *= f1;
+      m0 = mn0;
+      m1 = mn1;
+      s_ref = sn;
+      wsc = sn > 0.f ? kWScale / sn : 0.f;
+#pragma unroll
+      for (int nvt = 0; nvt < C::NV; ++nvt) {
+        const float fa = __shfl_sync(0xffffffffu, f0, nvt), fb = __shfl_sync(0xffffffffu, f1, nvt);
+        const float F = ((t >> 1) ? fb : fa) * ratio;
+#pragma unroll
+        for (int mb = 0; mb < C::MB; ++mb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) rescale_pair(e1[nvt][mb][e], e2[nvt][mb][e], F);
+      }
+    }
+    // p = 2^(x - m_ref) <= 2; W_q = rint(p s^V kWScale / s_ref) < 2^16 from the
+    // low 16 bits of p s^V wsc + 2^23.  u[T][hh]: (W head 2t, W head 2t+1) of
+    // token 16T + 8hh + g.
+    uint32_t u[2][2];
+#pragma unroll
+    for (int T = 0; T < 2; ++T) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const float p0 = ex2f(x[T][2 * hh] - m0), p1 = ex2f(x[T][2 * hh + 1] - m1);
+        l0 += p0;
+        l1 += p1;
+        const float w = sv[T][hh] * wsc;
+        const float wq0 = real0 ? fmaf(p0, w, 8388608.f) : 8388608.f;
+        const float wq1 = real1 ? fmaf(p1, w, 8388608.f) : 8388608.f;
+        u[T][hh] = pack_lo16(__float_as_uint(wq0), __float_as_uint(wq1));
+      }
+    }
+
+    // ---- PV, per 16-token half: this lane's tokens t, t+4, t+8, t+12 ----
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      // B fragments of W for each N tile nv (heads 2nv, 2nv+1): column g =
+      // (head 2nv + (g >> 2), parity g & 3); MMA c covers tokens 16 h2 + 8c +
+      // {t, t+4}, held by the QK lanes (t or t+4, nv) in u[h2][c].
+      uint32_t bh[C::NV][2][2], bl[C::NV][2][2];
+#pragma unroll
+      for (int nvt = 0; nvt < C::NV; ++nvt) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t xa = __shfl_sync(0xffffffffu, u[h2][c], 4 * t + nvt);
+          const uint32_t xb = __shfl_sync(0xffffffffu, u[h2][c], 4 * t + 16 + nvt);
+          bh[nvt][c][0] = prmt(xa, 0u, sel_hi);
+          bh[nvt][c][1] = prmt(xb, 0u, sel_hi);
+          bl[nvt][c][0] = prmt(xa, 0u, sel_lo);
+          bl[nvt][c][1] = prmt(xb, 0u, sel_lo);
+        }
+      }
+      uint32_t vs[4][8];
+      {
+        const int goff = (D == 256 ? g : (g >> 1)) * 12;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const unsigned char *row = vc + (16 * h2 + t + 4 * r) * C::PB + goff;
+          group_sel8(lds32(row), lds32(row + 4), lds32(row + 8), vs[r]);
+        }
+      }
+#pragma unroll
+      for (int mb = 0; mb < C::MB; ++mb) {
+        // Quads of the lane: 2mb, 2mb+1 of its group (d = 256) or of its half
+        // group (d = 128: codes 16..31 for odd g).
+        uint32_t ah[4][2], al[4][2];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          uint32_t s0, s1;
+          if constexpr (D == 256) {
+            s0 = vs[r][2 * mb];
+            s1 = vs[r][2 * mb + 1];
+          } else {
+            s0 = (g & 1) ? vs[r][4 + 2 * mb] : vs[r][2 * mb];
+            s1 = (g & 1) ? vs[r][5 + 2 * mb] : vs[r][2 * mb + 1];
+          }
+          ah[r][0] = prmt(lut.vh0, lut.vh1, s0);
+          ah[r][1] = prmt(lut.vh0, lut.vh1, s1);
+          al[r][0] = prmt(lut.vl0, lut.vl1, s0);
+          al[r][1] = prmt(lut.vl0, lut.vl1, s1);
+        }
+#pragma unroll
+        for (int nvt = 0; nvt < C::NV; ++nvt) {
+          mma_s8u8(e1[nvt][mb], ah[0][0], ah[0][1], ah[1][0], ah[1][1], bh[nvt][0][0], bh[nvt][0][1]);
+          mma_s8u8(e1[nvt][mb], ah[2][0], ah[2][1], ah[3][0], ah[3][1], bh[nvt][1][0], bh[nvt][1][1]);
+          mma_s8u8(e2[nvt][mb], ah[0][0], ah[0][1], ah[1][0], ah[1][1], bl[nvt][0][0], bl[nvt][0][1]);
+          mma_s8u8(e2[nvt][mb], ah[2][0], ah[2][1], ah[3][0], ah[3][1], bl[nvt][1][0], bl[nvt][1][1]);
+          mma_s8u8(e2[nvt][mb], al[0][0], al[0][1], al[1][0], al[1][1], bh[nvt][0][0], bh[nvt][0][1]);
+          mma_s8u8(e2[nvt][mb], al[2][0], al[2][1], al[3][0], al[3][1], bh[nvt][1][0], bh[nvt][1][1]);
+        }
+      }
+    }
+    __syncwarp();
+    consumed = i + 1;
+    // The warp is done reading stage s: refill it with the block kI8Stages on.
+    if (lane == 0 && issued < n_mine) {
+      fence_proxy_async_smem();
+      issue(issued);
+      ++issued;
+    }
+  }
+  if (failed && lane == 0) {
+    // Let every copy still in flight land before the CTA may exit.
+    for (int k = consumed; k < issued; ++k)
+      if (!mbar_wait_bounded(&full_bar[k % kI8Stages], (k / kI8Stages) & 1)) break;
+  }
+
+  // Per-warp totals over the 8 lanes sharing t.
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  __syncthreads();   // all warps are done with the q~ scratch
+  if (g == 0) {
+    wm[warp * 8 + 2 * t] = m0;
+    wm[warp * 8 + 2 * t + 1] = m1;
+    wl[warp * 8 + 2 * t] = l0;
+    wl[warp * 8 + 2 * t + 1] = l1;
+  }
+  __syncthreads();
+  // Merge the warps' accumulators into scratch[head][dim] (rotated domain),
+  // one warp after the other so that the sum order is fixed.  One unit of
+  // 256 E1 + E2 is 2^7 s_ref / kWScale of sum p s^V C.
+  {
+    const float unit = s_ref * (128.f / kWScale);
+    const int grp = D == 256 ? g : (g >> 1);
+    const int qoff = D == 256 ? 0 : 4 * (g & 1);
+    float f[C::NV];
+#pragma unroll
+    for (int nvt = 0; nvt < C::NV; ++nvt) {
+      const int h = 2 * nvt + (t >> 1);
+      float mstar = -INFINITY;
+      for (int w2 = 0; w2 < kI8Warps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
+      const float mine = wm[warp * 8 + h];
+      f[nvt] = (mine == -INFINITY) ? 0.f : exp2f(mine - mstar) * unit;
+    }
+    for (int w2 = 0; w2 < kI8Warps; ++w2) {
+      if (warp == w2) {
+#pragma unroll
+        for (int nvt = 0; nvt < C::NV; ++nvt) {
+          const int h = 2 * nvt + (t >> 1);
+          if (h < G) {
+#pragma unroll
+            for (int mb = 0; mb < C::MB; ++mb) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int dim = 32 * grp + 4 * (2 * mb + (e >> 1) + qoff) + 2 * (t & 1) + (e & 1);
+                float *dst = scratch + h * D + dim;
+                const float v = fmaf(static_cast<float>(e1[nvt][mb][e]), 256.f,
+                                     static_cast<float>(e2[nvt][mb][e])) * f[nvt];
+                *dst = (w2 == 0) ? v : *dst + v;
+              }
+            }
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // One partial state per query head: natural-log max, sum, acc (unscaled).
+  for (int h = 0; h < G; ++h) {
+    const long long slot = (static_cast<long long>(b) * a.hq + kvh * G + h) * a.n_splits + split;
+    float *acc_out = a.ws_acc + slot * D;
+    for (int i = tid; i < D; i += kI8Threads) acc_out[i] = scratch[h * D + i] * out_scale;
+    if (tid == 0) {
+      float mstar = -INFINITY, l = 0.f;
+      for (int w2 = 0; w2 < kI8Warps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
+      for (int w2 = 0; w2 < kI8Warps; ++w2) {
+        const float mw = wm[w2 * 8 + h];
+        if (mw != -INFINITY) l += wl[w2 * 8 + h] * exp2f(mw - mstar);
+      }
+      a.ws_ml[slot] = make_float2(mstar == -INFINITY ? -INFINITY : mstar * 0.69314718055994531f, l);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+struct I8Tables {
+  double scale;   // S: C_k = rint(S c_k) for the unit-variance centroids c_k
+  I8Lut lut;
+};
+
+inline int floor_div128(int x) { return x >= 0 ? x / 128 : -((-x + 127) / 128); }
+
+// S in [0.75, 1] * 16319 / c_max minimising the largest relative rounding
+// error of S c_k over the four positive 3-bit centroids (searched once).
+const I8Tables &i8_tables() {
+  static I8Tables tb;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    double c[8];
+    codebook_unit_f64(3, c);
+    const double s_max = kCentroidIntMax / c[7];
+    double best = s_max, best_err = 1.0;
+    const int steps = 1 << 22;
+    for (int i = 0; i <= steps; ++i) {
+      const double s = s_max * (0.75 + 0.25 * static_cast<double>(i) / steps);
+      double err = 0.0;
+      for (int k = 4; k < 8 && err < best_err; ++k) {
+        const double v = s * c[k];
+        err = std::fmax(err, std::fabs(std::nearbyint(v) - v) / v);
+      }
+      if (err < best_err) {
+        best_err = err;
+        best = s;
+      }
+    }
+    tb.scale = best;
+    uint32_t kh[2] = {0, 0}, kl[2] = {0, 0}, vl[2] = {0, 0};
+    for (int k = 0; k < 8; ++k) {
+      const int ck = static_cast<int>(std::lrint(best * c[k]));
+      const int ch = floor_div128(ck + 64);
+      const int cl = ck - 128 * ch;
+      const int sh = 8 * (k % 4);
+      kh[k / 4] |= (static_cast<uint32_t>(ch) & 0xFFu) << sh;
+      kl[k / 4] |= (static_cast<uint32_t>(cl) & 0xFFu) << sh;
+      vl[k / 4] |= (static_cast<uint32_t>(2 * cl) & 0xFFu) << sh;
+    }
+    tb.lut = I8Lut{kh[0], kh[1], kl[0], kl[1], kh[0], kh[1], vl[0], vl[1]};
+  });
+  return tb;
+}
+
+template <int D, bool FULL, int GP>
+int launch_split_i8(const SplitArgs &a, cudaStream_t stream) {
+  using C = I8Cfg<D, GP>;
+  auto kernel = split_i8_kernel<D, FULL, GP>;
+  static bool configured = false;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured) {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+      if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode i8: %s", cudaGetErrorString(e));
+      configured = true;
+    }
+  }
+  const I8Tables &tb = i8_tables();
+  const double unit = 1.0 / (tb.scale * std::sqrt(static_cast<double>(D)));
+  const float score_unit = static_cast<float>(a.scale * unit * 1.4426950408889634);
+  const float out_scale = static_cast<float>(unit);
+  dim3 grid(a.n_splits, a.hkv, a.batch);
+  kernel<<<grid, kI8Threads, C::SMEM, stream>>>(a, tb.lut, score_unit, out_scale);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode i8 launch: %s", cudaGetErrorString(e));
+  return ISOQ_OK;
+}
+
+// The int32 PV sums of a warp stay below 2^31 for up to 2^16 tokens per warp
+// (|Ch Wh| <= 128 * 255, |Ch Wl + 2 Cl Wh| <= 2 * 128 * 255 per token).
+bool i8_path_supported(const SplitArgs &a) { return a.chunk <= 4LL * kI8Warps * 16384; }
+
+template <int D, bool FULL>
+int run_split_i8_d(const SplitArgs &a, cudaStream_t st) {
+  const int G = a.group;
+  if (G == 1) return launch_split_i8<D, FULL, 1>(a, st);
+  if (G == 2) return launch_split_i8<D, FULL, 2>(a, st);
+  if (G <= 4) return launch_split_i8<D, FULL, 4>(a, st);
+  return launch_split_i8<D, FULL, 8>(a, st);
+}
+
+int run_split_i8(int d, int variant, const SplitArgs &a, cudaStream_t st) {
+  if (d == 128)
+    return variant == ISOQ_FULL ? run_split_i8_d<128, true>(a, st) : run_split_i8_d<128, false>(a, st);
+  return variant == ISOQ_FULL ? run_split_i8_d<256, true>(a, st) : run_split_i8_d<256, false>(a, st);
+}

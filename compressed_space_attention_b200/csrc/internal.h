@@ -29,6 +29,8 @@ struct CodebookF32 {
 };
 // Memoised; safe to call from several threads.  Returns false on bad args.
 bool codebook_f32(int d, int bits, CodebookF32 *out);
+// Centroids of the unit-variance (N(0, 1)) codebook in double, L = 2^bits.
+bool codebook_unit_f64(int bits, double *centroids);
 
 // Split policy of the decode path.
 constexpr int kDecodeTokenQuantum = 64;   // chunk sizes are multiples of this

@@ -291,6 +291,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
 }
 
 #include "decode_mma.cuh"
+#include "decode_i8.cuh"
 
 // ---------------------------------------------------------------------------
 // Host launchers
@@ -435,7 +436,9 @@ int isoq_decode_split(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
   codebook_f32(d, bits, &cb);
   for (int j = 0; j < 16; ++j) a.centroid[j] = j < cb.levels ? cb.centroid[j] : 0.f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (decode::mma_path_supported(dtype, d, bits, a)) return decode::run_split_mma(d, variant, a, s);
+  if (decode::mma_path_supported(dtype, d, bits, a))
+    return decode::i8_path_supported(a) ? decode::run_split_i8(d, variant, a, s)
+                                        : decode::run_split_mma(d, variant, a, s);
   return decode::run_split_generic(dtype, d, bits, variant, a, s);
 }
 

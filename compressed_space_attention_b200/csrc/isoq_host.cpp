@@ -157,6 +157,13 @@ bool codebook_f32(int d, int bits, CodebookF32 *out) {
   return true;
 }
 
+bool codebook_unit_f64(int bits, double *centroids) {
+  if (!supported_bits(bits)) return false;
+  const UnitCodebook &u = unit_codebook(bits);
+  for (int k = 0; k < (1 << bits); ++k) centroids[k] = u.c[k];
+  return true;
+}
+
 // Each split covers a fixed number of tokens (a multiple of 64) chosen so
 // that B * Hkv * n_splits is about 8 CTAs per SM of a 148-SM B200, with
 // chunks between 256 and 4096 tokens.
