@@ -43,6 +43,7 @@ METRIC = "packed-3-bit decode attn KV GB/s (% of HBM peak); quantize Mvec/s"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["compressed_space_attention_b200/csrc/isoq_decode.cu",
                   "compressed_space_attention_b200/csrc/decode_mma.cuh",
+                  "compressed_space_attention_b200/csrc/decode_i8.cuh",
                   "compressed_space_attention_b200/csrc/common.cuh"]
 TRAFFIC_PROFILE = "profiles/decode_split_b32_gqa16_8_d256_t65536.md"
 
@@ -468,7 +469,7 @@ def run_isoq(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": workload_config(args.workload, n_ranks, args.batch),
         "frac_of_hbm_peak": value / n_ranks / hbm,
-        "roofline": {"bound": "hbm", "kernel": "split_mma_kernel<256,Full> (decode split)",
+        "roofline": {"bound": "hbm", "kernel": "split_i8_kernel<256,Full,GP=2> (decode split)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": read_traffic(), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                      "algorithmic_bytes_per_launch": kv_bytes},

@@ -35,7 +35,9 @@
 //
 // The quantiser compares the unnormalised R x with s * t_k (no division per
 // element) using the symmetry of the codebook: the sign picks the half, and
-// the magnitude is counted against the positive thresholds.
+// the magnitude is counted against the positive thresholds.  Both decisions
+// are exact 0/1 steps from saturating FMAs, so the search and the packing of
+// the codes run as float arithmetic on the FMA pipe.
 //
 // Data movement.  Each warp of a quantize CTA streams its own rows through a
 // ring of 128B-swizzled TMA tiles (no producer warp); each lane reads its own
@@ -241,52 +243,97 @@ __device__ __forceinline__ void wht_cross_full(uint64_t (&xp)[kPairs], int part)
   }
 }
 
-// Lloyd-Max code of one coordinate against thresholds scaled by the norm.
-template <int BITS>
-__device__ __forceinline__ uint32_t quant_code(float y, const float *ts) {
-  constexpr int L = 1 << BITS, NPOS = L / 2 - 1;
-  const float a = fabsf(y);
-  uint32_t m = 0;
-#pragma unroll
-  for (int j = 0; j < NPOS; ++j) m += (a > ts[j]) ? 1u : 0u;
-  return (y > 0.f) ? static_cast<uint32_t>(L / 2) + m : static_cast<uint32_t>(L / 2 - 1) - m;
+// The Lloyd-Max search runs on the FMA pipe.  With `big` a power of two that
+// scales a coordinate of the vector to about 2^40 (one float ulp of any scaled
+// threshold is then >= 1), fma.sat(|y|, big, -t big) is exactly 1.0 when
+// |y| > t and 0.0 otherwise (ties go to the lower code).  The sign step uses
+// two multiplies by 2^127, which take any nonzero y to +-inf-or-beyond-1 and
+// keep +-0 at 0.  Codes are then small exact integers in float32, and the
+// packing accumulates them as exact integers below 2^24 (offset by 2^23, so
+// that the low 16 bits of the float are the packed field).
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
-// Codes of one group (16 pairs from xp[base]) packed into its GB/4 words
-// (layout in common.cuh).
+__device__ __forceinline__ float mul_sat(float a, float b) {
+  float r;
+  asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// Power of two about 2^40 / norm (clamped to [2^-126, 2^127]; 2^127 for a
+// zero norm).
+__device__ __forceinline__ float search_scale(float norm) {
+  int e = 294 - static_cast<int>((__float_as_uint(norm) >> 23) & 0xFFu);
+  e = e < 1 ? 1 : (e > 254 ? 254 : e);
+  return __uint_as_float(static_cast<uint32_t>(e) << 23);
+}
+
+// Codes of one group (16 pairs (e, e + 16) from xp[base]) packed into its
+// GB/4 words (layout in common.cuh).  tb[j] = -t_j big for the positive
+// thresholds t_j scaled by the norm.
 template <int BITS>
 __device__ __forceinline__ void quantize_group(const uint64_t (&xp)[kPairs], int base,
-                                               const float *ts, uint32_t *w) {
-  uint32_t code[32];
+                                               const float *tb, float big, uint32_t *w) {
+  constexpr int L = 1 << BITS, NPOS = L / 2 - 1;
+  const float p127 = 1.7014118346046923e38f;   // 2^127
+  const uint64_t one2 = f2_pack(1.f, 1.f), two2 = f2_pack(2.f, 2.f);
+  const uint64_t low2 = f2_pack(static_cast<float>(L / 2 - 1), static_cast<float>(L / 2 - 1));
+  uint64_t cp[kGP];   // (code of element e, code of element e + 16) per pair
 #pragma unroll
   for (int p = 0; p < kGP; ++p) {
-    float lo, hi;
-    f2_unpack(xp[base + p], lo, hi);
-    code[p] = quant_code<BITS>(lo, ts);
-    code[p + 16] = quant_code<BITS>(hi, ts);
+    float y0, y1;
+    f2_unpack(xp[base + p], y0, y1);
+    const float a0 = fabsf(y0), a1 = fabsf(y1);
+    // m = #{j : |y| > t_j}
+    uint64_t m = f2_pack(fma_sat(a0, big, tb[0]), fma_sat(a1, big, tb[0]));
+#pragma unroll
+    for (int j = 1; j < NPOS; ++j) m = f2_add(m, f2_pack(fma_sat(a0, big, tb[j]), fma_sat(a1, big, tb[j])));
+    // s = [y > 0]
+    const uint64_t s = f2_pack(mul_sat(y0 * p127, p127), mul_sat(y1 * p127, p127));
+    // code = s ? L/2 + m : L/2 - 1 - m  =  (L/2 - 1 - m) + s (2m + 1)
+    cp[p] = f2_fma(s, f2_fma(m, two2, one2), f2_sub(low2, m));
   }
-  if constexpr (BITS == 3) {
-    uint32_t x = 0;
+  // Exact integer packing: acc_q = 2^23 + sum of the pair's codes times their
+  // field weights; the low 16 bits of each float are one half word.
+  constexpr int PER_HALF = 16 / BITS == 5 ? 4 : 16 / BITS;   // codes per 16-bit half (3 bits: 4-bit fields)
+  constexpr int FIELD = BITS == 3 ? 4 : BITS;
+  constexpr int NACC = kGP / PER_HALF;
+  const uint64_t magic2 = f2_pack(8388608.f, 8388608.f);
+  uint32_t lo[NACC], hi[NACC];
 #pragma unroll
-    for (int r = 0; r < 3; ++r) {
-      uint32_t v = 0;
+  for (int q = 0; q < NACC; ++q) {
+    uint64_t acc = f2_add(cp[PER_HALF * q], magic2);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v += code[8 * r + j] << (4 * j);
-      w[r] = v;
+    for (int j = 1; j < PER_HALF; ++j) {
+      const float wgt = static_cast<float>(1u << (FIELD * j));
+      acc = f2_fma(cp[PER_HALF * q + j], f2_pack(wgt, wgt), acc);
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) x += code[24 + j] << (4 * j);
-    w[0] |= (x & 0x11111111u) << 3;
-    w[1] |= (x & 0x22222222u) << 2;
-    w[2] |= (x & 0x44444444u) << 1;
+    float fl, fh;
+    f2_unpack(acc, fl, fh);
+    lo[q] = __float_as_uint(fl);
+    hi[q] = __float_as_uint(fh);
+  }
+  if constexpr (BITS == 2) {
+    // words: codes 0..15 (low elements), codes 16..31 (high elements)
+    w[0] = __byte_perm(lo[0], lo[1], 0x5410);
+    w[1] = __byte_perm(hi[0], hi[1], 0x5410);
   } else {
-    constexpr int PER = 32 / BITS;  // codes per word
-#pragma unroll
-    for (int r = 0; r < 32 / PER; ++r) {
-      uint32_t v = 0;
-#pragma unroll
-      for (int j = 0; j < PER; ++j) v += code[PER * r + j] << (BITS * j);
-      w[r] = v;
+    // words: codes 0..7, 8..15 (low elements), 16..23, 24..31 (high elements)
+    const uint32_t w0 = __byte_perm(lo[0], lo[1], 0x5410), w1 = __byte_perm(lo[2], lo[3], 0x5410);
+    const uint32_t w2 = __byte_perm(hi[0], hi[1], 0x5410), w3 = __byte_perm(hi[2], hi[3], 0x5410);
+    if constexpr (BITS == 3) {
+      // codes 24..31 go to the spare bits: bit r of code 24 + j -> bit 4j + 3 of word r
+      w[0] = w0 + (w3 & 0x11111111u) * 8u;
+      w[1] = w1 + (w3 & 0x22222222u) * 4u;
+      w[2] = w2 + (w3 & 0x44444444u) * 2u;
+    } else {
+      w[0] = w0;
+      w[1] = w1;
+      w[2] = w2;
+      w[3] = w3;
     }
   }
 }
@@ -463,9 +510,10 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     apply_group_matrices(xp, kGP, mat_s + 512 * grp[1]);
 
     // Steps 3-4: Lloyd-Max codes and bit-packing, one 32-code group at a time.
-    float ts[C::NPOS];
+    const float big = search_scale(norm);
+    float tb[C::NPOS];
 #pragma unroll
-    for (int j = 0; j < C::NPOS; ++j) ts[j] = args.tau[j] * norm;
+    for (int j = 0; j < C::NPOS; ++j) tb[j] = -(args.tau[j] * norm) * big;
     const long long v = (t % args.tiles_per_head) * C::NV + warp * VPW + vl;
     if (v < args.n_vec) {
       const long long idx = static_cast<long long>(head) * args.out_head_stride + v;
@@ -473,7 +521,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
 #pragma unroll
       for (int G = 0; G < 2; ++G) {
         uint32_t w[C::GB / 4];
-        quantize_group<BITS>(xp, kGP * G, ts, w);
+        quantize_group<BITS>(xp, kGP * G, tb, big, w);
         uint8_t *gd = dst + grp[G] * C::GB;
         if constexpr (C::GB == 16) {
           *reinterpret_cast<uint4 *>(gd) = make_uint4(w[0], w[1], w[2], w[3]);
