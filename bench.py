@@ -273,9 +273,10 @@ def run_reference(args):
     return 0
 
 
-def workload_config(workload, n_gpus, batch=0):
+def workload_config(workload, n_gpus, batch=0, context=0):
     B, Hq, Hkv, T, d = WORKLOADS[workload]
     B = batch or B
+    T = context or T
     return {
         "workload": workload + "+stage1_quantize_dequantize_d128_b3_f16_n1048576",
         "batch": B, "context": T, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d, "bits": 3,
@@ -338,6 +339,8 @@ def run_isoq(args):
     B, Hq, Hkv, T, d = WORKLOADS[args.workload]
     if args.batch:
         B = args.batch
+    if args.context:
+        T = args.context
     bits, variant = 3, isoq.ISOQ_FULL
     pb = d * bits // 8
     seed0 = rank_seed(rank)
@@ -467,7 +470,7 @@ def run_isoq(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_ranks, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": workload_config(args.workload, n_ranks, args.batch),
+        "config": workload_config(args.workload, n_ranks, args.batch, args.context),
         "frac_of_hbm_peak": value / n_ranks / hbm,
         "roofline": {"bound": "hbm", "kernel": "split_i8_kernel<256,Full,GP=2> (decode split)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
@@ -513,6 +516,8 @@ def main():
                     help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the decode batch size (smaller profiling cases)")
+    ap.add_argument("--context", type=int, default=0,
+                    help="override the decode context length (the long-context sweep)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -19,6 +19,7 @@ struct SplitArgs {
   const float *params_k;
   float *ws_acc;   // [B][Hq][n_splits][d]
   float2 *ws_ml;   // [B][Hq][n_splits] (max, sum)
+  uint32_t *ws_qprep;  // [B][Hkv][decode_qprep_words(d)] prepared queries (int8 path)
   long long tmax;
   long long chunk;  // tokens per split
   int batch, hq, hkv, group, n_splits;

@@ -82,8 +82,9 @@ struct I8Cfg {
   static constexpr int MB = D / 64;                         // PV M-blocks (64 dims each)
   static constexpr int NQ = GP <= 2 ? 1 : (GP == 4 ? 2 : 3);  // QK N tiles (3 parts x GP columns)
   static constexpr int NV = (GP + 1) / 2;                   // PV N tiles (2 heads each)
-  static constexpr int SCRATCH_FLOATS = GP * D;             // q~, then the warp merge
-  static constexpr int SMEM = kI8Warps * RING_BYTES + SCRATCH_FLOATS * 4 + 8 * 4 +
+  static constexpr int SCRATCH_FLOATS = GP * D;             // the warp merge
+  static constexpr int QPREP_WORDS = 3 * KK * 2 * 32 + 8;   // per (b, kvh), see prep_i8_kernel
+  static constexpr int SMEM = kI8Warps * RING_BYTES + SCRATCH_FLOATS * 4 +
                               2 * kI8Warps * 8 * 4 + kI8Warps * kI8Stages * 8 + 128;
   static constexpr int MIN_BLOCKS = (D == 256 && GP == 8) ? 2 : ((D == 256 && GP == 4) || GP == 8 ? 3 : 4);
 };
@@ -165,11 +166,87 @@ __device__ __forceinline__ void rescale_pair(int &e1, int &e2, float f) {
   e2 = __float2int_rn(static_cast<float>(e2) * f);
 }
 
+// Query preparation, one CTA per (b, kvh): rotate the G queries once,
+// q~ = R_K q, and write for every lane of the split kernel the B-fragment
+// words of the fixed-point query Q = rint(q~ / qinv) = 2^14 Qh + 2^7 Qm + Ql
+// (qinv = max|q~_h| / kQueryIntMax per head), then the per-head score factors
+// qinv_h * score_unit (0 for padded heads).  Word ((nq KK + kk) 2 + half) 32
+// + lane holds tile nq, k-step kk, half `half` of lane (g, t): column g is
+// (head, part) with part p of head h in tile 0, column p GP + h (GP <= 2);
+// tile 0, column 4p + h for p < 2 and tile 1, column h for p = 2 (GP = 4);
+// tile p, column h (GP = 8); the four int8 values are the dims of quad
+// 2 (kk mod 4) + half of lane t's 32-code group (D = 128: group t; D = 256:
+// group 2t + kk / 4).
+template <int D, bool FULL, int GP>
+__global__ void __launch_bounds__(kI8Threads) prep_i8_kernel(const SplitArgs a, float score_unit) {
+  using C = I8Cfg<D, GP>;
+  __shared__ float qs[GP * D];
+  __shared__ float qinv[8];
+  const int kvh = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.group;
+  for (int i = tid; i < GP * D; i += kI8Threads) {
+    const int gq = i / D;
+    float v = 0.f;
+    if (gq < G) {
+      const __half *qp = static_cast<const __half *>(a.q) +
+                         (static_cast<long long>(b) * a.hq + kvh * G + gq) * D;
+      v = __half2float(qp[i % D]);
+    }
+    qs[i] = v;
+  }
+  __syncthreads();
+  rotate_forward_smem<D, FULL>(qs, G, a.params_k + static_cast<size_t>(kvh) * 2 * D, tid, kI8Threads, 0);
+  for (int h = warp; h < 8; h += kI8Warps) {
+    float mx = 0.f;
+    if (h < G)
+      for (int i = lane; i < D; i += 32) mx = fmaxf(mx, fabsf(qs[h * D + i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) qinv[h] = mx / static_cast<float>(kQueryIntMax);
+  }
+  __syncthreads();
+
+  uint32_t *out = a.ws_qprep + (static_cast<long long>(b) * a.hkv + kvh) * C::QPREP_WORDS;
+  constexpr int NWORDS = C::NQ * C::KK * 2 * 32;
+  for (int idx = tid; idx < NWORDS; idx += kI8Threads) {
+    const int ln = idx & 31, half = (idx >> 5) & 1, kk = (idx >> 6) % C::KK, nq = (idx >> 6) / C::KK;
+    const int g = ln >> 2, t = ln & 3;
+    int head, part;
+    if constexpr (GP <= 2) {
+      part = g / GP;
+      head = g % GP;
+    } else if constexpr (GP == 4) {
+      part = nq == 0 ? (g >> 2) : (g < 4 ? 2 : 3);
+      head = g & 3;
+    } else {
+      part = nq;
+      head = g;
+    }
+    const bool live = part < 3 && head < G;
+    const float qi = live ? qinv[head] : 0.f;
+    const float qsc = qi > 0.f ? 1.f / qi : 0.f;
+    const int grp = (D == 256 ? 2 * t : t) + kk / 4;
+    const int base = 32 * grp + 4 * (2 * (kk & 3) + half);
+    int v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int q = live ? __float2int_rn(qs[head * D + base + i] * qsc) : 0;
+      q = q > kQueryIntMax ? kQueryIntMax : (q < -kQueryIntMax ? -kQueryIntMax : q);
+      const int r1 = (q + 64) >> 7, ql = q - 128 * r1;     // arithmetic shifts: floor
+      const int r2 = (r1 + 64) >> 7, qm = r1 - 128 * r2;
+      v[i] = part == 0 ? r2 : (part == 1 ? qm : ql);
+    }
+    out[idx] = pack_s8x4(v[0], v[1], v[2], v[3]);
+  }
+  if (tid < 8) out[3 * C::KK * 2 * 32 + tid] = __float_as_uint(tid < G ? qinv[tid] * score_unit : 0.f);
+}
+
 // GP: query heads per KV head rounded up to 1, 2, 4 or 8 (padded heads carry
 // zero queries and zero weights).
 template <int D, bool FULL, int GP>
 __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
-    split_i8_kernel(const SplitArgs a, const I8Lut lut, float score_unit, float out_scale) {
+    split_i8_kernel(const SplitArgs a, const I8Lut lut, float out_scale) {
   using C = I8Cfg<D, GP>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -180,8 +257,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
 
   unsigned char *ring = smem + warp * C::RING_BYTES;
   float *scratch = reinterpret_cast<float *>(smem + kI8Warps * C::RING_BYTES);
-  float *qinv = scratch + C::SCRATCH_FLOATS;        // [8] max|q~_h| / kQueryIntMax
-  float *wm = qinv + 8;                             // [warps][8]
+  float *wm = scratch + C::SCRATCH_FLOATS;          // [warps][8]
   float *wl = wm + kI8Warps * 8;                    // [warps][8]
   uint64_t *full_bar = reinterpret_cast<uint64_t *>(wl + kI8Warps * 8) + warp * kI8Stages;
 
@@ -222,79 +298,23 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     mbar_fence_init();
     for (; issued < kI8Stages && issued < n_mine; ++issued) issue(issued);
   }
-
-  // Rotate the G queries of this KV head once, q~ = R_K q, while the first
-  // blocks stream in; padded heads stay zero.
-  for (int i = tid; i < GP * D; i += kI8Threads) {
-    const int gq = i / D;
-    float v = 0.f;
-    if (gq < G) {
-      const __half *qp = static_cast<const __half *>(a.q) +
-                         (static_cast<long long>(b) * a.hq + kvh * G + gq) * D;
-      v = __half2float(qp[i % D]);
-    }
-    scratch[i] = v;
-  }
-  __syncthreads();
-  rotate_forward_smem<D, FULL>(scratch, G, a.params_k + static_cast<size_t>(kvh) * 2 * D, tid,
-                               kI8Threads, 0);
-  // Per-head fixed-point step of the query: max|q~_h| / kQueryIntMax.
-  for (int h = warp; h < 8; h += kI8Warps) {
-    float mx = 0.f;
-    if (h < G)
-      for (int i = lane; i < D; i += 32) mx = fmaxf(mx, fabsf(scratch[h * D + i]));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) qinv[h] = mx / static_cast<float>(kQueryIntMax);
-  }
-  __syncthreads();
+  __syncwarp();   // the other lanes wait on the barriers lane 0 initialised
 
   const int g = lane >> 2, t = lane & 3;
 
-  // B fragments of the fixed-point query Q = rint(q~ / qinv) =
-  // 2^14 Qh + 2^7 Qm + Ql: tile nq, column g = (head, part), dims of quads
-  // 2kk, 2kk+1 of lane t.  Part p of head h sits in tile 0, column p GP + h
-  // (GP <= 2); tile 0, column 4p + h for p < 2 and tile 1, column h for p = 2
-  // (GP = 4); tile p, column h (GP = 8).
+  // B fragments of the fixed-point query and the per-head score factors,
+  // prepared once per (b, kvh) by prep_i8_kernel.
+  const uint32_t *qp = a.ws_qprep + pair * C::QPREP_WORDS;
   uint32_t qb[C::NQ][C::KK][2];
 #pragma unroll
-  for (int nq = 0; nq < C::NQ; ++nq) {
-    int head, part;
-    if constexpr (GP <= 2) {
-      part = g / GP;
-      head = g % GP;
-    } else if constexpr (GP == 4) {
-      part = nq == 0 ? (g >> 2) : (g < 4 ? 2 : 3);
-      head = g & 3;
-    } else {
-      part = nq;
-      head = g;
-    }
-    const bool live = part < 3 && head < G;
-    const float qi = live ? qinv[head] : 0.f;
-    const float qs = qi > 0.f ? 1.f / qi : 0.f;
+  for (int nq = 0; nq < C::NQ; ++nq)
 #pragma unroll
-    for (int kk = 0; kk < C::KK; ++kk) {
-      const int grp = (D == 256 ? 2 * t : t) + kk / 4;
+    for (int kk = 0; kk < C::KK; ++kk)
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int base = 32 * grp + 4 * (2 * (kk & 3) + half);
-        int v[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int q = live ? __float2int_rn(scratch[head * D + base + i] * qs) : 0;
-          q = q > kQueryIntMax ? kQueryIntMax : (q < -kQueryIntMax ? -kQueryIntMax : q);
-          const int r1 = (q + 64) >> 7, ql = q - 128 * r1;     // arithmetic shifts: floor
-          const int r2 = (r1 + 64) >> 7, qm = r1 - 128 * r2;
-          v[i] = part == 0 ? r2 : (part == 1 ? qm : ql);
-        }
-        qb[nq][kk][half] = pack_s8x4(v[0], v[1], v[2], v[3]);
-      }
-    }
-  }
+      for (int half = 0; half < 2; ++half) qb[nq][kk][half] = qp[((nq * C::KK + kk) * 2 + half) * 32 + lane];
   const bool real0 = 2 * t < G, real1 = 2 * t + 1 < G;
-  const float qk0 = real0 ? qinv[2 * t] * score_unit : 0.f;
-  const float qk1 = real1 ? qinv[2 * t + 1] * score_unit : 0.f;
+  const float qk0 = __uint_as_float(qp[3 * C::KK * 2 * 32 + 2 * t]);       // 0 for padded heads
+  const float qk1 = __uint_as_float(qp[3 * C::KK * 2 * 32 + 2 * t + 1]);
 
   // prmt selectors that move byte k of a packed (W_a, W_b) word to byte g&3
   // of a PV B register (zeros elsewhere): lo / hi byte of head parity g>>2.
@@ -706,7 +726,9 @@ int launch_split_i8(const SplitArgs &a, cudaStream_t stream) {
   const float score_unit = static_cast<float>(a.scale * unit * 1.4426950408889634);
   const float out_scale = static_cast<float>(unit);
   dim3 grid(a.n_splits, a.hkv, a.batch);
-  kernel<<<grid, kI8Threads, C::SMEM, stream>>>(a, tb.lut, score_unit, out_scale);
+  static_assert(C::QPREP_WORDS == decode_qprep_words(D), "prepared-query layout");
+  prep_i8_kernel<D, FULL, GP><<<dim3(a.hkv, a.batch), kI8Threads, 0, stream>>>(a, score_unit);
+  kernel<<<grid, kI8Threads, C::SMEM, stream>>>(a, tb.lut, out_scale);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode i8 launch: %s", cudaGetErrorString(e));
   return ISOQ_OK;

@@ -36,5 +36,10 @@ bool codebook_unit_f64(int bits, double *centroids);
 constexpr int kDecodeTokenQuantum = 64;   // chunk sizes are multiples of this
 int64_t decode_chunk_tokens(int B, int Hkv, int64_t Tmax, int d);
 int decode_num_splits(int B, int Hkv, int64_t Tmax, int d);
+// Per (b, kvh): the prepared query of the int8 decode path, as the B-fragment
+// words of up to 3 N tiles x d/32 k-steps x 2 halves x 32 lanes, then 8
+// per-head score factors (float32).
+constexpr int decode_qprep_words(int d) { return 3 * (d / 32) * 2 * 32 + 8; }
+size_t decode_qprep_bytes(int B, int Hkv, int d);
 
 }  // namespace isoq

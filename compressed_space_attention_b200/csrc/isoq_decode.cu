@@ -385,9 +385,15 @@ int validate_common(int dtype, int B, int Hq, int Hkv, int64_t Tmax, int d, int 
   return ISOQ_OK;
 }
 
-void workspace_views(void *ws, int B, int Hq, int n_splits, int d, float **acc, float2 **ml) {
+void workspace_views(void *ws, int B, int Hq, int n_splits, int d, float **acc, float2 **ml,
+                     uint32_t **qprep = nullptr) {
   *acc = static_cast<float *>(ws);
   *ml = reinterpret_cast<float2 *>(static_cast<float *>(ws) + static_cast<size_t>(B) * Hq * n_splits * d);
+  if (qprep) {
+    size_t n = static_cast<size_t>(B) * Hq * n_splits * (d + 2) * 4;
+    n = (n + 255) / 256 * 256;
+    *qprep = reinterpret_cast<uint32_t *>(static_cast<unsigned char *>(ws) + n);
+  }
 }
 
 }  // namespace decode
@@ -431,7 +437,7 @@ int isoq_decode_split(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
   a.chunk = decode_chunk_tokens(B, Hkv, Tmax, d);
   a.n_splits = decode_num_splits(B, Hkv, Tmax, d);
   a.scale = scale;
-  decode::workspace_views(workspace_dev, B, Hq, a.n_splits, d, &a.ws_acc, &a.ws_ml);
+  decode::workspace_views(workspace_dev, B, Hq, a.n_splits, d, &a.ws_acc, &a.ws_ml, &a.ws_qprep);
   CodebookF32 cb;
   codebook_f32(d, bits, &cb);
   for (int j = 0; j < 16; ++j) a.centroid[j] = j < cb.levels ? cb.centroid[j] : 0.f;

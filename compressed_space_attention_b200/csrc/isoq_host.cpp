@@ -178,6 +178,11 @@ int64_t decode_chunk_tokens(int B, int Hkv, int64_t Tmax, int d) {
   return chunk;
 }
 
+size_t decode_qprep_bytes(int B, int Hkv, int d) {
+  const size_t n = static_cast<size_t>(B) * Hkv * decode_qprep_words(d) * 4;
+  return (n + 255) / 256 * 256;
+}
+
 int decode_num_splits(int B, int Hkv, int64_t Tmax, int d) {
   int64_t chunk = decode_chunk_tokens(B, Hkv, Tmax, d);
   int64_t n = (Tmax + chunk - 1) / chunk;
@@ -270,7 +275,8 @@ int isoq_decode_num_splits(int B, int Hkv, int64_t Tmax, int d) {
 size_t isoq_decode_workspace_size(int B, int Hq, int Hkv, int64_t Tmax, int d) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tmax <= 0 || !supported_d(d) || Hq % Hkv) return 0;
   size_t n = static_cast<size_t>(B) * Hq * decode_num_splits(B, Hkv, Tmax, d) * (d + 2) * 4;
-  return (n + 255) / 256 * 256;
+  n = (n + 255) / 256 * 256;
+  return n + decode_qprep_bytes(B, Hkv, d);
 }
 
 }  // extern "C"

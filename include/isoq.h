@@ -156,9 +156,10 @@ int isoq_dequantize(const uint8_t *codes_dev, const uint16_t *norms_dev, int n_h
 int isoq_decode_num_splits(int B, int Hkv, int64_t Tmax, int d);
 
 /*
- * Bytes of device workspace isoq_decode_attention needs:
- * B * Hq * n_splits * (d + 2) * 4, rounded up to 256.  Returns 0 on invalid
- * shapes.
+ * Bytes of device workspace isoq_decode_attention needs: the split-K partial
+ * states, B * Hq * n_splits * (d + 2) * 4 rounded up to 256, then the
+ * prepared queries, B * Hkv * (24 d + 32) rounded up to 256.  Returns 0 on
+ * invalid shapes.
  */
 size_t isoq_decode_workspace_size(int B, int Hq, int Hkv, int64_t Tmax, int d);
 
