@@ -312,7 +312,6 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     for (int kk = 0; kk < C::KK; ++kk)
 #pragma unroll
       for (int half = 0; half < 2; ++half) qb[nq][kk][half] = qp[((nq * C::KK + kk) * 2 + half) * 32 + lane];
-  const bool real0 = 2 * t < G, real1 = 2 * t + 1 < G;
   const float qk0 = __uint_as_float(qp[3 * C::KK * 2 * 32 + 2 * t]);       // 0 for padded heads
   const float qk1 = __uint_as_float(qp[3 * C::KK * 2 * 32 + 2 * t + 1]);
 
@@ -457,9 +456,10 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
         const float svr = lds_half(nv + 2 * j);
         sv[T][hh] = ok ? svr : 0.f;
         vmx = fmaxf(vmx, sv[T][hh]);
-        // Padded heads hold a constant 0 so that they never move the maximum.
-        x[T][2 * hh] = real0 ? (ok ? sc[T][2 * hh] * sk * qk0 : -INFINITY) : 0.f;
-        x[T][2 * hh + 1] = real1 ? (ok ? sc[T][2 * hh + 1] * sk * qk1 : -INFINITY) : 0.f;
+        // Padded heads (qk = 0) score 0 and never move a maximum; their
+        // weights only reach accumulators that are never stored.
+        x[T][2 * hh] = ok ? sc[T][2 * hh] * sk * qk0 : -INFINITY;
+        x[T][2 * hh + 1] = ok ? sc[T][2 * hh + 1] * sk * qk1 : -INFINITY;
         mx0 = fmaxf(mx0, x[T][2 * hh]);
         mx1 = fmaxf(mx1, x[T][2 * hh + 1]);
       }
@@ -506,8 +506,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
         l0 += p0;
         l1 += p1;
         const float w = sv[T][hh] * wsc;
-        const float wq0 = real0 ? fmaf(p0, w, 8388608.f) : 8388608.f;
-        const float wq1 = real1 ? fmaf(p1, w, 8388608.f) : 8388608.f;
+        const float wq0 = fmaf(p0, w, 8388608.f), wq1 = fmaf(p1, w, 8388608.f);
         u[T][hh] = pack_lo16(__float_as_uint(wq0), __float_as_uint(wq1));
       }
     }
