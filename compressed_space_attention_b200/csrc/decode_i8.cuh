@@ -444,36 +444,47 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     }
 
     // ---- softmax bookkeeping (log2 domain) ----
+    // x[T][e]: token 16T + 8(e >> 1) + g, head 2t + (e & 1).  Padded heads
+    // (qk = 0) score 0 and never move a maximum; their weights only reach
+    // accumulators that are never stored.
     float x[2][4], sv[2][2];
-    float mx0 = -INFINITY, mx1 = -INFINITY, vmx = 0.f;
 #pragma unroll
     for (int T = 0; T < 2; ++T) {
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int j = 16 * T + 8 * hh + g;
-        const bool ok = j < nvalid;
         const float sk = lds_half(nk + 2 * j);
-        const float svr = lds_half(nv + 2 * j);
-        sv[T][hh] = ok ? svr : 0.f;
-        vmx = fmaxf(vmx, sv[T][hh]);
-        // Padded heads (qk = 0) score 0 and never move a maximum; their
-        // weights only reach accumulators that are never stored.
-        x[T][2 * hh] = ok ? sc[T][2 * hh] * sk * qk0 : -INFINITY;
-        x[T][2 * hh + 1] = ok ? sc[T][2 * hh + 1] * sk * qk1 : -INFINITY;
-        mx0 = fmaxf(mx0, x[T][2 * hh]);
-        mx1 = fmaxf(mx1, x[T][2 * hh + 1]);
+        sv[T][hh] = lds_half(nv + 2 * j);
+        x[T][2 * hh] = sc[T][2 * hh] * sk * qk0;
+        x[T][2 * hh + 1] = sc[T][2 * hh + 1] * sk * qk1;
       }
     }
+    if (nvalid < kBlk) {   // the chunk's partial last block (warp-uniform)
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
+      for (int T = 0; T < 2; ++T) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const bool ok = 16 * T + 8 * hh + g < nvalid;
+          sv[T][hh] = ok ? sv[T][hh] : 0.f;
+          x[T][2 * hh] = ok ? x[T][2 * hh] : -INFINITY;
+          x[T][2 * hh + 1] = ok ? x[T][2 * hh + 1] : -INFINITY;
+        }
+      }
     }
     // Move the references only when this block would leave the fixed-point
-    // range: a score above m_ref + 1 or a V norm above s_ref.
-    const bool ev0 = mx0 > m0 + 1.f, ev1 = mx1 > m1 + 1.f, evs = vmx > s_ref;
-    if (__any_sync(0xffffffffu, ev0 || ev1 || evs)) {
+    // range: a score above m_ref + 1 or a V norm above s_ref.  Lane-local
+    // maxima decide; the warp-wide ones are only formed when a lane objects.
+    float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+    float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+    float vmx = fmaxf(fmaxf(sv[0][0], sv[0][1]), fmaxf(sv[1][0], sv[1][1]));
+    if (__any_sync(0xffffffffu, mx0 > m0 + 1.f || mx1 > m1 + 1.f || vmx > s_ref)) {
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
+      }
+      const bool ev0 = mx0 > m0 + 1.f, ev1 = mx1 > m1 + 1.f, evs = vmx > s_ref;
       const float mn0 = ev0 ? mx0 : m0, mn1 = ev1 ? mx1 : m1;
       const float f0 = ex2f(m0 - mn0), f1 = ex2f(m1 - mn1);   // 0 on the first block
       const float sn = evs ? vmx * kNormHeadroom : s_ref;
