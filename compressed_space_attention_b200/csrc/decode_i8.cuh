@@ -34,13 +34,17 @@
 // one prmt lookup produces.  W = p s^V is block-scaled per 16-token slab and
 // head to 16 bits, W = 256 Wh + Wl (u8 parts); C W = 2^15 Ch Wh +
 // 2^7 (Ch Wl + 2 Cl Wh) + Cl Wl, of which the last term (below 2^-15 of one
-// token's largest contribution) is dropped.  W is fixed-point against a
-// per-warp reference, W_q = rint(p s^V 32000 / s_ref) with p = 2^(x - m_ref)
-// <= 2 and s^V <= s_ref, so the two int32 sums accumulate across the whole
-// chunk; they are rescaled only when a block's maximum score
-// passes m_ref + 1 or a V norm passes s_ref, which after the first block is
-// rare.  The pair (m_ref, l) it leaves is a valid partial state: l and acc
-// are both relative to 2^m_ref.
+// token's largest contribution) is dropped.  W is fixed-point against the
+// largest p s^V of its 32-token block and head, W_q = rint(p s^V 64000 /
+// max_block(p s^V)) with p = 2^(x - m_ref): every block keeps 16 bits
+// relative to its own largest weight, so a block of small weights next to
+// one dominant token (an attention sink) loses nothing to the dominant
+// token's scale.  The int32 sums of each 16-token half are converted once
+// and added into float32 accumulators with the block's scale; m_ref moves
+// (and l and the accumulators are rescaled) only when a block's maximum
+// score passes m_ref + 1, which after the first block is rare.  The pair
+// (m_ref, l) it leaves is a valid partial state: l and acc are both relative
+// to 2^m_ref.
 //
 // Fragment orders.  A fixed permutation of the rotated coordinates cancels in
 // q~.k~ and is undone when the accumulator is written out:
@@ -67,8 +71,7 @@ constexpr int kBlk = 32;                 // tokens per ring stage (two 16-token 
 constexpr int kI8Stages = 2;             // per-warp ring depth
 constexpr int kCentroidIntMax = 16319;   // |C_k| bound that keeps Ch, 2 Cl in int8
 constexpr int kQueryIntMax = 2088000;    // |Q| bound that keeps Qh, Qm, Ql in int8
-constexpr float kWScale = 32000.f;       // W_q = rint(p s^V kWScale / s_ref), p <= 2
-constexpr float kNormHeadroom = 1.25f;   // s_ref = 1.25 x the largest V norm seen
+constexpr float kWMax = 64000.f;         // W_q = rint(p s^V kWMax / max_block(p s^V)) < 2^16
 
 template <int D, int GP>
 struct I8Cfg {
@@ -120,13 +123,22 @@ __device__ __forceinline__ void mma_s8s8_z(int (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// c += A B (s8 x u8).
+// c += A B (s8 x u8), and the same with a zero accumulator.
 __device__ __forceinline__ void mma_s8u8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_s8u8_z(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                           uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{0,0,0,0};"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
@@ -158,13 +170,6 @@ __device__ __forceinline__ uint32_t pack_s8x4(int v0, int v1, int v2, int v3) {
          ((static_cast<uint32_t>(v2) & 0xFFu) << 16) | ((static_cast<uint32_t>(v3) & 0xFFu) << 24);
 }
 
-// E <- rint(E F) for one pair of int32 sums representing 256 E1 + E2 (F <= 1;
-// the fraction of E1 F that is dropped is below 2^-15 of one token's largest
-// contribution).
-__device__ __forceinline__ void rescale_pair(int &e1, int &e2, float f) {
-  e1 = __float2int_rn(static_cast<float>(e1) * f);
-  e2 = __float2int_rn(static_cast<float>(e2) * f);
-}
 
 // Query preparation, one CTA per (b, kvh): rotate the G queries once,
 // q~ = R_K q, and write for every lane of the split kernel the B-fragment
@@ -322,19 +327,18 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
   const uint32_t sel_lo = (0x4444u & ~(0xFu << r4)) | (hpb << r4);
   const uint32_t sel_hi = (0x4444u & ~(0xFu << r4)) | ((hpb + 1u) << r4);
 
-  // PV sums 256 E1 + E2 (int32, whole chunk) in the PV layout: head
-  // 2nv + (t >> 1).
-  int e1[C::NV][C::MB][4], e2[C::NV][C::MB][4];
+  // PV accumulators sum p s^V C (float32, whole chunk, relative to
+  // 2^m_ref) in the PV layout: head 2nv + (t >> 1).
+  float acc[C::NV][C::MB][4];
 #pragma unroll
   for (int nvt = 0; nvt < C::NV; ++nvt)
 #pragma unroll
     for (int mb = 0; mb < C::MB; ++mb)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) e1[nvt][mb][e] = e2[nvt][mb][e] = 0;
+      for (int e = 0; e < 4; ++e) acc[nvt][mb][e] = 0.f;
   // Softmax state in the QK layout (heads 2t, 2t+1; log2 domain): reference
-  // maximum and sum; the V-norm reference is warp-uniform.
+  // maximum and sum.
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  float s_ref = 0.f, wsc = 0.f;
 
   int consumed = 0;
   bool failed = false;
@@ -471,44 +475,35 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
         }
       }
     }
-    // Move the references only when this block would leave the fixed-point
-    // range: a score above m_ref + 1 or a V norm above s_ref.  Lane-local
-    // maxima decide; the warp-wide ones are only formed when a lane objects.
+    // Move the reference maximum only when a score passes m_ref + 1.
+    // Lane-local maxima decide; the warp-wide ones are only formed when a
+    // lane objects.
     float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
     float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
-    float vmx = fmaxf(fmaxf(sv[0][0], sv[0][1]), fmaxf(sv[1][0], sv[1][1]));
-    if (__any_sync(0xffffffffu, mx0 > m0 + 1.f || mx1 > m1 + 1.f || vmx > s_ref)) {
+    if (__any_sync(0xffffffffu, mx0 > m0 + 1.f || mx1 > m1 + 1.f)) {
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-        vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
       }
-      const bool ev0 = mx0 > m0 + 1.f, ev1 = mx1 > m1 + 1.f, evs = vmx > s_ref;
-      const float mn0 = ev0 ? mx0 : m0, mn1 = ev1 ? mx1 : m1;
+      const float mn0 = mx0 > m0 + 1.f ? mx0 : m0, mn1 = mx1 > m1 + 1.f ? mx1 : m1;
       const float f0 = ex2f(m0 - mn0), f1 = ex2f(m1 - mn1);   // 0 on the first block
-      const float sn = evs ? vmx * kNormHeadroom : s_ref;
-      const float ratio = sn > 0.f ? s_ref / sn : 0.f;
       l0 *= f0;
       l1 *= f1;
       m0 = mn0;
       m1 = mn1;
-      s_ref = sn;
-      wsc = sn > 0.f ? kWScale / sn : 0.f;
 #pragma unroll
       for (int nvt = 0; nvt < C::NV; ++nvt) {
         const float fa = __shfl_sync(0xffffffffu, f0, nvt), fb = __shfl_sync(0xffffffffu, f1, nvt);
-        const float F = ((t >> 1) ? fb : fa) * ratio;
+        const float F = (t >> 1) ? fb : fa;
 #pragma unroll
         for (int mb = 0; mb < C::MB; ++mb)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) rescale_pair(e1[nvt][mb][e], e2[nvt][mb][e], F);
+          for (int e = 0; e < 4; ++e) acc[nvt][mb][e] *= F;
       }
     }
-    // p = 2^(x - m_ref) <= 2; W_q = rint(p s^V kWScale / s_ref) < 2^16 from the
-    // low 16 bits of p s^V wsc + 2^23.  u[T][hh]: (W head 2t, W head 2t+1) of
-    // token 16T + 8hh + g.
-    uint32_t u[2][2];
+    // p = 2^(x - m_ref) <= 2 and the block's largest p s^V per head.
+    float pw[2][4], pm0 = 0.f, pm1 = 0.f;
 #pragma unroll
     for (int T = 0; T < 2; ++T) {
 #pragma unroll
@@ -516,10 +511,36 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
         const float p0 = ex2f(x[T][2 * hh] - m0), p1 = ex2f(x[T][2 * hh + 1] - m1);
         l0 += p0;
         l1 += p1;
-        const float w = sv[T][hh] * wsc;
-        const float wq0 = fmaf(p0, w, 8388608.f), wq1 = fmaf(p1, w, 8388608.f);
+        pw[T][2 * hh] = p0 * sv[T][hh];
+        pw[T][2 * hh + 1] = p1 * sv[T][hh];
+        pm0 = fmaxf(pm0, pw[T][2 * hh]);
+        pm1 = fmaxf(pm1, pw[T][2 * hh + 1]);
+      }
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, o));
+      pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, o));
+    }
+    // W_q = rint(p s^V kWMax / pm) <= kWMax from the low 16 bits of
+    // p s^V r + 2^23; one unit of 256 E1 + E2 is then 2^7 pm / kWMax of
+    // sum p s^V C (dinv, in the PV layout).  u[T][hh]: (W head 2t, W head
+    // 2t+1) of token 16T + 8hh + g.
+    const float r0 = pm0 > 0.f ? kWMax / pm0 : 0.f, r1 = pm1 > 0.f ? kWMax / pm1 : 0.f;
+    uint32_t u[2][2];
+#pragma unroll
+    for (int T = 0; T < 2; ++T) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const float wq0 = fmaf(pw[T][2 * hh], r0, 8388608.f), wq1 = fmaf(pw[T][2 * hh + 1], r1, 8388608.f);
         u[T][hh] = pack_lo16(__float_as_uint(wq0), __float_as_uint(wq1));
       }
+    }
+    float dinv[C::NV];
+#pragma unroll
+    for (int nvt = 0; nvt < C::NV; ++nvt) {
+      const float da = __shfl_sync(0xffffffffu, pm0, nvt), db = __shfl_sync(0xffffffffu, pm1, nvt);
+      dinv[nvt] = ((t >> 1) ? db : da) * (128.f / kWMax);
     }
 
     // ---- PV, per 16-token half: this lane's tokens t, t+4, t+8, t+12 ----
@@ -572,12 +593,17 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
         }
 #pragma unroll
         for (int nvt = 0; nvt < C::NV; ++nvt) {
-          mma_s8u8(e1[nvt][mb], ah[0][0], ah[0][1], ah[1][0], ah[1][1], bh[nvt][0][0], bh[nvt][0][1]);
-          mma_s8u8(e1[nvt][mb], ah[2][0], ah[2][1], ah[3][0], ah[3][1], bh[nvt][1][0], bh[nvt][1][1]);
-          mma_s8u8(e2[nvt][mb], ah[0][0], ah[0][1], ah[1][0], ah[1][1], bl[nvt][0][0], bl[nvt][0][1]);
-          mma_s8u8(e2[nvt][mb], ah[2][0], ah[2][1], ah[3][0], ah[3][1], bl[nvt][1][0], bl[nvt][1][1]);
-          mma_s8u8(e2[nvt][mb], al[0][0], al[0][1], al[1][0], al[1][1], bh[nvt][0][0], bh[nvt][0][1]);
-          mma_s8u8(e2[nvt][mb], al[2][0], al[2][1], al[3][0], al[3][1], bh[nvt][1][0], bh[nvt][1][1]);
+          // This half's sums: |256 E1 + E2| < 16 x 2^15 x 255 < 2^31.
+          int e1[4], e2[4];
+          mma_s8u8_z(e1, ah[0][0], ah[0][1], ah[1][0], ah[1][1], bh[nvt][0][0], bh[nvt][0][1]);
+          mma_s8u8(e1, ah[2][0], ah[2][1], ah[3][0], ah[3][1], bh[nvt][1][0], bh[nvt][1][1]);
+          mma_s8u8_z(e2, ah[0][0], ah[0][1], ah[1][0], ah[1][1], bl[nvt][0][0], bl[nvt][0][1]);
+          mma_s8u8(e2, ah[2][0], ah[2][1], ah[3][0], ah[3][1], bl[nvt][1][0], bl[nvt][1][1]);
+          mma_s8u8(e2, al[0][0], al[0][1], al[1][0], al[1][1], bh[nvt][0][0], bh[nvt][0][1]);
+          mma_s8u8(e2, al[2][0], al[2][1], al[3][0], al[3][1], bh[nvt][1][0], bh[nvt][1][1]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            acc[nvt][mb][e] = fmaf(static_cast<float>(256 * e1[e] + e2[e]), dinv[nvt], acc[nvt][mb][e]);
         }
       }
     }
@@ -611,10 +637,8 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
   }
   __syncthreads();
   // Merge the warps' accumulators into scratch[head][dim] (rotated domain),
-  // one warp after the other so that the sum order is fixed.  One unit of
-  // 256 E1 + E2 is 2^7 s_ref / kWScale of sum p s^V C.
+  // one warp after the other so that the sum order is fixed.
   {
-    const float unit = s_ref * (128.f / kWScale);
     const int grp = D == 256 ? g : (g >> 1);
     const int qoff = D == 256 ? 0 : 4 * (g & 1);
     float f[C::NV];
@@ -624,7 +648,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
       float mstar = -INFINITY;
       for (int w2 = 0; w2 < kI8Warps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
       const float mine = wm[warp * 8 + h];
-      f[nvt] = (mine == -INFINITY) ? 0.f : exp2f(mine - mstar) * unit;
+      f[nvt] = (mine == -INFINITY) ? 0.f : exp2f(mine - mstar);
     }
     for (int w2 = 0; w2 < kI8Warps; ++w2) {
       if (warp == w2) {
@@ -638,8 +662,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
               for (int e = 0; e < 4; ++e) {
                 const int dim = 32 * grp + 4 * (2 * mb + (e >> 1) + qoff) + 2 * (t & 1) + (e & 1);
                 float *dst = scratch + h * D + dim;
-                const float v = fmaf(static_cast<float>(e1[nvt][mb][e]), 256.f,
-                                     static_cast<float>(e2[nvt][mb][e])) * f[nvt];
+                const float v = acc[nvt][mb][e] * f[nvt];
                 *dst = (w2 == 0) ? v : *dst + v;
               }
             }
@@ -744,9 +767,9 @@ int launch_split_i8(const SplitArgs &a, cudaStream_t stream) {
   return ISOQ_OK;
 }
 
-// The int32 PV sums of a warp stay below 2^31 for up to 2^16 tokens per warp
-// (|Ch Wh| <= 128 * 255, |Ch Wl + 2 Cl Wh| <= 2 * 128 * 255 per token).
-bool i8_path_supported(const SplitArgs &a) { return a.chunk <= 4LL * kI8Warps * 16384; }
+// The int32 PV sums cover 16 tokens and the QK sums one token, so any chunk
+// length is in range.
+bool i8_path_supported(const SplitArgs &) { return true; }
 
 template <int D, bool FULL>
 int run_split_i8_d(const SplitArgs &a, cudaStream_t st) {

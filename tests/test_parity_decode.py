@@ -206,3 +206,36 @@ def test_scale_argument_is_used():
         ref = O.decode_attention(q, pk, pv, nk, nv, [256], prk, prv, 3, O.FULL, scale)
         got = _gpu_decode(q, pk, pv, nk, nv, [256], prk, prv, 3, O.FULL, scale)
         check_attention(got, ref, np.float16)
+
+
+@pytest.mark.parametrize("d,hq,hkv", [(128, 32, 4), (256, 16, 8)])
+def test_attention_sink_with_small_value_norm(d, hq, hkv):
+    """One dominant token (its score 12 nats above every other) whose V norm
+    is 40 times below the others', as attention sinks often are, among 700
+    tokens: the other tokens' small weights must still be accumulated to the
+    float16 tolerance, not rounded away against the sink's scale."""
+    b, t, bits = 2, 700, 3
+    k, v = synth.student_t_kv(hkv, t, d, seed=71, batch=b)
+    prk = O.make_params(d, O.FULL, seed=1, n_heads=hkv)
+    prv = O.make_params(d, O.FULL, seed=2, n_heads=hkv)
+    pk, nk = O.quantize(k.reshape(b * hkv, t, d).astype(np.float64), np.tile(prk, (b, 1, 1)), bits, O.FULL)
+    pv, nv = O.quantize(v.reshape(b * hkv, t, d).astype(np.float64), np.tile(prv, (b, 1, 1)), bits, O.FULL)
+    pb = d * bits // 8
+    pk, pv = pk.reshape(b, hkv, t, pb), pv.reshape(b, hkv, t, pb)
+    nk, nv = nk.reshape(b, hkv, t), nv.reshape(b, hkv, t)
+    sink = [3, 450]
+    scale = 1 / math.sqrt(d)
+    q = np.empty((b, hq, d), dtype=np.float16)
+    for bb in range(b):
+        nv[bb, :, sink[bb]] = (nv[bb, :, sink[bb]].astype(np.float64) / 40).astype(np.float16)
+        for kvh in range(hkv):
+            khat = O.dequantize(pk[bb, kvh:kvh + 1], nk[bb, kvh:kvh + 1], prk[kvh:kvh + 1], bits, O.FULL, d)[0]
+            k0 = khat[sink[bb]]
+            others = np.delete(khat, sink[bb], axis=0) @ k0
+            alpha = 12.0 / (scale * (k0 @ k0 - others.max()))
+            for g in range(hq // hkv):
+                q[bb, kvh * (hq // hkv) + g] = (alpha * (1.0 + 0.05 * g) * k0).astype(np.float16)
+    lens = [t, t]
+    ref = O.decode_attention(q, pk, pv, nk, nv, lens, prk, prv, bits, O.FULL, scale)
+    got = _gpu_decode(q, pk, pv, nk, nv, lens, prk, prv, bits, O.FULL, scale)
+    check_attention(got, ref, np.float16)
