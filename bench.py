@@ -42,7 +42,6 @@ sys.path.insert(0, ROOT)
 METRIC = "packed-3-bit decode attn KV GB/s (% of HBM peak); quantize Mvec/s"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["compressed_space_attention_b200/csrc/isoq_decode.cu",
-                  "compressed_space_attention_b200/csrc/decode_mma.cuh",
                   "compressed_space_attention_b200/csrc/decode_i8.cuh",
                   "compressed_space_attention_b200/csrc/common.cuh"]
 TRAFFIC_PROFILE = "profiles/decode_split_b32_gqa16_8_d256_t65536.md"
@@ -456,9 +455,37 @@ def run_isoq(args):
     if dist:
         dist.barrier()
 
+    # ---- decode-step append, then the whole step (append + attention) ----
+    # Timed after the main region on rows set to half their capacity, so the
+    # appended positions never reach Tmax; the cache contents past the
+    # original lengths do not affect the numbers above.
+    kn = synth.queries_torch(B, Hkv, d, seed=seed0 + 21, device=dev)
+    vn = synth.queries_torch(B, Hkv, d, seed=seed0 + 22, device=dev)
+    lens_a = torch.full((B,), T // 2, dtype=torch.int32, device=dev)
+    n_app = max(args.steps, 3)
+    for _ in range(2):
+        isoq.isoq_decode_append(kn, vn, pk, pv, nk, nv, lens_a, prk, prv, bits, variant)
+    torch.cuda.synchronize()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a2 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(n_app):
+        isoq.isoq_decode_append(kn, vn, pk, pv, nk, nv, lens_a, prk, prv, bits, variant)
+    a1.record(stream)
+    for _ in range(n_app):
+        isoq.isoq_decode_step(q, kn, vn, pk, pv, nk, nv, lens_a, prk, prv, bits, variant, out=out,
+                              workspace=ws)
+    a2.record(stream)
+    torch.cuda.synchronize()
+    assert isoq.isoq_check_device_error() == 0
+    t_app = a0.elapsed_time(a1) / n_app
+    t_dstep = a1.elapsed_time(a2) / n_app
+    app_bytes = 2 * B * Hkv * (2 * d + pb + 2)
+
     # ---- reduce over ranks: max time, summed bytes ----
-    total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms = max_over_ranks(
-        [total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms], dist, dev)
+    total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms, t_app, t_dstep = max_over_ranks(
+        [total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms, t_app, t_dstep], dist, dev)
     n_ranks = world
 
     peaks, peak_kind = measured_peaks()
@@ -487,6 +514,12 @@ def run_isoq(args):
         "e2e": {"value": (n_ranks * kv_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9) if e2e_steps else None, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "path": "pinned host cache -> device copy -> isoq_decode_attention -> host copy of the output"},
+        "decode_step": {"append_ms": t_app, "append_gbps": app_bytes / (t_app * 1e-3) / 1e9,
+                        "append_bytes": app_bytes, "step_ms": t_dstep, "launches": n_app,
+                        "what": "isoq_decode_append of one float16 K and V token per (b, kvh) "
+                                "(append_kernel + length advance), and isoq_decode_step = append "
+                                "then decode attention over the cache at half capacity; timed "
+                                "outside the main region"},
         "gpu_launches": 4 * args.steps,
         "clocks": sampler.summary(),
     }

@@ -18,10 +18,12 @@ from .binding import (  # noqa: F401
     IsoqError,
     isoq_abi_version,
     isoq_check_device_error,
+    isoq_decode_append,
     isoq_decode_attention,
     isoq_decode_combine,
     isoq_decode_num_splits,
     isoq_decode_split,
+    isoq_decode_step,
     isoq_decode_workspace_size,
     isoq_dequantize,
     isoq_make_codebook,

@@ -51,6 +51,9 @@ SIGNATURES = [
     ("isoq_decode_split", _I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _P,
                                _F, _P, _SZ, _P]),
     ("isoq_decode_combine", _I, [_I, _P, _I, _I, _I, _I64, _I, _I, _P, _P, _P, _SZ, _P]),
+    ("isoq_decode_append", _I, [_P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _P, _P, _P]),
+    ("isoq_decode_step", _I, [_P, _P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _P, _P,
+                              _F, _P, _P, _SZ, _P]),
     ("isoq_check_device_error", _I, [_P]),
     ("isoq_decode_static_workspace_bytes", _SZ, []),
     ("isoq_decode_attention_static", _I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I,
@@ -270,6 +273,51 @@ def isoq_decode_attention(q, packed_k, packed_v, norms_k, norms_v, seq_lens, par
             float(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
             _stream(dev, stream))
     _check(st, "isoq_decode_attention")
+    return out
+
+
+def isoq_decode_append(k_new, v_new, packed_k, packed_v, norms_k, norms_v, seq_lens, params_k,
+                       params_v, bits: int, variant: int, stream=None):
+    """Compresses k_new/v_new [B][Hkv][d] into the packed cache at seq_lens[b]
+    and advances seq_lens, in place on the device."""
+    B, Hkv, d = k_new.shape
+    _, _, Tmax, pb = packed_k.shape
+    if pb != isoq_packed_bytes(d, bits):
+        raise ValueError("packed row size does not match d and bits")
+    dev = _require_cuda(k_new, v_new, packed_k, packed_v, norms_k, norms_v, seq_lens, params_k,
+                        params_v)
+    torch = _torch()
+    with torch.cuda.device(dev):
+        st = lib().isoq_decode_append(
+            _ptr(k_new), _ptr(v_new), _dtype_code(k_new), _ptr(packed_k), _ptr(packed_v),
+            _ptr(norms_k), _ptr(norms_v), _ptr(seq_lens), B, Hkv, Tmax, d, bits, variant,
+            _ptr(params_k), _ptr(params_v), _stream(dev, stream))
+    _check(st, "isoq_decode_append")
+
+
+def isoq_decode_step(q, k_new, v_new, packed_k, packed_v, norms_k, norms_v, seq_lens, params_k,
+                     params_v, bits: int, variant: int, scale: Optional[float] = None, out=None,
+                     workspace=None, stream=None):
+    """Append (k_new, v_new) to the packed cache, then decode attention of q
+    over it; returns out [B][Hq][d] (dtype of q)."""
+    torch = _torch()
+    B, Hq, Hkv, Tmax, d = _decode_shapes(q, packed_k, bits)
+    dev = _require_cuda(q, k_new, v_new, packed_k, packed_v, norms_k, norms_v, seq_lens, params_k,
+                        params_v, out, workspace)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=q.dtype, device=dev)
+    ws_bytes = isoq_decode_workspace_size(B, Hq, Hkv, Tmax, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().isoq_decode_step(
+            _ptr(q), _ptr(k_new), _ptr(v_new), _dtype_code(q), _ptr(packed_k), _ptr(packed_v),
+            _ptr(norms_k), _ptr(norms_v), _ptr(seq_lens), B, Hq, Hkv, Tmax, d, bits, variant,
+            _ptr(params_k), _ptr(params_v), float(scale), _ptr(out), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(dev, stream))
+    _check(st, "isoq_decode_step")
     return out
 
 

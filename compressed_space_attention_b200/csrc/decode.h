@@ -35,9 +35,7 @@ struct CombineArgs {
   int batch, hq, group, n_splits;
 };
 
-bool mma_path_supported(int dtype, int d, int bits, const SplitArgs &a);
-int run_split_mma(int d, int variant, const SplitArgs &a, cudaStream_t stream);
-bool i8_path_supported(const SplitArgs &a);
+bool i8_path_supported(int dtype, int d, int bits, const SplitArgs &a);
 int run_split_i8(int d, int variant, const SplitArgs &a, cudaStream_t stream);
 
 }  // namespace decode

@@ -1,15 +1,14 @@
 // Integer tensor-core split kernel of the compressed-space decode: float16
 // queries, 3-bit codes, d in {128, 256}, up to 8 query heads per KV head.
-// Included by isoq_decode.cu inside namespace isoq::decode, after
-// decode_mma.cuh (whose slab ring, shared-memory loads and selectors it uses).
+// Included by isoq_decode.cu inside namespace isoq::decode.
 //
 // The work per token is RotaryQuant Table 2 kernels A-C on the packed codes:
 // z_j = s^K_j <q~, c[K_j]> scale, online softmax, acc += p_j s^V_j c[V_j], all
-// in the rotated domain.  What makes this kernel different from the float16
-// one is how a code becomes a tensor-core operand.
+// in the rotated domain, with every code turned into an int8 tensor-core
+// operand by a register lookup.
 //
 // Exact integer centroids.  The unit-variance centroids are scaled by a
-// host-chosen S (about 7,500) so that every C_k = round(S c_k) is within a few
+// host-chosen S (about 6,324) so that every C_k = round(S c_k) is within a few
 // hundredths of S c_k; |C_k| <= 16319 is split as C = 128 Ch + Cl with
 // Ch in [-128, 127] and Cl in [-64, 63].  Each part is an int8 table of 8
 // entries held in two registers, so one prmt turns four codes (a 4-nibble
@@ -94,6 +93,31 @@ struct I8Cfg {
 
 // int8 tables of the centroid parts, four entries per register: kh/kl =
 // (Ch, Cl) for the K side, vh/vl = (Ch, 2 Cl) for the V side.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// Shared-memory loads by explicit shared-window address (no generic LD).
+__device__ __forceinline__ uint32_t lds32(const unsigned char *p) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds64(const unsigned char *p) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
+  return v;
+}
+
+__device__ __forceinline__ float lds_half(const unsigned char *p) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_u32(p)));
+  return __half2float(__ushort_as_half(v));
+}
+
 struct I8Lut {
   uint32_t kh0, kh1, kl0, kl1, vh0, vh1, vl0, vl1;
 };
@@ -767,9 +791,15 @@ int launch_split_i8(const SplitArgs &a, cudaStream_t stream) {
   return ISOQ_OK;
 }
 
-// The int32 PV sums cover 16 tokens and the QK sums one token, so any chunk
-// length is in range.
-bool i8_path_supported(const SplitArgs &) { return true; }
+// Float16 queries, 3-bit codes, d in {128, 256}, G <= 8, and chunks and
+// rows whose bulk copies start on 16-byte boundaries (the int32 PV sums cover
+// 16 tokens and the QK sums one token, so any chunk length is in range).
+bool i8_path_supported(int dtype, int d, int bits, const SplitArgs &a) {
+  return dtype == ISOQ_F16 && bits == 3 && (d == 128 || d == 256) && a.group <= 8 &&
+         a.tmax % 8 == 0 && a.chunk % kDecodeTokenQuantum == 0 &&
+         (reinterpret_cast<uintptr_t>(a.norms_k) & 15u) == 0 &&
+         (reinterpret_cast<uintptr_t>(a.norms_v) & 15u) == 0;
+}
 
 template <int D, bool FULL>
 int run_split_i8_d(const SplitArgs &a, cudaStream_t st) {

@@ -16,8 +16,9 @@
 //            applies R_V^T = H_d R_SO4^T / sqrt(d) and stores the output.
 //
 // This file holds the generic split kernel (CUDA-core FMAs; any dtype, d and
-// bits) and the combine kernel; decode_mma.cuh (included below) holds the
-// tensor-core split kernel used for float16 queries with 3-bit codes.
+// bits) and the combine kernel; decode_i8.cuh (included below) holds the
+// integer tensor-core split kernel used for float16 queries with 3-bit codes,
+// and decode_append.cuh the decode-step append.
 
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -290,8 +291,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
   for (int i = tid; i < D; i += kCombineThreads) out[i] = from_f32<T>(v[i] * inv_sqrt_d);
 }
 
-#include "decode_mma.cuh"
 #include "decode_i8.cuh"
+#include "decode_append.cuh"
 
 // ---------------------------------------------------------------------------
 // Host launchers
@@ -442,9 +443,7 @@ int isoq_decode_split(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
   codebook_f32(d, bits, &cb);
   for (int j = 0; j < 16; ++j) a.centroid[j] = j < cb.levels ? cb.centroid[j] : 0.f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (decode::mma_path_supported(dtype, d, bits, a))
-    return decode::i8_path_supported(a) ? decode::run_split_i8(d, variant, a, s)
-                                        : decode::run_split_mma(d, variant, a, s);
+  if (decode::i8_path_supported(dtype, d, bits, a)) return decode::run_split_i8(d, variant, a, s);
   return decode::run_split_generic(dtype, d, bits, variant, a, s);
 }
 
@@ -502,6 +501,71 @@ __attribute__((visibility("hidden"))) int isoq_detail_take_decode_error(cudaStre
                                 cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   return e == cudaSuccess ? ISOQ_OK : set_error(ISOQ_ERR_CUDA, "error word: %s", cudaGetErrorString(e));
+}
+
+int isoq_decode_append(const void *k_new_dev, const void *v_new_dev, int dtype,
+                       uint8_t *packed_k_dev, uint8_t *packed_v_dev, uint16_t *norms_k_dev,
+                       uint16_t *norms_v_dev, int32_t *seq_lens_dev, int B, int Hkv, int64_t Tmax,
+                       int d, int bits, int variant, const float *params_k_dev,
+                       const float *params_v_dev, isoq_stream_t stream) {
+  clear_error();
+  if (!supported_d(d)) return set_error(ISOQ_ERR_UNSUPPORTED, "d=%d not supported", d);
+  if (!supported_bits(bits)) return set_error(ISOQ_ERR_UNSUPPORTED, "bits=%d not supported", bits);
+  if (!supported_variant(variant)) return set_error(ISOQ_ERR_UNSUPPORTED, "variant=%d", variant);
+  if (!supported_dtype(dtype)) return set_error(ISOQ_ERR_UNSUPPORTED, "dtype=%d", dtype);
+  if (B <= 0 || Hkv <= 0 || Tmax <= 0)
+    return set_error(ISOQ_ERR_INVALID_ARG, "B, Hkv and Tmax must be positive");
+  if (Tmax >= (1ll << 31) || B > 65535 || Hkv > 65535)
+    return set_error(ISOQ_ERR_INVALID_ARG, "shape too large");
+  if (!k_new_dev || !v_new_dev || !packed_k_dev || !packed_v_dev || !norms_k_dev || !norms_v_dev ||
+      !seq_lens_dev || !params_k_dev || !params_v_dev)
+    return set_error(ISOQ_ERR_INVALID_ARG, "null pointer");
+  if (!decode::aligned(packed_k_dev, 16) || !decode::aligned(packed_v_dev, 16) ||
+      !decode::aligned(params_k_dev, 16) || !decode::aligned(params_v_dev, 16) ||
+      !decode::aligned(k_new_dev, 16) || !decode::aligned(v_new_dev, 16) ||
+      !decode::aligned(norms_k_dev, 2) || !decode::aligned(norms_v_dev, 2) || !decode::aligned(seq_lens_dev, 4))
+    return set_error(ISOQ_ERR_UNSUPPORTED, "misaligned pointer");
+  decode::AppendArgs a;
+  a.k_new = k_new_dev;
+  a.v_new = v_new_dev;
+  a.packed_k = packed_k_dev;
+  a.packed_v = packed_v_dev;
+  a.norms_k = norms_k_dev;
+  a.norms_v = norms_v_dev;
+  a.seq_lens = seq_lens_dev;
+  a.params_k = params_k_dev;
+  a.params_v = params_v_dev;
+  a.tmax = Tmax;
+  a.batch = B;
+  a.hkv = Hkv;
+  CodebookF32 cb;
+  codebook_f32(d, bits, &cb);
+  for (int k = 0; k < 15; ++k) a.thr[k] = k < cb.levels - 1 ? cb.threshold[k] : 0.f;
+  return decode::run_append(dtype, d, bits, variant, a, seq_lens_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int isoq_decode_step(const void *q_dev, const void *k_new_dev, const void *v_new_dev, int dtype,
+                     uint8_t *packed_k_dev, uint8_t *packed_v_dev, uint16_t *norms_k_dev,
+                     uint16_t *norms_v_dev, int32_t *seq_lens_dev, int B, int Hq, int Hkv,
+                     int64_t Tmax, int d, int bits, int variant, const float *params_k_dev,
+                     const float *params_v_dev, float scale, void *out_dev, void *workspace_dev,
+                     size_t workspace_bytes, isoq_stream_t stream) {
+  // Every argument of the attention half is checked before the cache is
+  // written, so a rejected call leaves the cache and the lengths as they were.
+  clear_error();
+  int st = decode::validate_common(dtype, B, Hq, Hkv, Tmax, d, variant, workspace_dev, workspace_bytes);
+  if (st) return st;
+  if (!q_dev || !out_dev) return set_error(ISOQ_ERR_INVALID_ARG, "null pointer");
+  if (!decode::aligned(q_dev, 16) || !decode::aligned(out_dev, 16))
+    return set_error(ISOQ_ERR_UNSUPPORTED, "misaligned pointer");
+  if (!std::isfinite(scale)) return set_error(ISOQ_ERR_INVALID_ARG, "scale is not finite");
+  st = isoq_decode_append(k_new_dev, v_new_dev, dtype, packed_k_dev, packed_v_dev, norms_k_dev,
+                          norms_v_dev, seq_lens_dev, B, Hkv, Tmax, d, bits, variant, params_k_dev,
+                          params_v_dev, stream);
+  if (st) return st;
+  return isoq_decode_attention(q_dev, dtype, packed_k_dev, packed_v_dev, norms_k_dev, norms_v_dev,
+                               seq_lens_dev, B, Hq, Hkv, Tmax, d, bits, variant, params_k_dev,
+                               params_v_dev, scale, out_dev, workspace_dev, workspace_bytes, stream);
 }
 
 }  // extern "C"

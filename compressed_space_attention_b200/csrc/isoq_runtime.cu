@@ -16,7 +16,10 @@ extern "C" int isoq_check_device_error(isoq_stream_t stream) {
   if (st) return st;
   st = isoq_detail_take_decode_error(s, &d);
   if (st) return st;
-  if (q | d)
+  // Bit 1: a bounded wait gave up.  Bit 2: a decode append found a full row.
+  if ((q | d) & 1u)
     return isoq::set_error(ISOQ_ERR_TIMEOUT, "device wait timed out (quantize=%u, decode=%u)", q, d);
+  if (d & 2u)
+    return isoq::set_error(ISOQ_ERR_INVALID_ARG, "decode append: a row already held Tmax tokens");
   return ISOQ_OK;
 }

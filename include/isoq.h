@@ -247,10 +247,49 @@ int isoq_decode_attention_static(const void *q_dev, int dtype, const uint8_t *pa
                                  float scale, void *out_dev, isoq_stream_t stream);
 
 /*
+ * Decode-step append ([RQ] §3.2 Algorithm 1 on the new token; Figure 1 and
+ * Appendix D: each decode step compresses its new K/V entry once and writes
+ * it into the packed cache that the fused attention reads).  For every batch
+ * row b and KV head kvh, with p = max(seq_lens[b], 0):
+ *   compress k_new[b][kvh] with params_k[kvh] and v_new[b][kvh] with
+ *   params_v[kvh] (float32 norm, rotation, Lloyd-Max codes against the
+ *   norm-scaled thresholds) into packed_k/v[b][kvh][p] and norms_k/v[b][kvh][p],
+ *   then set seq_lens[b] = p + 1.
+ *   k_new_dev, v_new_dev  [B][Hkv][d] of `dtype`, 16-byte aligned.
+ *   packed_*, norms_*, params_*, seq_lens_dev: the cache and rotations of
+ *                isoq_decode_attention (read and written in place).
+ * A row with p >= Tmax is left unchanged; the next isoq_check_device_error
+ * reports ISOQ_ERR_INVALID_ARG for it.  Argument errors as isoq_quantize.
+ * The bulk compression of an FP16 prefill buffer at the prefill-to-decode
+ * boundary ([RQ] Appendix C) is isoq_quantize on that buffer.
+ */
+int isoq_decode_append(const void *k_new_dev, const void *v_new_dev, int dtype,
+                       uint8_t *packed_k_dev, uint8_t *packed_v_dev, uint16_t *norms_k_dev,
+                       uint16_t *norms_v_dev, int32_t *seq_lens_dev, int B, int Hkv, int64_t Tmax,
+                       int d, int bits, int variant, const float *params_k_dev,
+                       const float *params_v_dev, isoq_stream_t stream);
+
+/*
+ * One decode step: isoq_decode_append of (k_new, v_new), then
+ * isoq_decode_attention of q over the cache including the new token, all on
+ * `stream` (four to five launches, no host synchronisation).  Arguments as
+ * those two functions.  Every argument of both halves is checked before
+ * anything is launched: a call that returns an error status has written
+ * nothing.
+ */
+int isoq_decode_step(const void *q_dev, const void *k_new_dev, const void *v_new_dev, int dtype,
+                     uint8_t *packed_k_dev, uint8_t *packed_v_dev, uint16_t *norms_k_dev,
+                     uint16_t *norms_v_dev, int32_t *seq_lens_dev, int B, int Hq, int Hkv,
+                     int64_t Tmax, int d, int bits, int variant, const float *params_k_dev,
+                     const float *params_v_dev, float scale, void *out_dev, void *workspace_dev,
+                     size_t workspace_bytes, isoq_stream_t stream);
+
+/*
  * Reads and clears the current device's error word after synchronising
  * `stream`.  Returns ISOQ_OK, ISOQ_ERR_TIMEOUT if a kernel's bounded wait
  * gave up since the last check (the kernel then stopped early and its
- * outputs are incomplete), or ISOQ_ERR_CUDA.
+ * outputs are incomplete), ISOQ_ERR_INVALID_ARG if a decode append met a
+ * row that already held Tmax tokens, or ISOQ_ERR_CUDA.
  */
 int isoq_check_device_error(isoq_stream_t stream);
 

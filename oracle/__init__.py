@@ -13,6 +13,7 @@ from .isoquant import (  # noqa: F401
     bitpack,
     bitunpack,
     combine_partials,
+    decode_append,
     decode_attention,
     decode_attention_reconstructed,
     dequantize,

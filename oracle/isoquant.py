@@ -566,6 +566,38 @@ def decode_attention_reconstructed(q, packed_k, packed_v, norms_k, norms_v,
     return out
 
 
+def decode_append(k_new, v_new, packed_k, packed_v, norms_k, norms_v, seq_lens,
+                  params_k, params_v, bits: int, variant: int):
+    """One decode step's cache write ([RQ] Figure 1 and Appendix D: during
+    decode each new K and V entry is compressed once and stored in the packed
+    cache, which attention then reads).
+
+    k_new, v_new: [B][Hkv][d]; cache arrays as in ``decode_attention``.
+    For each batch row b with t = max(seq_lens[b], 0) < Tmax, the new vectors
+    of every KV head are compressed by ``quantize`` (Algorithm 1) and stored
+    at position t, and the row's length becomes t + 1.  A row already
+    holding Tmax tokens is left unchanged and reported.
+    Returns (packed_k, packed_v, norms_k, norms_v, seq_lens, full_rows) as
+    new arrays; full_rows lists the rows that could not take the token.
+    """
+    packed_k, packed_v = np.array(packed_k), np.array(packed_v)
+    norms_k, norms_v = np.array(norms_k), np.array(norms_v)
+    lens = np.array(seq_lens, dtype=np.int64)
+    tmax = packed_k.shape[2]
+    full_rows = []
+    for b in range(lens.shape[0]):
+        t = max(int(lens[b]), 0)
+        if t >= tmax:
+            full_rows.append(b)
+            continue
+        pk, nk = quantize(np.asarray(k_new[b])[:, None, :], params_k, bits, variant)
+        pv, nv = quantize(np.asarray(v_new[b])[:, None, :], params_v, bits, variant)
+        packed_k[b, :, t], norms_k[b, :, t] = pk[:, 0], nk[:, 0]
+        packed_v[b, :, t], norms_v[b, :, t] = pv[:, 0], nv[:, 0]
+        lens[b] = t + 1
+    return packed_k, packed_v, norms_k, norms_v, lens, full_rows
+
+
 def split_partials(z, values, bounds):
     """Split-K partial states of softmax attention for one query row.
 

@@ -137,3 +137,50 @@ def test_binding_rejects_cpu_tensors():
     p = torch.zeros((1, 32, 8))
     with pytest.raises(ValueError, match="CUDA"):
         isoq.isoq_quantize(x, p, 3, isoq.ISOQ_FULL)
+
+
+def test_append_and_step_validation_happens_on_host():
+    lib = isoq.lib()
+    ws = isoq.isoq_decode_workspace_size(1, 8, 2, 64, 128)
+
+    def append(**kw):
+        a = dict(k=256, v=256, dtype=isoq.ISOQ_F16, pk=256, pv=256, nk=256, nv=256, sl=256, B=1,
+                 Hkv=2, Tmax=64, d=128, bits=3, variant=0, prk=256, prv=256)
+        a.update(kw)
+        return lib.isoq_decode_append(a["k"], a["v"], a["dtype"], a["pk"], a["pv"], a["nk"], a["nv"],
+                                      a["sl"], a["B"], a["Hkv"], a["Tmax"], a["d"], a["bits"],
+                                      a["variant"], a["prk"], a["prv"], None)
+
+    assert append(d=96) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert append(bits=5) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert append(variant=3) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert append(dtype=7) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert append(B=0) == isoq.ISOQ_ERR_INVALID_ARG
+    assert append(Tmax=0) == isoq.ISOQ_ERR_INVALID_ARG
+    assert append(Tmax=1 << 31) == isoq.ISOQ_ERR_INVALID_ARG
+    assert append(k=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert append(sl=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert append(prv=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert append(k=256 + 8) == isoq.ISOQ_ERR_UNSUPPORTED               # misaligned
+    assert append(sl=256 + 2) == isoq.ISOQ_ERR_UNSUPPORTED
+
+    def step(**kw):
+        a = dict(q=256, k=256, v=256, dtype=isoq.ISOQ_F16, pk=256, pv=256, nk=256, nv=256, sl=256,
+                 B=1, Hq=8, Hkv=2, Tmax=64, d=128, bits=3, variant=0, prk=256, prv=256, scale=0.088,
+                 out=256, ws=4096, wsb=ws)
+        a.update(kw)
+        return lib.isoq_decode_step(a["q"], a["k"], a["v"], a["dtype"], a["pk"], a["pv"], a["nk"],
+                                    a["nv"], a["sl"], a["B"], a["Hq"], a["Hkv"], a["Tmax"], a["d"],
+                                    a["bits"], a["variant"], a["prk"], a["prv"], a["scale"], a["out"],
+                                    a["ws"], a["wsb"], None)
+
+    # each of these is an attention-half error, caught before the append
+    assert step(Hq=7) == isoq.ISOQ_ERR_INVALID_ARG
+    assert step(wsb=ws - 1) == isoq.ISOQ_ERR_INVALID_ARG
+    assert step(q=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert step(out=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert step(scale=float("inf")) == isoq.ISOQ_ERR_INVALID_ARG
+    assert step(out=256 + 4) == isoq.ISOQ_ERR_UNSUPPORTED
+    # and the append half's own checks
+    assert step(k=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert step(bits=1) == isoq.ISOQ_ERR_UNSUPPORTED

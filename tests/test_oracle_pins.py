@@ -536,6 +536,48 @@ def test_attention_special_cases():
     assert np.max(np.abs(o_rot - a[0, 0])) > 0.1
 
 
+@pytest.mark.parametrize("variant", [O.FULL, O.FAST])
+def test_decode_append_token_by_token_equals_bulk_compression(variant):
+    """RotaryQuant Figure 1 / Appendix D: compressing each decode-step entry
+    on arrival gives the cache that compressing the whole sequence at once
+    gives, at the positions the lengths name; rows already at Tmax stay as
+    they were and are reported; negative lengths count as empty."""
+    g = np.random.default_rng(61)
+    bsz, hkv, tmax, d, bits, steps = 3, 2, 12, 128, 3, 5
+    start = np.array([0, 4, -3])
+    pk0, pv0, nk0, nv0 = _random_cache(g, bsz, hkv, tmax, d, bits)
+    kseq = g.standard_normal((bsz, hkv, steps, d))
+    vseq = g.standard_normal((bsz, hkv, steps, d)) * 3.0
+    prk = O.make_params(d, variant, 1, hkv)
+    prv = O.make_params(d, variant, 2, hkv)
+    cache = (pk0, pv0, nk0, nv0, start)
+    for s in range(steps):
+        *cache, full = O.decode_append(kseq[:, :, s], vseq[:, :, s], *cache, prk, prv, bits, variant)
+        assert full == []
+    pk, pv, nk, nv, lens = cache
+    np.testing.assert_array_equal(lens, np.maximum(start, 0) + steps)
+    for b in range(bsz):
+        t0 = max(start[b], 0)
+        bk, bnk = O.quantize(kseq[b], prk, bits, variant)
+        bv, bnv = O.quantize(vseq[b], prv, bits, variant)
+        np.testing.assert_array_equal(pk[b, :, t0:t0 + steps], bk)
+        np.testing.assert_array_equal(pv[b, :, t0:t0 + steps], bv)
+        np.testing.assert_array_equal(nk[b, :, t0:t0 + steps].view(np.uint16), bnk.view(np.uint16))
+        np.testing.assert_array_equal(nv[b, :, t0:t0 + steps].view(np.uint16), bnv.view(np.uint16))
+        # everything outside the written span is untouched
+        keep = np.ones(tmax, bool)
+        keep[t0:t0 + steps] = False
+        np.testing.assert_array_equal(pk[b][:, keep], pk0[b][:, keep])
+        np.testing.assert_array_equal(nv[b][:, keep].view(np.uint16), nv0[b][:, keep].view(np.uint16))
+    # a full row takes no token
+    out = O.decode_append(kseq[:, :, 0], vseq[:, :, 0], pk, pv, nk, nv, np.array([tmax, 3, tmax + 5]),
+                          prk, prv, bits, variant)
+    assert out[5] == [0, 2]
+    np.testing.assert_array_equal(out[4], [tmax, 4, tmax + 5])
+    np.testing.assert_array_equal(out[0][0], pk[0])
+    np.testing.assert_array_equal(out[0][2], pk[2])
+
+
 def test_split_k_combine_is_partition_independent():
     g = np.random.default_rng(51)
     t, d = 300, 16
