@@ -7,7 +7,11 @@ readings it follows.
 """
 
 from .isoquant import (  # noqa: F401
+    BLOCK_SO4,
     FAST,
+    PLANAR,
+    SO3,
+    VARIANTS,
     FULL,
     SplitMix64,
     bitpack,
@@ -23,6 +27,7 @@ from .isoquant import (  # noqa: F401
     make_codebook,
     make_params,
     packed_bytes,
+    planar_forward,
     qconj,
     quantize,
     quantize_scalar,
@@ -32,6 +37,7 @@ from .isoquant import (  # noqa: F401
     so4_forward,
     so4_inverse,
     split_partials,
+    uses_wht,
     wht,
     wht_op_count,
 )

@@ -56,8 +56,12 @@ import math
 
 import numpy as np
 
-FULL = 0
-FAST = 1
+FULL = 0        # [IQ] IsoQuant-Full, after the WHT ([RQ] v3: R_SO4 o H_d)
+FAST = 1        # [IQ] IsoQuant-Fast: left isoclinic factor only, after the WHT
+PLANAR = 2      # [IQ] the 2-D special case, after the WHT (reading: see make_params)
+BLOCK_SO4 = 3   # [RQ] §4.6 Table 8 v2: block SO(4) (Full map) without the WHT
+SO3 = 4         # [RQ] §4.6 Table 8 v1: single-quaternion conjugation q v conj(q), no WHT
+VARIANTS = (FULL, FAST, PLANAR, BLOCK_SO4, SO3)
 
 _MASK64 = (1 << 64) - 1
 
@@ -121,6 +125,16 @@ def make_params(d: int, variant: int, seed: int, n_heads: int = 1) -> np.ndarray
     normals), then q_R (4 normals).  IsoQuant-Fast ([IQ]) keeps only q_L: its
     q_L equals Full's for the same seed (q_R's draws are still consumed) and
     its q_R slot holds the identity (1, 0, 0, 0).
+
+    Every variant consumes the same eight normals per block:
+      BLOCK_SO4 ([RQ] Table 8 v2) stores Full's pair unchanged;
+      SO3 ([RQ] Table 8 v1, v -> q v conj(q)) stores q_L in both slots;
+      PLANAR ([IQ]'s 2-D special case, a reading: the pages name it without
+      detail) restricts both quaternions to the complex line span{1, i}:
+      q_L = (a0, a1, 0, 0) / |(a0, a1)| from the first two of q_L's normals,
+      q_R likewise from q_R's, so each is uniform on that circle.  For such
+      a pair the block map q_L v conj(q_R) rotates the coordinate pairs
+      (v0, v1) and (v2, v3) of the block independently (see ``planar_forward``).
     """
     if d % 4:
         raise ValueError("d must be a multiple of 4")
@@ -128,10 +142,19 @@ def make_params(d: int, variant: int, seed: int, n_heads: int = 1) -> np.ndarray
     out = np.empty((n_heads, d // 4, 8), dtype=np.float32)
     for h in range(n_heads):
         for i in range(d // 4):
-            ql = _unit4([next(g) for _ in range(4)])
-            qr = _unit4([next(g) for _ in range(4)])
+            a = [next(g) for _ in range(4)]
+            b = [next(g) for _ in range(4)]
+            if variant == PLANAR:
+                ql = _unit4([a[0], a[1], 0.0, 0.0])
+                qr = _unit4([b[0], b[1], 0.0, 0.0])
+            else:
+                ql, qr = _unit4(a), _unit4(b)
+            if variant == FAST:
+                qr = [1.0, 0.0, 0.0, 0.0]
+            elif variant == SO3:
+                qr = ql
             out[h, i, 0:4] = ql
-            out[h, i, 4:8] = qr if variant == FULL else [1.0, 0.0, 0.0, 0.0]
+            out[h, i, 4:8] = qr
     return out
 
 
@@ -279,49 +302,89 @@ def qconj(q):
     return q * np.array([1.0, -1.0, -1.0, -1.0])
 
 
+def planar_forward(v, ql, qr, counter=None):
+    """The 2-D special case ([IQ] abstract) written as plane rotations.
+
+    With q_L = (cos a, sin a, 0, 0) and q_R = (cos b, sin b, 0, 0), Hamilton's
+    rules give q_L v = rotation of both pairs (v0, v1) and (v2, v3) by a, and
+    v conj(q_R) = rotation of (v0, v1) by -b and of (v2, v3) by +b; so the
+    block map is the plane rotation by a - b on the first pair and by a + b
+    on the second, with cos(a -+ b) = w_L w_R +- x_L x_R and
+    sin(a -+ b) = x_L w_R -+ w_L x_R.  Four multiply-adds per pair
+    (``counter``), d * 2 per vector.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    ql = np.asarray(ql, dtype=np.float64)
+    qr = np.asarray(qr, dtype=np.float64)
+    c1 = ql[..., 0] * qr[..., 0] + ql[..., 1] * qr[..., 1]
+    s1 = ql[..., 1] * qr[..., 0] - ql[..., 0] * qr[..., 1]
+    c2 = ql[..., 0] * qr[..., 0] - ql[..., 1] * qr[..., 1]
+    s2 = ql[..., 1] * qr[..., 0] + ql[..., 0] * qr[..., 1]
+    u = np.empty(np.broadcast_shapes(v.shape, ql.shape), dtype=np.float64)
+    u[..., 0] = c1 * v[..., 0] - s1 * v[..., 1]
+    u[..., 1] = s1 * v[..., 0] + c1 * v[..., 1]
+    u[..., 2] = c2 * v[..., 2] - s2 * v[..., 3]
+    u[..., 3] = s2 * v[..., 2] + c2 * v[..., 3]
+    if counter is not None:
+        counter[0] += 8 * int(np.prod(u.shape[:-1], dtype=np.int64))
+    return u
+
+
 def so4_forward(v, ql, qr, variant, counter=None):
     """[IQ] abstract / [RQ] Algorithm 1: T(v) = q_L v conj(q_R) per 4-block.
 
-    v: [..., nblk, 4]; ql, qr: [nblk, 4].  Full applies both products; Fast
-    keeps only the left isoclinic factor, T(v) = q_L v.
+    v: [..., nblk, 4]; ql, qr: [nblk, 4].  Full (and the no-WHT BLOCK_SO4,
+    and SO3 whose q_R = q_L) applies both products; Fast keeps only the left
+    isoclinic factor, T(v) = q_L v; PLANAR applies its two plane rotations.
     """
+    if variant == PLANAR:
+        return planar_forward(v, ql, qr, counter)
     u = hamilton(ql, v, counter)
-    if variant == FULL:
+    if variant != FAST:
         u = hamilton(u, qconj(qr), counter)
     return u
 
 
 def so4_inverse(u, ql, qr, variant):
-    """Inverse block map: conj(q_L) u q_R (Full) or conj(q_L) u (Fast).
+    """Inverse block map: conj(q_L) u q_R (Full and every variant but Fast)
+    or conj(q_L) u (Fast).
 
     [RQ] §3.4 / Table 2 kernel D: the inverse rotation uses the transposed
     SO(4) blocks; for unit quaternions the transpose of v -> q_L v conj(q_R)
     is u -> conj(q_L) u q_R.
     """
     v = hamilton(qconj(ql), u)
-    if variant == FULL:
+    if variant != FAST:
         v = hamilton(v, qr)
     return v
 
 
+def uses_wht(variant: int) -> bool:
+    """[RQ] §4.6 Table 8: v3 (FULL, and FAST and PLANAR built the same way)
+    composes the block map with the WHT; v1 (SO3) and v2 (BLOCK_SO4) do not."""
+    return variant in (FULL, FAST, PLANAR)
+
+
 def rotate(xhat, params_head, variant):
-    """R x = R_SO4(H_d x / sqrt(d)) along the last axis ([RQ] eq. (2))."""
+    """R x = R_SO4(H_d x / sqrt(d)) along the last axis ([RQ] eq. (2));
+    R x = R_SO4 x for the variants without the WHT."""
     xhat = np.asarray(xhat, dtype=np.float64)
     d = xhat.shape[-1]
     p = np.asarray(params_head, dtype=np.float64).reshape(d // 4, 8)
-    z = wht(xhat) / math.sqrt(d)
+    z = wht(xhat) / math.sqrt(d) if uses_wht(variant) else xhat
     blocks = z.reshape(z.shape[:-1] + (d // 4, 4))
     return so4_forward(blocks, p[:, 0:4], p[:, 4:8], variant).reshape(xhat.shape)
 
 
 def rotate_inverse(y, params_head, variant):
-    """R^T y = H_d (R_SO4^T y) / sqrt(d) ([RQ] Appendix A: R^-1 = R^T)."""
+    """R^T y = H_d (R_SO4^T y) / sqrt(d) ([RQ] Appendix A: R^-1 = R^T);
+    R_SO4^T y for the variants without the WHT."""
     y = np.asarray(y, dtype=np.float64)
     d = y.shape[-1]
     p = np.asarray(params_head, dtype=np.float64).reshape(d // 4, 8)
     blocks = y.reshape(y.shape[:-1] + (d // 4, 4))
     v = so4_inverse(blocks, p[:, 0:4], p[:, 4:8], variant).reshape(y.shape)
-    return wht(v) / math.sqrt(d)
+    return wht(v) / math.sqrt(d) if uses_wht(variant) else v
 
 
 # ---------------------------------------------------------------------------

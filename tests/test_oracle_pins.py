@@ -130,10 +130,19 @@ def _block_matrix(ql, qr, variant):
     return np.stack(cols, axis=1)
 
 
-@pytest.mark.parametrize("variant", [O.FULL, O.FAST])
+def _complex_line(g, n):
+    a = g.standard_normal((n, 2))
+    a /= np.linalg.norm(a, axis=1, keepdims=True)
+    return np.concatenate([a, np.zeros((n, 2))], axis=1)
+
+
+@pytest.mark.parametrize("variant", O.VARIANTS)
 def test_block_map_is_rotation_in_so4(variant):
     g = np.random.default_rng(3)
-    for ql, qr in zip(_rand_unit_quats(g, 50), _rand_unit_quats(g, 50)):
+    draw = _complex_line if variant == O.PLANAR else _rand_unit_quats
+    for ql, qr in zip(draw(g, 50), draw(g, 50)):
+        if variant == O.SO3:
+            qr = ql
         m = _block_matrix(ql, qr, variant)
         np.testing.assert_allclose(m.T @ m, np.eye(4), atol=1e-14)
         assert abs(np.linalg.det(m) - 1.0) < 1e-13  # SO(4), not a reflection
@@ -173,6 +182,53 @@ def test_fast_is_left_isoclinic_and_full_with_identity_right():
         np.testing.assert_allclose(m, _block_matrix(q, _rand_unit_quats(g, 1)[0], O.FAST), atol=0)
 
 
+def test_planar_is_the_complex_line_special_case():
+    """IsoQuant names a 2-D special case of q_L v conj(q_R).  With both
+    quaternions on the complex line span{1, i} the Hamilton products reduce
+    to two independent plane rotations, by angle(q_L) - angle(q_R) on the
+    block's first coordinate pair and angle(q_L) + angle(q_R) on the second
+    (angles from atan2, independently of the product formulas)."""
+    g = np.random.default_rng(8)
+    ql, qr = _complex_line(g, 40), _complex_line(g, 40)
+    v = g.standard_normal((40, 4))
+    hamilton_full = O.so4_forward(v, ql, qr, O.FULL)
+    np.testing.assert_allclose(O.planar_forward(v, ql, qr), hamilton_full, atol=1e-14)
+    a = np.arctan2(ql[:, 1], ql[:, 0])
+    b = np.arctan2(qr[:, 1], qr[:, 0])
+
+    def rot(t, x, y):
+        return np.cos(t) * x - np.sin(t) * y, np.sin(t) * x + np.cos(t) * y
+
+    u01 = rot(a - b, v[:, 0], v[:, 1])
+    u23 = rot(a + b, v[:, 2], v[:, 3])
+    np.testing.assert_allclose(hamilton_full, np.stack([*u01, *u23], axis=1), atol=1e-13)
+    # the planar inverse is the Full inverse with the same pair
+    back = O.so4_inverse(O.planar_forward(v, ql, qr), ql, qr, O.PLANAR)
+    np.testing.assert_allclose(back, v, atol=1e-14)
+    # "lightweight": four multiply-adds per coordinate pair
+    assert O.so4_fma_count(128, O.PLANAR) == 2 * 128
+
+
+def test_single_quaternion_variant_leaves_a_quarter_unmixed():
+    """RotaryQuant §4.6 Table 8, v1: v -> q v conj(q) spans only SO(3) and
+    leaves one coordinate per block (25 % of all) unmixed; v2 (block SO(4)
+    without the WHT) mixes only inside each block; v3 (WHT + SO(4)) mixes
+    every coordinate into every other."""
+    d = 128
+    x = np.random.default_rng(9).standard_normal(d)
+    y1 = O.rotate(x, O.make_params(d, O.SO3, seed=3)[0], O.SO3)
+    # (|q|^2 = 1 to float32 rounding of the stored parameters)
+    np.testing.assert_allclose(y1[0::4], x[0::4], rtol=1e-6)
+    assert np.max(np.abs(y1[1::4] - x[1::4])) > 0.1
+    # Jacobians: block-diagonal for v1 and v2, dense for v3
+    for var in (O.SO3, O.BLOCK_SO4):
+        r = O.rotate(np.eye(d), O.make_params(d, var, seed=3)[0], var).T
+        mask = np.kron(np.eye(d // 4), np.ones((4, 4))) > 0
+        assert np.all(r[~mask] == 0.0)
+    r3 = O.rotate(np.eye(d), O.make_params(d, O.FULL, seed=3)[0], O.FULL).T
+    assert np.count_nonzero(np.abs(r3) > 1e-12) > 0.99 * d * d
+
+
 def test_rotation_fma_counts_match_pages():
     figs = _read_golden_pairs("page_figures.txt")
     assert O.so4_fma_count(128, O.FULL) == figs["isoquant_full_fmas_d128"]
@@ -187,7 +243,7 @@ def test_rotation_fma_counts_match_pages():
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("d", [128, 256])
-@pytest.mark.parametrize("variant", [O.FULL, O.FAST])
+@pytest.mark.parametrize("variant", O.VARIANTS)
 def test_composite_rotation_orthogonal_and_inverse(d, variant):
     p32 = O.make_params(d, variant, seed=11)[0]
     # The stored parameters are float32, so their quaternions have unit norm
@@ -197,6 +253,8 @@ def test_composite_rotation_orthogonal_and_inverse(d, variant):
     # With exactly normalised float64 quaternions R is orthogonal to rounding.
     p = p32.astype(np.float64).reshape(d // 4, 2, 4)
     p = (p / np.linalg.norm(p, axis=-1, keepdims=True)).reshape(d // 4, 8)
+    if variant == O.SO3:
+        p[:, 4:] = p[:, :4]
     r = O.rotate(np.eye(d), p, variant).T          # column j = R e_j
     np.testing.assert_allclose(r.T @ r, np.eye(d), atol=1e-13)
     rinv = O.rotate_inverse(np.eye(d), p, variant).T
@@ -207,7 +265,7 @@ def test_composite_rotation_orthogonal_and_inverse(d, variant):
     assert abs(O.rotate(x, p, variant) @ O.rotate(y, p, variant) - x @ y) < 1e-11
     # Block structure: R e_j restricted to one block equals the block map of
     # the WHT column, independently rebuilt from the Sylvester matrix.
-    h = _sylvester(d) / math.sqrt(d)
+    h = _sylvester(d) / math.sqrt(d) if O.uses_wht(variant) else np.eye(d)
     blk = 5
     m = _block_matrix(p[blk, :4].astype(np.float64), p[blk, 4:].astype(np.float64), variant)
     np.testing.assert_allclose(r[4 * blk:4 * blk + 4, :], m @ h[4 * blk:4 * blk + 4, :], atol=1e-14)
@@ -254,6 +312,18 @@ def test_params_layout_and_draws():
     g = O.gaussian_stream(O.SplitMix64(1))
     v = np.array([next(g) for _ in range(4)])
     np.testing.assert_array_equal(full[0, 0, :4], (v / np.linalg.norm(v)).astype(np.float32))
+    # The variants consume the same eight normals per block.
+    np.testing.assert_array_equal(O.make_params(128, O.BLOCK_SO4, seed=1, n_heads=3), full)
+    so3 = O.make_params(128, O.SO3, seed=1, n_heads=3)
+    np.testing.assert_array_equal(so3[..., :4], full[..., :4])
+    np.testing.assert_array_equal(so3[..., 4:], full[..., :4])
+    pl = O.make_params(128, O.PLANAR, seed=1, n_heads=3)
+    np.testing.assert_array_equal(pl[..., 2:4], 0.0)
+    np.testing.assert_array_equal(pl[..., 6:8], 0.0)
+    np.testing.assert_allclose(np.hypot(pl[..., 0], pl[..., 1]), 1.0, atol=1e-6)
+    w = np.array([next(g) for _ in range(4)])             # q_R's normals of block 0
+    np.testing.assert_array_equal(pl[0, 0, :2], (v[:2] / np.linalg.norm(v[:2])).astype(np.float32))
+    np.testing.assert_array_equal(pl[0, 0, 4:6], (w[:2] / np.linalg.norm(w[:2])).astype(np.float32))
 
 
 def test_params_are_haar_distributed():
@@ -395,7 +465,7 @@ def test_threshold_count_is_nearest_centroid(bits):
 # End-to-end quantise / dequantise
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("variant", [O.FULL, O.FAST])
+@pytest.mark.parametrize("variant", O.VARIANTS)
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_requantising_a_reconstruction_returns_its_codes(variant, bits):
     d = 128
@@ -426,21 +496,46 @@ def test_requantising_a_reconstruction_returns_its_codes(variant, bits):
     np.testing.assert_allclose(xr, expect, atol=1e-13)
 
 
+@pytest.mark.parametrize("variant", O.VARIANTS)
 @pytest.mark.parametrize("bits", [2, 3, 4])
-def test_stage1_mse_close_to_lloyd_distortion(bits):
+def test_stage1_mse_close_to_lloyd_distortion(bits, variant):
     """Unit vectors: per-coordinate rotated marginal ~ N(0, 1/d), so the mean
     squared reconstruction error is close to the Gaussian Lloyd-Max
     distortion (Max 1960), slightly below it (the exact marginal, a scaled
-    Beta, has lighter tails)."""
+    Beta, has lighter tails).  An isotropic input stays isotropic under any
+    rotation, so every variant lands in the same band."""
     table = _read_max_table()
     d = 128
-    params = O.make_params(d, O.FULL, seed=1)
+    params = O.make_params(d, variant, seed=1)
     x = synth.unit_vectors(2000, d, seed=3, dtype=np.float64)
-    packed, norms = O.quantize(x, params, bits, O.FULL)
-    xr = O.dequantize(packed, norms, params, bits, O.FULL, d)
+    packed, norms = O.quantize(x, params, bits, variant)
+    xr = O.dequantize(packed, norms, params, bits, variant, d)
     mse = np.mean(np.sum((x - xr) ** 2, axis=-1))
     ref = table[(bits, "mse")][0]
     assert 0.85 * ref < mse < 1.05 * ref
+
+
+def test_rotation_ablation_ordering_on_outlier_channels():
+    """RotaryQuant §4.6 Table 8 on keys and values with outlier channels
+    (Student-t, 4 channels x10, RoPE on K): the WHT-composed rotations
+    (v3 Full, Fast, the 2-D case) spread the outliers and stay near the
+    Lloyd-Max distortion; v2 (block SO(4), no WHT) keeps each outlier inside
+    its block and v1 (one quaternion) also leaves a quarter of the
+    coordinates unrotated, so their relative errors order v1 > v2 >> v3."""
+    table = _read_max_table()
+    d, bits = 128, 3
+    k, v = synth.student_t_kv(1, 1000, d, seed=5, dtype=np.float64)
+    for x in (k[0, 0], v[0, 0]):
+        rel = {}
+        for var in O.VARIANTS:
+            p = O.make_params(d, var, seed=1)
+            packed, norms = O.quantize(x[None], p, bits, var)
+            xr = O.dequantize(packed, norms, p, bits, var, d)[0]
+            rel[var] = np.mean(np.sum((x - xr) ** 2, -1) / np.sum(x * x, -1))
+        ref = table[(bits, "mse")][0]
+        for var in (O.FULL, O.FAST, O.PLANAR):
+            assert 0.85 * ref < rel[var] < 1.05 * ref
+        assert rel[O.SO3] > 1.1 * rel[O.BLOCK_SO4] > 4 * max(rel[O.FULL], rel[O.FAST], rel[O.PLANAR])
 
 
 def test_zero_vector_and_tie_codes():
