@@ -41,8 +41,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "packed-3-bit decode attn KV GB/s (% of HBM peak); quantize Mvec/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["compressed_space_attention_b200/csrc/isoq_decode.cu",
-                  "compressed_space_attention_b200/csrc/decode_i8.cuh",
+# The files holding the decode split kernel's device code (its traffic in the
+# committed ncu summary is valid only while they are unchanged).
+KERNEL_SOURCES = ["compressed_space_attention_b200/csrc/decode_i8.cuh",
                   "compressed_space_attention_b200/csrc/common.cuh"]
 TRAFFIC_PROFILE = "profiles/decode_split_b32_gqa16_8_d256_t65536.md"
 
@@ -313,6 +314,44 @@ def rank_seed(rank):
 # CUDA arm
 # ---------------------------------------------------------------------------
 
+VARIANT_NAMES = {0: "Full (WHT+SO(4), v3)", 1: "Fast (WHT+q_L)", 2: "2-D special case (WHT+planar)",
+                 3: "v2: block SO(4), no WHT", 4: "v1: single quaternion, no WHT"}
+
+
+def measure_variants(isoq, synth, torch, dev, stream, x1, seed0, reps=5):
+    """Per rotation variant: quantize throughput on the stage-1 workload and
+    the relative round-trip error on it and on outlier-channel keys."""
+    n1, d1, bits = x1.shape[1], x1.shape[2], STAGE1["bits"]
+    k, _ = synth.student_t_kv_torch(1, 1, 65536, d1, seed=seed0 + 31, device=dev)
+    xk = k[0]
+    out = {}
+    for var, name in VARIANT_NAMES.items():
+        p = torch.from_numpy(isoq.isoq_make_params(d1, var, 1, 1)).to(dev)
+        codes = torch.empty((1, n1, d1 * bits // 8), dtype=torch.uint8, device=dev)
+        norms = torch.empty((1, n1), dtype=torch.float16, device=dev)
+        for _ in range(2):
+            isoq.isoq_quantize(x1, p, bits, var, codes=codes, norms=norms)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            isoq.isoq_quantize(x1, p, bits, var, codes=codes, norms=norms)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        rel = {}
+        for label, x in (("unit_vectors", x1), ("outlier_keys", xk)):
+            c, nrm = isoq.isoq_quantize(x, p, bits, var)
+            r = isoq.isoq_dequantize(c, nrm, p, d1, bits, var, out_dtype=torch.float32)
+            xf = x.float()
+            rel[label] = float((((r - xf) ** 2).sum(-1) / (xf * xf).sum(-1)).mean())
+        out[name] = {"quantize_mvec_s": n1 / (ms * 1e-3) / 1e6, "quantize_ms": ms,
+                     "rel_mse_unit_vectors": rel["unit_vectors"], "rel_mse_outlier_keys": rel["outlier_keys"]}
+    assert isoq.isoq_check_device_error() == 0
+    return {"workload": f"2^20 float16 unit vectors (stage-1) and 65,536 Student-t keys with outlier "
+                        f"channels and RoPE; d={d1}, {bits}-bit", "by_variant": out}
+
+
 def run_isoq(args):
     import torch
 
@@ -483,6 +522,9 @@ def run_isoq(args):
     t_dstep = a1.elapsed_time(a2) / n_app
     app_bytes = 2 * B * Hkv * (2 * d + pb + 2)
 
+    # ---- rotation variants (IsoQuant's 2-D case, RotaryQuant §4.6 v1, v2) ----
+    variants = measure_variants(isoq, synth, torch, dev, stream, x1, seed0) if not args.no_variants else None
+
     # ---- reduce over ranks: max time, summed bytes ----
     total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms, t_app, t_dstep = max_over_ranks(
         [total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms, t_app, t_dstep], dist, dev)
@@ -520,6 +562,7 @@ def run_isoq(args):
                                 "(append_kernel + length advance), and isoq_decode_step = append "
                                 "then decode attention over the cache at half capacity; timed "
                                 "outside the main region"},
+        "variants": variants,
         "gpu_launches": 4 * args.steps,
         "clocks": sampler.summary(),
     }
@@ -545,6 +588,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle CPU baseline (profiling runs)")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the rotation-variant measurements (2-D case, ablation v1/v2)")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--batch", type=int, default=0,

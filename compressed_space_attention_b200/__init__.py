@@ -12,9 +12,12 @@ from .binding import (  # noqa: F401
     ISOQ_ERR_UNSUPPORTED,
     ISOQ_F16,
     ISOQ_F32,
+    ISOQ_BLOCK_SO4,
     ISOQ_FAST,
     ISOQ_FULL,
     ISOQ_OK,
+    ISOQ_PLANAR,
+    ISOQ_SO3,
     IsoqError,
     isoq_abi_version,
     isoq_check_device_error,

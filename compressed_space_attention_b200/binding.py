@@ -23,6 +23,9 @@ ISOQ_ERR_CUDA = -3
 ISOQ_ERR_TIMEOUT = -4
 ISOQ_FULL = 0
 ISOQ_FAST = 1
+ISOQ_PLANAR = 2
+ISOQ_BLOCK_SO4 = 3
+ISOQ_SO3 = 4
 ISOQ_F16 = 0
 ISOQ_F32 = 1
 

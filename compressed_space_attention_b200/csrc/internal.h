@@ -18,6 +18,11 @@ void clear_error();
 bool supported_d(int d);
 bool supported_bits(int bits);
 bool supported_variant(int v);
+// Variants the decode path takes; block_map_variant gives the one whose
+// block map the decode kernels apply (PLANAR's parameters make the Full map
+// its two plane rotations).
+bool supported_decode_variant(int v);
+inline int block_map_variant(int v) { return v == ISOQ_FAST ? ISOQ_FAST : ISOQ_FULL; }
 bool supported_dtype(int t);
 inline int elt_size(int dtype) { return dtype == ISOQ_F16 ? 2 : 4; }
 

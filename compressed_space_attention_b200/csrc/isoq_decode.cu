@@ -370,7 +370,7 @@ bool aligned(const void *p, unsigned a) { return (reinterpret_cast<uintptr_t>(p)
 int validate_common(int dtype, int B, int Hq, int Hkv, int64_t Tmax, int d, int variant,
                     const void *ws, size_t ws_bytes) {
   if (!supported_d(d)) return set_error(ISOQ_ERR_UNSUPPORTED, "d=%d not supported", d);
-  if (!supported_variant(variant)) return set_error(ISOQ_ERR_UNSUPPORTED, "variant=%d", variant);
+  if (!supported_decode_variant(variant)) return set_error(ISOQ_ERR_UNSUPPORTED, "variant=%d", variant);
   if (!supported_dtype(dtype)) return set_error(ISOQ_ERR_UNSUPPORTED, "dtype=%d", dtype);
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tmax <= 0)
     return set_error(ISOQ_ERR_INVALID_ARG, "B, Hq, Hkv and Tmax must be positive");
@@ -421,6 +421,7 @@ int isoq_decode_split(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
       !decode::aligned(seq_lens_dev, 4))
     return set_error(ISOQ_ERR_UNSUPPORTED, "misaligned pointer");
   if (!std::isfinite(scale)) return set_error(ISOQ_ERR_INVALID_ARG, "scale is not finite");
+  variant = block_map_variant(variant);
 
   decode::SplitArgs a;
   a.q = q_dev;
@@ -457,6 +458,7 @@ int isoq_decode_combine(int dtype, const int32_t *seq_lens_dev, int B, int Hq, i
   if (!params_v_dev || !out_dev || !seq_lens_dev) return set_error(ISOQ_ERR_INVALID_ARG, "null pointer");
   if (!decode::aligned(params_v_dev, 16) || !decode::aligned(out_dev, 16))
     return set_error(ISOQ_ERR_UNSUPPORTED, "misaligned pointer");
+  variant = block_map_variant(variant);
   decode::CombineArgs a;
   a.params_v = params_v_dev;
   a.out = out_dev;
@@ -511,7 +513,7 @@ int isoq_decode_append(const void *k_new_dev, const void *v_new_dev, int dtype,
   clear_error();
   if (!supported_d(d)) return set_error(ISOQ_ERR_UNSUPPORTED, "d=%d not supported", d);
   if (!supported_bits(bits)) return set_error(ISOQ_ERR_UNSUPPORTED, "bits=%d not supported", bits);
-  if (!supported_variant(variant)) return set_error(ISOQ_ERR_UNSUPPORTED, "variant=%d", variant);
+  if (!supported_decode_variant(variant)) return set_error(ISOQ_ERR_UNSUPPORTED, "variant=%d", variant);
   if (!supported_dtype(dtype)) return set_error(ISOQ_ERR_UNSUPPORTED, "dtype=%d", dtype);
   if (B <= 0 || Hkv <= 0 || Tmax <= 0)
     return set_error(ISOQ_ERR_INVALID_ARG, "B, Hkv and Tmax must be positive");
@@ -525,6 +527,7 @@ int isoq_decode_append(const void *k_new_dev, const void *v_new_dev, int dtype,
       !decode::aligned(k_new_dev, 16) || !decode::aligned(v_new_dev, 16) ||
       !decode::aligned(norms_k_dev, 2) || !decode::aligned(norms_v_dev, 2) || !decode::aligned(seq_lens_dev, 4))
     return set_error(ISOQ_ERR_UNSUPPORTED, "misaligned pointer");
+  variant = block_map_variant(variant);
   decode::AppendArgs a;
   a.k_new = k_new_dev;
   a.v_new = v_new_dev;

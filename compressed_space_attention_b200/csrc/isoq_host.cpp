@@ -28,7 +28,8 @@ void clear_error() { g_last_error[0] = '\0'; }
 
 bool supported_d(int d) { return d == 128 || d == 256 || d == 512; }
 bool supported_bits(int bits) { return bits >= 2 && bits <= 4; }
-bool supported_variant(int v) { return v == ISOQ_FULL || v == ISOQ_FAST; }
+bool supported_variant(int v) { return v >= ISOQ_FULL && v <= ISOQ_SO3; }
+bool supported_decode_variant(int v) { return v == ISOQ_FULL || v == ISOQ_FAST || v == ISOQ_PLANAR; }
 bool supported_dtype(int t) { return t == ISOQ_F16 || t == ISOQ_F32; }
 
 // ---------------------------------------------------------------------------
@@ -234,17 +235,19 @@ int isoq_make_params(int d, int variant, uint64_t seed, int n_heads, float *out_
     for (int i = 0; i < d / 4; ++i) {
       double q[8];
       for (int k = 0; k < 8; ++k) q[k] = g.next();
+      if (variant == ISOQ_PLANAR) q[2] = q[3] = q[6] = q[7] = 0.0;   // the complex line
       for (int half = 0; half < 2; ++half) {
         double *v = q + 4 * half;
         double n = std::sqrt(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
         for (int k = 0; k < 4; ++k) v[k] = v[k] / n;
       }
       for (int k = 0; k < 4; ++k) p[k] = static_cast<float>(q[k]);
-      if (variant == ISOQ_FULL) {
-        for (int k = 0; k < 4; ++k) p[4 + k] = static_cast<float>(q[4 + k]);
-      } else {
+      if (variant == ISOQ_FAST) {
         p[4] = 1.0f;
         p[5] = p[6] = p[7] = 0.0f;
+      } else {
+        const double *r = variant == ISOQ_SO3 ? q : q + 4;
+        for (int k = 0; k < 4; ++k) p[4 + k] = static_cast<float>(r[k]);
       }
       p += 8;
     }

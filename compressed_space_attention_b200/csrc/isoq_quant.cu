@@ -67,6 +67,15 @@ constexpr int kQuantWarps = 4;
 constexpr int kQuantThreads = 32 * kQuantWarps;
 constexpr int kDequantThreads = 128;
 
+// Rotation kinds of the kernels (the variants of include/isoq.h map onto
+// them in rotation_kind): the WHT composed with the full block map
+// q_L v conj(q_R) (Full, and the 2-D special case, whose parameters make the
+// same map two plane rotations), the WHT with the left factor only (Fast),
+// and the full block map alone (the ablation's v2, and v1 with q_R = q_L).
+constexpr int kRotWhtFull = 0;
+constexpr int kRotWhtFast = 1;
+constexpr int kRotBlock = 2;
+
 __device__ unsigned int g_quant_error = 0;
 
 // Lane geometry shared by both directions.
@@ -150,31 +159,38 @@ __host__ __device__ constexpr bool group_negated(int g) {
 // Per-block 4x4 matrices of one head, stored for the packed product:
 // group g, block pair beta (blocks 8g + beta and 8g + beta + 4), entry
 // (j, c) -> float pair at mat[128 g + 32 beta + 2 (4 j + c) + {0, 1}].
-//   forward: M_i = R_i H_4 / sqrt(d); inverse: N_i = H_4 R_i^T / sqrt(d).
-template <int D, bool FULL, bool FORWARD>
+//   forward: M_i = R_i H_4 / sqrt(d); inverse: N_i = H_4 R_i^T / sqrt(d);
+//   without the WHT (kRotBlock): M_i = R_i, N_i = R_i^T.
+template <int D, int RK, bool FORWARD>
 __device__ void build_block_matrices(const float *params_head, float *mat, int tid, int nthreads) {
-  const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+  constexpr bool FULL = RK != kRotWhtFast;
+  constexpr bool WHT = RK != kRotBlock;
+  const float inv_sqrt_d = WHT ? rsqrtf(static_cast<float>(D)) : 1.f;
   for (int b = tid; b < D / 4; b += nthreads) {
     const Quat ql = load_quat(params_head + 8 * b);
     const Quat qr = load_quat(params_head + 8 * b + 4);
     float m[4][4];
     for (int c = 0; c < 4; ++c) {
+      const Quat e{c == 0 ? 1.f : 0.f, c == 1 ? 1.f : 0.f, c == 2 ? 1.f : 0.f, c == 3 ? 1.f : 0.f};
       if (FORWARD) {
-        // column c = R_i (H_4 e_c)
-        const Quat u = block_forward(ql, qr, h4_column(c), FULL);
+        // column c = R_i (H_4 e_c), or R_i e_c without the WHT
+        const Quat u = block_forward(ql, qr, WHT ? h4_column(c) : e, FULL);
         m[0][c] = u.w; m[1][c] = u.x; m[2][c] = u.y; m[3][c] = u.z;
-      } else {
+      } else if (WHT) {
         // column c = H_4 (R_i^T e_c)
-        Quat e{c == 0 ? 1.f : 0.f, c == 1 ? 1.f : 0.f, c == 2 ? 1.f : 0.f, c == 3 ? 1.f : 0.f};
         const Quat u = block_inverse(ql, qr, e, FULL);
         m[0][c] = u.w + u.x + u.y + u.z;
         m[1][c] = u.w - u.x + u.y - u.z;
         m[2][c] = u.w + u.x - u.y - u.z;
         m[3][c] = u.w - u.x - u.y + u.z;
+      } else {
+        // column c = R_i^T e_c
+        const Quat u = block_inverse(ql, qr, e, FULL);
+        m[0][c] = u.w; m[1][c] = u.x; m[2][c] = u.y; m[3][c] = u.z;
       }
     }
     const int g = b >> 3, r = b & 7, beta = r & 3, half = r >> 2;
-    const float sc = group_negated<D>(g) ? -inv_sqrt_d : inv_sqrt_d;
+    const float sc = WHT && group_negated<D>(g) ? -inv_sqrt_d : inv_sqrt_d;
     float *out = mat + 128 * g + 32 * beta + half;
     for (int j = 0; j < 4; ++j)
       for (int c = 0; c < 4; ++c) out[2 * (4 * j + c)] = m[j][c] * sc;
@@ -342,7 +358,7 @@ __device__ __forceinline__ void quantize_group(const uint64_t (&xp)[kPairs], int
 // Quantize
 // ---------------------------------------------------------------------------
 
-template <typename T, int D, int BITS, bool FULL>
+template <typename T, int D, int BITS, int RK>
 __global__ void __launch_bounds__(kQuantThreads, 4)
     quantize_kernel(const __grid_constant__ CUtensorMap xmap, const QuantArgs args) {
   using C = Cfg<T, D, BITS>;
@@ -388,16 +404,19 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
   int cur_head = -1;
   if (n_mine > 0) {
     cur_head = static_cast<int>(tile_begin / args.tiles_per_head);
-    build_block_matrices<D, FULL, true>(args.params + static_cast<size_t>(cur_head) * 2 * D, mat,
+    build_block_matrices<D, RK, true>(args.params + static_cast<size_t>(cur_head) * 2 * D, mat,
                                         tid, kQuantThreads);
   }
   __syncthreads();
 
+  constexpr bool WHT = RK != kRotBlock;
   const int part = lane / VPW;
   const int vl = lane % VPW;
   const bool hb = (part & KH) != 0;
-  int grp[2];
-  lane_groups<D>(part, grp);
+  // Without the WHT nothing moves between lanes: each lane keeps the two
+  // groups it loaded.
+  int grp[2] = {2 * part, 2 * part + 1};
+  if (WHT) lane_groups<D>(part, grp);
   const uint32_t mat_s = smem_u32(mat);
   const float sg = hb ? -1.f : 1.f;
   const uint64_t sig2 = f2_pack(sg, sg), nsig2 = f2_pack(-sg, -sg);
@@ -410,7 +429,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     if (head != cur_head) {
       // Every warp walks the same tiles, so all of them meet here.
       named_barrier(1, kQuantThreads);
-      build_block_matrices<D, FULL, true>(args.params + static_cast<size_t>(head) * 2 * D, mat,
+      build_block_matrices<D, RK, true>(args.params + static_cast<size_t>(head) * 2 * D, mat,
                                           tid, kQuantThreads);
       named_barrier(1, kQuantThreads);
       cur_head = head;
@@ -443,8 +462,13 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
           for (int j = 0; j < 4; ++j) {
             const float2 a = __half22float2(hl[j]);
             const float2 b = __half22float2(hh[j]);
-            xp[kGP * G + 8 * c + 2 * j] = f2_pack(a.x + b.x, a.x - b.x);
-            xp[kGP * G + 8 * c + 2 * j + 1] = f2_pack(a.y + b.y, a.y - b.y);
+            if (WHT) {
+              xp[kGP * G + 8 * c + 2 * j] = f2_pack(a.x + b.x, a.x - b.x);
+              xp[kGP * G + 8 * c + 2 * j + 1] = f2_pack(a.y + b.y, a.y - b.y);
+            } else {
+              xp[kGP * G + 8 * c + 2 * j] = f2_pack(a.x, b.x);
+              xp[kGP * G + 8 * c + 2 * j + 1] = f2_pack(a.y, b.y);
+            }
           }
         }
       }
@@ -460,10 +484,17 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
           const float a2 = __uint_as_float(ulo.z), a3 = __uint_as_float(ulo.w);
           const float b0 = __uint_as_float(uhi.x), b1 = __uint_as_float(uhi.y);
           const float b2 = __uint_as_float(uhi.z), b3 = __uint_as_float(uhi.w);
-          xp[kGP * G + 4 * c] = f2_pack(a0 + b0, a0 - b0);
-          xp[kGP * G + 4 * c + 1] = f2_pack(a1 + b1, a1 - b1);
-          xp[kGP * G + 4 * c + 2] = f2_pack(a2 + b2, a2 - b2);
-          xp[kGP * G + 4 * c + 3] = f2_pack(a3 + b3, a3 - b3);
+          if (WHT) {
+            xp[kGP * G + 4 * c] = f2_pack(a0 + b0, a0 - b0);
+            xp[kGP * G + 4 * c + 1] = f2_pack(a1 + b1, a1 - b1);
+            xp[kGP * G + 4 * c + 2] = f2_pack(a2 + b2, a2 - b2);
+            xp[kGP * G + 4 * c + 3] = f2_pack(a3 + b3, a3 - b3);
+          } else {
+            xp[kGP * G + 4 * c] = f2_pack(a0, b0);
+            xp[kGP * G + 4 * c + 1] = f2_pack(a1, b1);
+            xp[kGP * G + 4 * c + 2] = f2_pack(a2, b2);
+            xp[kGP * G + 4 * c + 3] = f2_pack(a3, b3);
+          }
         }
       }
     }
@@ -476,35 +507,37 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
       ++issued;
     }
 
-    // Step 1: norm.  The pairs hold (a + b, a - b), whose squares sum to
-    // twice a^2 + b^2.
+    // Step 1: norm.  With the WHT the pairs hold (a + b, a - b), whose
+    // squares sum to twice a^2 + b^2.
     uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < kPairs; ++k) acc2 = f2_fma(xp[k], xp[k], acc2);
     float ss_lo, ss_hi;
     f2_unpack(acc2, ss_lo, ss_hi);
-    float ss = 0.5f * (ss_lo + ss_hi);
+    float ss = WHT ? 0.5f * (ss_lo + ss_hi) : ss_lo + ss_hi;
 #pragma unroll
     for (int k = 1; k < P; k <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, k * VPW);
     const float norm = sqrtf(ss);
 
     // Step 2: the remaining WHT stages, then the folded block matrices.
-    wht_pairs_h4_h8(xp);
-    // h = 32, arranged so that group 0 holds what this lane keeps in the
-    // half exchange: (G0, G1) <- (G0 + sg G1, G0 - sg G1).
+    if (WHT) {
+      wht_pairs_h4_h8(xp);
+      // h = 32, arranged so that group 0 holds what this lane keeps in the
+      // half exchange: (G0, G1) <- (G0 + sg G1, G0 - sg G1).
 #pragma unroll
-    for (int p = 0; p < kGP; ++p) {
-      const uint64_t a = xp[p], b = xp[kGP + p];
-      xp[p] = f2_fma(sig2, b, a);
-      xp[kGP + p] = f2_fma(nsig2, b, a);
-    }
-    wht_cross_full<D>(xp, part);
+      for (int p = 0; p < kGP; ++p) {
+        const uint64_t a = xp[p], b = xp[kGP + p];
+        xp[p] = f2_fma(sig2, b, a);
+        xp[kGP + p] = f2_fma(nsig2, b, a);
+      }
+      wht_cross_full<D>(xp, part);
 #pragma unroll
-    for (int p = 0; p < kGP; ++p) {
-      const uint64_t r = __shfl_xor_sync(0xffffffffu, xp[kGP + p], KH * VPW);
-      const uint64_t k = xp[p];
-      xp[p] = f2_add(k, r);
-      xp[kGP + p] = f2_sub(k, r);
+      for (int p = 0; p < kGP; ++p) {
+        const uint64_t r = __shfl_xor_sync(0xffffffffu, xp[kGP + p], KH * VPW);
+        const uint64_t k = xp[p];
+        xp[p] = f2_add(k, r);
+        xp[kGP + p] = f2_sub(k, r);
+      }
     }
     apply_group_matrices(xp, 0, mat_s + 512 * grp[0]);
     apply_group_matrices(xp, kGP, mat_s + 512 * grp[1]);
@@ -561,7 +594,7 @@ struct DequantArgs {
   float centroid[16];
 };
 
-template <typename T, int D, int BITS, bool FULL>
+template <typename T, int D, int BITS, int RK>
 __global__ void __launch_bounds__(kDequantThreads) dequantize_kernel(const DequantArgs args) {
   constexpr int P = Lanes<D>::P, VPW = Lanes<D>::VPW, KH = Lanes<D>::KH;
   constexpr int NV = kDequantThreads / P;
@@ -570,12 +603,13 @@ __global__ void __launch_bounds__(kDequantThreads) dequantize_kernel(const Dequa
   __shared__ __align__(16) float mat[D * 4];
   __shared__ float cent[16];
 
+  constexpr bool WHT = RK != kRotBlock;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int part = lane / VPW, vl = lane % VPW;
   const int vt = warp * VPW + vl;
-  const bool hb = (part & KH) != 0;
-  int grp[2];
-  lane_groups<D>(part, grp);
+  const bool hb = WHT && (part & KH) != 0;
+  int grp[2] = {2 * part, 2 * part + 1};
+  if (WHT) lane_groups<D>(part, grp);
   if (tid < L) cent[tid] = args.centroid[tid];
   const uint32_t mat_s = smem_u32(mat);
 
@@ -590,7 +624,7 @@ __global__ void __launch_bounds__(kDequantThreads) dequantize_kernel(const Dequa
     const long long v = (t % args.tiles_per_head) * NV + vt;
     if (head != cur_head) {
       __syncthreads();
-      build_block_matrices<D, FULL, false>(args.params + static_cast<size_t>(head) * 2 * D, mat,
+      build_block_matrices<D, RK, false>(args.params + static_cast<size_t>(head) * 2 * D, mat,
                                            tid, kDequantThreads);
       __syncthreads();
       cur_head = head;
@@ -623,25 +657,27 @@ __global__ void __launch_bounds__(kDequantThreads) dequantize_kernel(const Dequa
 
     apply_group_matrices(xp, 0, mat_s + 512 * grp[0]);
     apply_group_matrices(xp, kGP, mat_s + 512 * grp[1]);
-    // Half exchange (h = d/2): keep G0 + G1, send G0 - G1.
+    if (WHT) {
+      // Half exchange (h = d/2): keep G0 + G1, send G0 - G1.
 #pragma unroll
-    for (int p = 0; p < kGP; ++p) {
-      const uint64_t a = xp[p], b = xp[kGP + p];
-      const uint64_t dsend = f2_sub(a, b);
-      xp[p] = f2_add(a, b);
-      xp[kGP + p] = __shfl_xor_sync(0xffffffffu, dsend, KH * VPW);
-    }
-    wht_cross_full<D>(xp, part);
-    // h = 32: afterwards G0 holds this lane's lower 32 elements and G1 its
-    // upper 32, the latter negated on lanes with the exchange bit set.
+      for (int p = 0; p < kGP; ++p) {
+        const uint64_t a = xp[p], b = xp[kGP + p];
+        const uint64_t dsend = f2_sub(a, b);
+        xp[p] = f2_add(a, b);
+        xp[kGP + p] = __shfl_xor_sync(0xffffffffu, dsend, KH * VPW);
+      }
+      wht_cross_full<D>(xp, part);
+      // h = 32: afterwards G0 holds this lane's lower 32 elements and G1 its
+      // upper 32, the latter negated on lanes with the exchange bit set.
 #pragma unroll
-    for (int p = 0; p < kGP; ++p) {
-      const uint64_t a = xp[p], b = xp[kGP + p];
-      xp[p] = f2_add(a, b);
-      xp[kGP + p] = f2_sub(a, b);
+      for (int p = 0; p < kGP; ++p) {
+        const uint64_t a = xp[p], b = xp[kGP + p];
+        xp[p] = f2_add(a, b);
+        xp[kGP + p] = f2_sub(a, b);
+      }
+      wht_pairs_h4_h8(xp);
+      wht_in_pair(xp);
     }
-    wht_pairs_h4_h8(xp);
-    wht_in_pair(xp);
     const uint64_t sc0 = f2_pack(s16, s16);
     const float s1 = hb ? -s16 : s16;
     const uint64_t sc1 = f2_pack(s1, s1);
@@ -712,12 +748,12 @@ int num_sms() {
   return n;
 }
 
-template <typename T, int D, int BITS, bool FULL>
+template <typename T, int D, int BITS, int RK>
 int launch_quantize(const void *x, int n_heads, long long n_vec, long long head_stride,
                     long long vec_stride, const float *params, uint8_t *codes, uint16_t *norms,
                     long long out_head_stride, cudaStream_t stream) {
   using C = Cfg<T, D, BITS>;
-  auto kernel = quantize_kernel<T, D, BITS, FULL>;
+  auto kernel = quantize_kernel<T, D, BITS, RK>;
   static int max_ctas_per_sm = -1;
   static std::mutex mu;
   {
@@ -771,12 +807,12 @@ int launch_quantize(const void *x, int n_heads, long long n_vec, long long head_
   return ISOQ_OK;
 }
 
-template <typename T, int D, int BITS, bool FULL>
+template <typename T, int D, int BITS, int RK>
 int launch_dequantize(const uint8_t *codes, const uint16_t *norms, int n_heads, long long n_vec,
                       long long in_head_stride, const float *params, void *out,
                       long long head_stride, long long vec_stride, cudaStream_t stream) {
   constexpr int NV = kDequantThreads / Lanes<D>::P;
-  auto kernel = dequantize_kernel<T, D, BITS, FULL>;
+  auto kernel = dequantize_kernel<T, D, BITS, RK>;
   static int max_ctas_per_sm = -1;
   static std::mutex mu;
   {
@@ -813,11 +849,15 @@ int launch_dequantize(const uint8_t *codes, const uint16_t *norms, int n_heads, 
 }
 
 // Expands the runtime (dtype, d, bits, variant) into a template instantiation.
-template <template <typename, int, int, bool> class F, typename... A>
+template <template <typename, int, int, int> class F, typename... A>
 int dispatch(int dtype, int d, int bits, int variant, A... args) {
-#define ISOQ_CASE_V(T, D, B)                                              \
-  return variant == ISOQ_FULL ? F<T, D, B, true>::run(args...)           \
-                              : F<T, D, B, false>::run(args...)
+  const int rk = variant == ISOQ_FAST ? kRotWhtFast
+               : (variant == ISOQ_BLOCK_SO4 || variant == ISOQ_SO3) ? kRotBlock
+                                                                      : kRotWhtFull;
+#define ISOQ_CASE_V(T, D, B)                                                    \
+  return rk == kRotWhtFull ? F<T, D, B, kRotWhtFull>::run(args...)             \
+       : rk == kRotWhtFast ? F<T, D, B, kRotWhtFast>::run(args...)             \
+                           : F<T, D, B, kRotBlock>::run(args...)
 #define ISOQ_CASE_B(T, D)                  \
   switch (bits) {                          \
     case 2: ISOQ_CASE_V(T, D, 2);          \
@@ -840,21 +880,21 @@ int dispatch(int dtype, int d, int bits, int variant, A... args) {
 #undef ISOQ_CASE_V
 }
 
-template <typename T, int D, int B, bool FULL>
+template <typename T, int D, int B, int RK>
 struct QuantizeRunner {
   static int run(const void *x, int n_heads, long long n_vec, long long hs, long long vs,
                  const float *params, uint8_t *codes, uint16_t *norms, long long ohs,
                  cudaStream_t st) {
-    return launch_quantize<T, D, B, FULL>(x, n_heads, n_vec, hs, vs, params, codes, norms, ohs, st);
+    return launch_quantize<T, D, B, RK>(x, n_heads, n_vec, hs, vs, params, codes, norms, ohs, st);
   }
 };
 
-template <typename T, int D, int B, bool FULL>
+template <typename T, int D, int B, int RK>
 struct DequantizeRunner {
   static int run(const uint8_t *codes, const uint16_t *norms, int n_heads, long long n_vec,
                  long long ihs, const float *params, void *out, long long hs, long long vs,
                  cudaStream_t st) {
-    return launch_dequantize<T, D, B, FULL>(codes, norms, n_heads, n_vec, ihs, params, out, hs, vs, st);
+    return launch_dequantize<T, D, B, RK>(codes, norms, n_heads, n_vec, ihs, params, out, hs, vs, st);
   }
 };
 

@@ -58,9 +58,27 @@ enum isoq_status {
   ISOQ_ERR_TIMEOUT = -4       /* a bounded device-side wait gave up (device error word) */
 };
 
+/*
+ * Rotation R of a variant, per 4-block (w, x, y, z) = w + x i + y j + z k:
+ *   FULL       R = R_SO4 o H_d/sqrt(d), R_SO4: v -> q_L v conj(q_R)
+ *              ([IQ] IsoQuant-Full; [RQ] §4.6 Table 8 v3)
+ *   FAST       R = R_SO4 o H_d/sqrt(d), R_SO4: v -> q_L v ([IQ] IsoQuant-Fast)
+ *   PLANAR     [IQ]'s 2-D special case, read as FULL with q_L and q_R on the
+ *              complex line span{1, i}: each block's coordinate pairs (0, 1)
+ *              and (2, 3) are rotated independently, by angle(q_L) -
+ *              angle(q_R) and angle(q_L) + angle(q_R)
+ *   BLOCK_SO4  R = R_SO4 (Full block map) without the WHT ([RQ] Table 8 v2)
+ *   SO3        R: v -> q v conj(q) per block, no WHT ([RQ] Table 8 v1; the
+ *              parameters hold q in both slots)
+ * isoq_quantize and isoq_dequantize take every variant; the decode entry
+ * points take FULL, FAST and PLANAR (ISOQ_ERR_UNSUPPORTED otherwise).
+ */
 enum isoq_variant {
-  ISOQ_FULL = 0,  /* [IQ] IsoQuant-Full: v -> q_L v conj(q_R)            */
-  ISOQ_FAST = 1   /* [IQ] IsoQuant-Fast: v -> q_L v (q_R slot = identity) */
+  ISOQ_FULL = 0,
+  ISOQ_FAST = 1,
+  ISOQ_PLANAR = 2,
+  ISOQ_BLOCK_SO4 = 3,
+  ISOQ_SO3 = 4
 };
 
 enum isoq_dtype {
@@ -98,7 +116,10 @@ size_t isoq_packed_bytes(int d, int bits);
  * (r cos, then r sin) -> standard normals.  Draw order: heads, blocks, q_L
  * (4 normals), q_R (4 normals); each quaternion is normalised in double and
  * rounded to float32.  ISOQ_FAST keeps Full's q_L (q_R's draws are still
- * consumed) and writes q_R = (1, 0, 0, 0).  Host only, no device work.
+ * consumed) and writes q_R = (1, 0, 0, 0); ISOQ_BLOCK_SO4 writes Full's
+ * pair; ISOQ_SO3 writes Full's q_L in both slots; ISOQ_PLANAR normalises
+ * the first two of each quaternion's four normals and writes
+ * (c, s, 0, 0) for q_L and q_R.  Host only, no device work.
  */
 int isoq_make_params(int d, int variant, uint64_t seed, int n_heads, float *out_host);
 

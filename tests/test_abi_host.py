@@ -35,7 +35,8 @@ def test_sizes():
     assert isoq.isoq_packed_bytes(128, 5) == 0
 
 
-@pytest.mark.parametrize("variant", [isoq.ISOQ_FULL, isoq.ISOQ_FAST])
+@pytest.mark.parametrize("variant", [isoq.ISOQ_FULL, isoq.ISOQ_FAST, isoq.ISOQ_PLANAR,
+                                     isoq.ISOQ_BLOCK_SO4, isoq.ISOQ_SO3])
 @pytest.mark.parametrize("d", [128, 256, 512])
 def test_make_params_matches_oracle(variant, d):
     got = isoq.isoq_make_params(d, variant, seed=1234, n_heads=3)
@@ -88,6 +89,8 @@ def test_quantize_validation_happens_on_host():
     assert _call_quantize(d=100) == isoq.ISOQ_ERR_UNSUPPORTED
     assert _call_quantize(bits=5) == isoq.ISOQ_ERR_UNSUPPORTED
     assert _call_quantize(variant=7) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert _call_quantize(variant=5) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert _call_quantize(variant=-1) == isoq.ISOQ_ERR_UNSUPPORTED
     assert _call_quantize(dtype=9) == isoq.ISOQ_ERR_UNSUPPORTED
     assert _call_quantize(n_vec=-1) == isoq.ISOQ_ERR_INVALID_ARG
     assert _call_quantize(x=None, n_vec=10) == isoq.ISOQ_ERR_INVALID_ARG
@@ -123,6 +126,10 @@ def test_decode_validation_happens_on_host():
     assert call(B=0) == isoq.ISOQ_ERR_INVALID_ARG
     assert call(scale=float("nan")) == isoq.ISOQ_ERR_INVALID_ARG
     assert call(out=None) == isoq.ISOQ_ERR_INVALID_ARG
+    # the ablation's no-WHT variants are stage-1 only
+    assert call(variant=isoq.ISOQ_BLOCK_SO4) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(variant=isoq.ISOQ_SO3) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(variant=5) == isoq.ISOQ_ERR_UNSUPPORTED
 
 
 def test_status_strings():
