@@ -99,75 +99,100 @@ def measured_peaks():
 
 
 # ---------------------------------------------------------------------------
-# Clock sampling (NVML) during the timed region
+# Clock sampling during the timed region
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    """Polls SM clock and throttle reasons of one GPU from a host thread."""
+    """Samples the SM clock and the clock-event reasons of one GPU while the
+    timed region runs.
 
+    An ``nvidia-smi -lms`` child process does the polling (no Python thread
+    competes with the launch loop for the interpreter); each sample carries
+    nvidia-smi's own timestamp, and only the samples inside the region (with
+    one sampling interval of slack on each side) are kept.  Without
+    nvidia-smi, a thread polls NVML instead.
+    """
     REASONS = {
         "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
         "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
     }
+    INTERVAL_MS = 20
 
     def __init__(self, torch_device_index):
-        self.samples = []
-        self.reasons = set()
+        self.samples = []          # (datetime, sm_mhz, reason mask)
         self.max_mhz = None
-        self._stop = threading.Event()
-        self._thread = None
-        self.ok = False
+        self.proc = None
+        self.reader = None
+        self.t0 = self.t1 = None
+        self.uuid = None
         try:
-            import pynvml
             import torch
-            pynvml.nvmlInit()
-            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
-            handle = None
-            for i in range(pynvml.nvmlDeviceGetCount()):
-                h = pynvml.nvmlDeviceGetHandleByIndex(i)
-                u = pynvml.nvmlDeviceGetUUID(h)
-                u = u.decode() if isinstance(u, bytes) else u
-                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
-                    handle = h
-            if handle is None and pynvml.nvmlDeviceGetCount() == 1:
-                handle = pynvml.nvmlDeviceGetHandleByIndex(0)
-            self.handle = handle
-            self.nvml = pynvml
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
-            self.ok = handle is not None
+            u = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            self.uuid = u if u.startswith("GPU-") else "GPU-" + u
         except Exception:
-            self.ok = False
+            self.uuid = None
 
-    def _run(self):
-        n = self.nvml
-        while not self._stop.is_set():
+    def _read(self):
+        import datetime
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 4:
+                continue
             try:
-                self.samples.append(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM))
-                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
-                for name, bit in self.REASONS.items():
-                    if mask & bit:
-                        self.reasons.add(name)
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                sm, mx = float(parts[1]), float(parts[2])
+                mask = int(parts[3], 16)
+            except ValueError:
+                continue
+            self.max_mhz = mx
+            self.samples.append((ts, sm, mask))
+
+    def start(self):
+        import shutil
+        import subprocess
+        exe = shutil.which("nvidia-smi")
+        if exe is None or self.uuid is None:
+            return
+        cmd = [exe, "-i", self.uuid, "--query-gpu=timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)]
+        self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        # let the first samples arrive before the region starts
+        deadline = time.time() + 3.0
+        while not self.samples and time.time() < deadline and self.proc.poll() is None:
+            time.sleep(0.01)
+
+    def stop(self):
+        if self.proc is not None:
+            time.sleep(2 * self.INTERVAL_MS / 1000)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
             except Exception:
-                pass
-            time.sleep(0.005)
+                self.proc.kill()
+            self.reader.join(timeout=5)
 
     def __enter__(self):
-        if self.ok:
-            self._thread = threading.Thread(target=self._run, daemon=True)
-            self._thread.start()
+        import datetime
+        self.t0 = datetime.datetime.now()
         return self
 
     def __exit__(self, *exc):
-        if self._thread:
-            self._stop.set()
-            self._thread.join()
+        import datetime
+        self.t1 = datetime.datetime.now()
 
     def summary(self):
-        if not self.ok or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                    "samples": len(self.samples)}
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        import datetime
+        if not self.samples or self.t0 is None or self.t1 is None:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvidia-smi" if self.proc is not None else "unavailable"}
+        slack = datetime.timedelta(milliseconds=self.INTERVAL_MS)
+        inside = [(sm, m) for ts, sm, m in self.samples if self.t0 - slack <= ts <= self.t1 + slack]
+        reasons = sorted({name for _, m in inside for name, bit in self.REASONS.items() if m & bit})
+        return {"sm_mhz": float(statistics.median([sm for sm, _ in inside])) if inside else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
+                "source": f"nvidia-smi -lms {self.INTERVAL_MS}, samples inside the timed region"}
 
 
 # ---------------------------------------------------------------------------
@@ -352,6 +377,62 @@ def measure_variants(isoq, synth, torch, dev, stream, x1, seed0, reps=5):
                         f"channels and RoPE; d={d1}, {bits}-bit", "by_variant": out}
 
 
+def measure_rotor_comparison(isoq, torch, dev, stream, n=1 << 20, reps=3):
+    """IsoQuant-Full against the RotorQuant comparator on the stage-1 sweep:
+    d in {128, 256, 512} x bits in {2, 3, 4} x {float16, float32}, N = 2^20
+    normalised N(0, I_d) vectors; quantize + dequantize time of each, CUDA
+    events on the launching stream."""
+    rows = []
+    gen = torch.Generator(device=dev)
+    for d in (128, 256, 512):
+        p = torch.from_numpy(isoq.isoq_make_params(d, isoq.ISOQ_FULL, 1, 1)).to(dev)
+        rot = torch.from_numpy(isoq.isoq_rotor_make_params(d, 1, 1)).to(dev)
+        for dt in (torch.float16, torch.float32):
+            gen.manual_seed(1000 + d)
+            x = torch.randn((1, n, d), generator=gen, device=dev)
+            x = (x / x.norm(dim=-1, keepdim=True)).to(dt)
+            r = torch.empty_like(x)
+            nrm = torch.empty((1, n), dtype=torch.float16, device=dev)
+            for bits in (2, 3, 4):
+                # outputs allocated once per arm: the timed calls launch kernels only
+                ci = torch.empty((1, n, isoq.isoq_packed_bytes(d, bits)), dtype=torch.uint8, device=dev)
+                cr = torch.empty((1, n, isoq.isoq_rotor_packed_bytes(d, bits)), dtype=torch.uint8, device=dev)
+                arms = {
+                    "isoquant": (lambda b=bits: isoq.isoq_quantize(x, p, b, isoq.ISOQ_FULL, codes=ci, norms=nrm),
+                                 lambda c, s, b=bits: isoq.isoq_dequantize(c, s, p, d, b, isoq.ISOQ_FULL, out=r)),
+                    "rotorquant": (lambda b=bits: isoq.isoq_rotor_quantize(x, rot, b, codes=cr, norms=nrm),
+                                   lambda c, s, b=bits: isoq.isoq_rotor_dequantize(c, s, rot, d, b, out=r)),
+                }
+                row = {"d": d, "bits": bits, "dtype": "f16" if dt == torch.float16 else "f32"}
+                for name, (qf, df) in arms.items():
+                    c, s_ = qf()
+                    df(c, s_)
+                    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                    e[0].record(stream)
+                    for _ in range(reps):
+                        qf()
+                    e[1].record(stream)
+                    for _ in range(reps):
+                        df(c, s_)
+                    e[2].record(stream)
+                    torch.cuda.synchronize()
+                    xf = x.float()
+                    mse = float(((r.float() - xf) ** 2).sum(-1).mean())
+                    row[name] = {"quantize_ms": e[0].elapsed_time(e[1]) / reps,
+                                 "dequantize_ms": e[1].elapsed_time(e[2]) / reps, "mse": mse}
+                iq, rq = row["isoquant"], row["rotorquant"]
+                row["speedup"] = (rq["quantize_ms"] + rq["dequantize_ms"]) / (iq["quantize_ms"] + iq["dequantize_ms"])
+                rows.append(row)
+                del ci, cr
+            del x, r, nrm
+    assert isoq.isoq_check_device_error() == 0
+    speedups = [r["speedup"] for r in rows]
+    return {"workload": "stage-1 sweep: d in {128,256,512} x bits in {2,3,4} x {f16,f32}, 2^20 unit "
+                        "vectors; quantize + dequantize, IsoQuant-Full vs the RotorQuant comparator",
+            "mean_speedup": sum(speedups) / len(speedups), "min_speedup": min(speedups),
+            "max_speedup": max(speedups), "settings": rows}
+
+
 def run_isoq(args):
     import torch
 
@@ -441,24 +522,28 @@ def run_isoq(args):
         if ev:
             ev[4].record(stream)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert isoq.isoq_check_device_error() == 0
-
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with sampler:
-        start.record(stream)
-        for i in range(args.steps):
-            step(events[i])
-        end.record(stream)
+    sampler.start()
+    try:
+        for _ in range(args.warmup):
+            step()
         torch.cuda.synchronize()
+        assert isoq.isoq_check_device_error() == 0
+
+        events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with sampler:
+            start.record(stream)
+            for i in range(args.steps):
+                step(events[i])
+            end.record(stream)
+            torch.cuda.synchronize()
+    finally:
+        sampler.stop()
     if dist:
         dist.barrier()
     total_ms = start.elapsed_time(end)
@@ -524,6 +609,7 @@ def run_isoq(args):
 
     # ---- rotation variants (IsoQuant's 2-D case, RotaryQuant §4.6 v1, v2) ----
     variants = measure_variants(isoq, synth, torch, dev, stream, x1, seed0) if not args.no_variants else None
+    comparator = measure_rotor_comparison(isoq, torch, dev, stream) if not args.no_comparator else None
 
     # ---- reduce over ranks: max time, summed bytes ----
     total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms, t_app, t_dstep = max_over_ranks(
@@ -563,6 +649,7 @@ def run_isoq(args):
                                 "then decode attention over the cache at half capacity; timed "
                                 "outside the main region"},
         "variants": variants,
+        "rotorquant_comparison": comparator,
         "gpu_launches": 4 * args.steps,
         "clocks": sampler.summary(),
     }
@@ -588,6 +675,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle CPU baseline (profiling runs)")
+    ap.add_argument("--no-comparator", action="store_true",
+                    help="skip the IsoQuant vs RotorQuant stage-1 sweep")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the rotation-variant measurements (2-D case, ablation v1/v2)")
     ap.add_argument("--no-e2e", action="store_true",

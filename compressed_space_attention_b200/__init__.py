@@ -34,6 +34,11 @@ from .binding import (  # noqa: F401
     isoq_packed_bytes,
     isoq_params_size,
     isoq_quantize,
+    isoq_rotor_dequantize,
+    isoq_rotor_groups,
+    isoq_rotor_make_params,
+    isoq_rotor_packed_bytes,
+    isoq_rotor_quantize,
     last_error,
     lib,
     status_string,

@@ -58,6 +58,11 @@ SIGNATURES = [
     ("isoq_decode_step", _I, [_P, _P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _P, _P,
                               _F, _P, _P, _SZ, _P]),
     ("isoq_check_device_error", _I, [_P]),
+    ("isoq_rotor_groups", _I, [_I]),
+    ("isoq_rotor_packed_bytes", _SZ, [_I, _I]),
+    ("isoq_rotor_make_params", _I, [_I, ctypes.c_uint64, _I, _P]),
+    ("isoq_rotor_quantize", _I, [_P, _I, _I, _I64, _I, _I, _I64, _I64, _P, _P, _P, _I64, _P]),
+    ("isoq_rotor_dequantize", _I, [_P, _P, _I, _I64, _I, _I, _I64, _P, _P, _I, _I64, _I64, _P]),
     ("isoq_decode_static_workspace_bytes", _SZ, []),
     ("isoq_decode_attention_static", _I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I,
                                           _I, _P, _P, _F, _P, _P]),
@@ -243,6 +248,61 @@ def isoq_dequantize(codes, norms, params, d: int, bits: int, variant: int, out_d
                                    in_head_stride, _ptr(params), _ptr(out), _dtype_code(out),
                                    out.stride(0), out.stride(1), _stream(dev, stream))
     _check(st, "isoq_dequantize")
+    return out
+
+
+def isoq_rotor_groups(d: int) -> int:
+    return lib().isoq_rotor_groups(d)
+
+
+def isoq_rotor_packed_bytes(d: int, bits: int) -> int:
+    return lib().isoq_rotor_packed_bytes(d, bits)
+
+
+def isoq_rotor_make_params(d: int, seed: int, n_heads: int = 1) -> np.ndarray:
+    """float32 [n_heads][G][4] unit rotors (s, p12, p13, p23) (host array)."""
+    out = np.empty((n_heads, max(isoq_rotor_groups(d), 0), 4), dtype=np.float32)
+    _check(lib().isoq_rotor_make_params(d, ctypes.c_uint64(seed & (2 ** 64 - 1)), n_heads,
+                                        out.ctypes.data_as(_P)), "isoq_rotor_make_params")
+    return out
+
+
+def isoq_rotor_quantize(x, rotors, bits: int, codes=None, norms=None, stream=None):
+    """RotorQuant comparator: compresses x [n_heads][n_vec][d]; returns (codes, norms)."""
+    torch = _torch()
+    if x.dim() == 2:
+        x = x.unsqueeze(0)
+    n_heads, n_vec, d = x.shape
+    if x.stride(2) != 1:
+        raise ValueError("the last dimension of x must be contiguous")
+    dev = _require_cuda(x, rotors, codes, norms)
+    if codes is None:
+        codes = torch.empty((n_heads, n_vec, isoq_rotor_packed_bytes(d, bits)), dtype=torch.uint8, device=dev)
+    if norms is None:
+        norms = torch.empty((n_heads, n_vec), dtype=torch.float16, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().isoq_rotor_quantize(_ptr(x), _dtype_code(x), n_heads, n_vec, d, bits, x.stride(0),
+                                       x.stride(1), _ptr(rotors), _ptr(codes), _ptr(norms), n_vec,
+                                       _stream(dev, stream))
+    _check(st, "isoq_rotor_quantize")
+    return codes, norms
+
+
+def isoq_rotor_dequantize(codes, norms, rotors, d: int, bits: int, out_dtype=None, out=None, stream=None):
+    """RotorQuant comparator: reconstructs [n_heads][n_vec][d] from codes and norms."""
+    torch = _torch()
+    if codes.dim() == 2:
+        codes = codes.unsqueeze(0)
+        norms = norms.unsqueeze(0)
+    n_heads, n_vec, _ = codes.shape
+    dev = _require_cuda(codes, norms, rotors, out)
+    if out is None:
+        out = torch.empty((n_heads, n_vec, d), dtype=out_dtype or torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().isoq_rotor_dequantize(_ptr(codes), _ptr(norms), n_heads, n_vec, d, bits, n_vec,
+                                         _ptr(rotors), _ptr(out), _dtype_code(out), out.stride(0),
+                                         out.stride(1), _stream(dev, stream))
+    _check(st, "isoq_rotor_dequantize")
     return out
 
 

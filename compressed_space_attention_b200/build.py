@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(HERE, "libisoq.so")
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3",
                 "-I", INCLUDE, "-I", CSRC]
-SOURCES = ["isoq_host.cpp", "isoq_quant.cu", "isoq_decode.cu", "isoq_runtime.cu"]
+SOURCES = ["isoq_host.cpp", "isoq_quant.cu", "isoq_decode.cu", "isoq_runtime.cu", "rotor_quant.cu"]
 
 
 def _nvcc() -> str:

@@ -255,6 +255,27 @@ int isoq_make_params(int d, int variant, uint64_t seed, int n_heads, float *out_
   return ISOQ_OK;
 }
 
+int isoq_rotor_make_params(int d, uint64_t seed, int n_heads, float *out_host) {
+  clear_error();
+  if (!supported_d(d)) return set_error(ISOQ_ERR_UNSUPPORTED, "d=%d not supported", d);
+  if (n_heads < 0) return set_error(ISOQ_ERR_INVALID_ARG, "n_heads < 0");
+  if (n_heads > 0 && !out_host) return set_error(ISOQ_ERR_INVALID_ARG, "out_host is NULL");
+  const int G = (d + 2) / 3;
+  Gaussian g;
+  g.rng.s = seed;
+  float *p = out_host;
+  for (int h = 0; h < n_heads; ++h) {
+    for (int k = 0; k < G; ++k) {
+      double v[4];
+      for (int j = 0; j < 4; ++j) v[j] = g.next();
+      const double n = std::sqrt(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
+      for (int j = 0; j < 4; ++j) p[j] = static_cast<float>(v[j] / n);
+      p += 4;
+    }
+  }
+  return ISOQ_OK;
+}
+
 int isoq_make_codebook(int d, int bits, double *centroids_host, double *thresholds_host) {
   clear_error();
   if (!supported_d(d)) return set_error(ISOQ_ERR_UNSUPPORTED, "d=%d not supported", d);

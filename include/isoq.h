@@ -306,6 +306,39 @@ int isoq_decode_step(const void *q_dev, const void *k_new_dev, const void *v_new
                      size_t workspace_bytes, isoq_stream_t stream);
 
 /*
+ * RotorQuant comparator (the RotorQuant page; [IQ] abstract compares
+ * IsoQuant's kernels with it on the stage-1 path).  Each vector is padded
+ * to 3G dimensions, G = ceil(d / 3), each group of three is rotated by its
+ * own unit rotor R = s + p12 e12 + p13 e13 + p23 e23 of Cl(3,0) with the
+ * sandwich R v rev(R), and all 3G rotated coordinates get the Lloyd-Max
+ * codes of isoq_make_codebook (N(0, 1/d)), packed as one LSB-first
+ * bitstream (code i at bits [b i, b i + b)) padded to whole 32-bit words;
+ * the float16 norm is stored as for isoq_quantize.
+ *
+ * isoq_rotor_groups(d): G, or ISOQ_ERR_UNSUPPORTED.
+ * isoq_rotor_packed_bytes(d, bits): 4 ceil(3 G bits / 32) (52 at d = 128,
+ *   bits = 3), or 0 for unsupported arguments.
+ * isoq_rotor_make_params: out_host[n_heads][G][4] = (s, p12, p13, p23),
+ *   four normals per group from the generator of isoq_make_params,
+ *   normalised in double, rounded to float32.  Host only.
+ * isoq_rotor_quantize / isoq_rotor_dequantize: arguments, layouts, strides
+ *   and errors as isoq_quantize / isoq_dequantize, with rotors_dev
+ *   [n_heads][G][4] (16-byte aligned) in place of the rotation parameters,
+ *   codes of isoq_rotor_packed_bytes per vector (4-byte aligned).
+ */
+int isoq_rotor_groups(int d);
+size_t isoq_rotor_packed_bytes(int d, int bits);
+int isoq_rotor_make_params(int d, uint64_t seed, int n_heads, float *out_host);
+int isoq_rotor_quantize(const void *x_dev, int dtype, int n_heads, int64_t n_vec, int d, int bits,
+                        int64_t head_stride, int64_t vec_stride, const float *rotors_dev,
+                        uint8_t *codes_dev, uint16_t *norms_dev, int64_t out_head_stride,
+                        isoq_stream_t stream);
+int isoq_rotor_dequantize(const uint8_t *codes_dev, const uint16_t *norms_dev, int n_heads,
+                          int64_t n_vec, int d, int bits, int64_t in_head_stride,
+                          const float *rotors_dev, void *out_dev, int out_dtype,
+                          int64_t head_stride, int64_t vec_stride, isoq_stream_t stream);
+
+/*
  * Reads and clears the current device's error word after synchronising
  * `stream`.  Returns ISOQ_OK, ISOQ_ERR_TIMEOUT if a kernel's bounded wait
  * gave up since the last check (the kernel then stopped early and its
