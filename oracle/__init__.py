@@ -28,6 +28,7 @@ from .isoquant import (  # noqa: F401
     make_params,
     packed_bytes,
     planar_forward,
+    prefill_attention,
     qconj,
     quantize,
     quantize_scalar,

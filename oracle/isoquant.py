@@ -599,6 +599,33 @@ def decode_attention(q, packed_k, packed_v, norms_k, norms_v, seq_lens,
     return out
 
 
+def prefill_attention(q, packed_k, packed_v, norms_k, norms_v, seq_lens,
+                      params_k, params_v, bits: int, variant: int, scale: float):
+    """Causal attention of a chunk of Tq new queries over the packed cache
+    that already holds them ([RQ] §3.4 "early termination via causal
+    masking" in kernel A; Figure 1's path with T_q > 1).
+
+    q: [B][Tq][Hq][d]; the cache as in ``decode_attention``, with
+    seq_lens[b] the cache length including the chunk.  Query t of row b sits
+    at position p = seq_lens[b] - Tq + t and attends to tokens
+    j <= p (and j < Tmax); a query with p < 0 gets a zero row.  Each query
+    row is the compressed-space decode of ``decode_attention`` with
+    p + 1 tokens.  Returns float64 [B][Tq][Hq][d].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    bsz, tq, hq, d = q.shape
+    out = np.zeros((bsz, tq, hq, d), dtype=np.float64)
+    for b in range(bsz):
+        for t in range(tq):
+            pos = int(seq_lens[b]) - tq + t
+            if pos < 0:
+                continue
+            out[b, t] = decode_attention(q[b:b + 1, t], packed_k[b:b + 1], packed_v[b:b + 1],
+                                         norms_k[b:b + 1], norms_v[b:b + 1], [pos + 1],
+                                         params_k, params_v, bits, variant, scale)[0]
+    return out
+
+
 def decode_attention_reconstructed(q, packed_k, packed_v, norms_k, norms_v,
                                    seq_lens, params_k, params_v, bits: int,
                                    variant: int, scale: float):

@@ -673,6 +673,44 @@ def test_decode_append_token_by_token_equals_bulk_compression(variant):
     np.testing.assert_array_equal(out[0][2], pk[2])
 
 
+def test_prefill_attention_is_causal_attention_over_the_reconstruction():
+    """Chunked prefill: a dense causal softmax over the dequantised K/V with
+    an explicit mask matrix (query t at position L - Tq + t sees tokens
+    0..position) equals the oracle's compressed-space prefill; the last
+    query equals a full-length decode; splitting the chunk in two changes
+    nothing; queries before the cache start give zero rows."""
+    g = np.random.default_rng(91)
+    d, bits, hkv, hq, tmax, tq = 128, 3, 2, 4, 40, 9
+    pk, pv, nk, nv = _random_cache(g, 2, hkv, tmax, d, bits)
+    prk = O.make_params(d, O.FULL, 1, hkv)
+    prv = O.make_params(d, O.FULL, 2, hkv)
+    q = g.standard_normal((2, tq, hq, d))
+    lens = np.array([33, 5])            # row 1: positions -4..4 (four empty queries)
+    scale = 1 / math.sqrt(d)
+    got = O.prefill_attention(q, pk, pv, nk, nv, lens, prk, prv, bits, O.FULL, scale)
+    for b in range(2):
+        for kvh in range(hkv):
+            kh = O.dequantize(pk[b, kvh:kvh + 1], nk[b, kvh:kvh + 1], prk[kvh:kvh + 1], bits, O.FULL, d)[0]
+            vh = O.dequantize(pv[b, kvh:kvh + 1], nv[b, kvh:kvh + 1], prv[kvh:kvh + 1], bits, O.FULL, d)[0]
+            pos = lens[b] - tq + np.arange(tq)
+            mask = np.arange(tmax)[None, :] <= pos[:, None]
+            for hh in range(hq // hkv):
+                qh = kvh * (hq // hkv) + hh
+                z = q[b, :, qh] @ kh.T * scale
+                z = np.where(mask, z, -np.inf)
+                zmax = np.max(z, axis=1, keepdims=True)
+                w = np.where(mask, np.exp(z - np.where(np.isfinite(zmax), zmax, 0)), 0.0)
+                den = w.sum(axis=1, keepdims=True)
+                o = np.where(den > 0, (w @ vh) / np.where(den > 0, den, 1), 0.0)
+                np.testing.assert_allclose(got[b, :, qh], o, atol=1e-12)
+    np.testing.assert_array_equal(got[1, :4], 0.0)
+    last = O.decode_attention(q[:, -1], pk, pv, nk, nv, lens, prk, prv, bits, O.FULL, scale)
+    np.testing.assert_allclose(got[:, -1], last, atol=1e-13)
+    a = O.prefill_attention(q[:, :4], pk, pv, nk, nv, lens - 5, prk, prv, bits, O.FULL, scale)
+    b2 = O.prefill_attention(q[:, 4:], pk, pv, nk, nv, lens, prk, prv, bits, O.FULL, scale)
+    np.testing.assert_allclose(np.concatenate([a, b2], axis=1), got, atol=1e-13)
+
+
 def test_split_k_combine_is_partition_independent():
     g = np.random.default_rng(51)
     t, d = 300, 16
