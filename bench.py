@@ -433,6 +433,60 @@ def measure_rotor_comparison(isoq, torch, dev, stream, n=1 << 20, reps=3):
             "max_speedup": max(speedups), "settings": rows}
 
 
+PREFILL_WORKLOADS = [
+    # (name, B, Hq, Hkv, context, chunk, d)
+    ("chunk2048_ctx32768_gqa32_4_d128", 1, 32, 4, 32768, 2048, 128),
+    ("chunk1024_ctx65536_gqa16_8_d256", 1, 16, 8, 65536, 1024, 256),
+]
+
+
+def measure_prefill(isoq, synth, torch, dev, stream, seed0, peak_tflops, reps=5):
+    """Chunked prefill (causal attention of the chunk's queries over the packed
+    cache that holds them) on each PREFILL_WORKLOADS shape: the cache is drawn
+    with the Student-t generator and compressed by isoq_quantize, the queries
+    are float16 N(0, 1).  Algorithmic FLOPs: 4 d per (query head, visible
+    token) (QK and PV multiply-adds, the causal triangle included)."""
+    out = {}
+    for name, B, Hq, Hkv, ctx, tq, d in PREFILL_WORKLOADS:
+        bits, variant, pb = 3, isoq.ISOQ_FULL, d * 3 // 8
+        prk = torch.from_numpy(isoq.isoq_make_params(d, variant, 1, Hkv)).to(dev)
+        prv = torch.from_numpy(isoq.isoq_make_params(d, variant, 2, Hkv)).to(dev)
+        k, v = synth.student_t_kv_torch(B, Hkv, ctx, d, seed=seed0 + 51, device=dev)
+        pk, nk = isoq.isoq_quantize(k.view(-1, ctx, d), prk.repeat(B, 1, 1), bits, variant)
+        pv, nv = isoq.isoq_quantize(v.view(-1, ctx, d), prv.repeat(B, 1, 1), bits, variant)
+        del k, v
+        pk, pv = pk.view(B, Hkv, ctx, pb), pv.view(B, Hkv, ctx, pb)
+        nk, nv = nk.view(B, Hkv, ctx), nv.view(B, Hkv, ctx)
+        q = synth.queries_torch(B * tq, Hq, d, seed=seed0 + 52, device=dev).view(B, tq, Hq, d)
+        lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+        o = torch.empty_like(q)
+        for _ in range(2):
+            isoq.isoq_prefill_attention(q, pk, pv, nk, nv, lens, prk, prv, bits, variant, out=o)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            isoq.isoq_prefill_attention(q, pk, pv, nk, nv, lens, prk, prv, bits, variant, out=o)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert isoq.isoq_check_device_error() == 0
+        ms = e0.elapsed_time(e1) / reps
+        visible = sum(ctx - tq + t + 1 for t in range(tq))        # tokens seen by the chunk's queries
+        flops = 4.0 * d * Hq * B * visible
+        kv_bytes = B * Hkv * ctx * 2 * (pb + 2)
+        tflops = flops / (ms * 1e-3) / 1e12
+        out[name] = {"ms": ms, "tflops": tflops, "frac_of_tensor_peak": tflops / peak_tflops,
+                     "queries_per_s": B * tq / (ms * 1e-3), "kv_bytes": kv_bytes,
+                     "kernel": f"prefill_kernel<__half, {d}, Full, GP={Hq // Hkv}>"}
+        del pk, pv, nk, nv, q, o
+    torch.cuda.empty_cache()
+    return {"workloads": out, "peak_tflops": peak_tflops,
+            "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst; float16 runs at the bf16 rate)",
+            "what": "isoq_prefill_attention: one chunk of float16 queries at the end of the context, "
+                    "causal, 3-bit Full, mma.sync float16 tiles"}
+
+
 def run_isoq(args):
     import torch
 
@@ -610,6 +664,9 @@ def run_isoq(args):
     # ---- rotation variants (IsoQuant's 2-D case, RotaryQuant §4.6 v1, v2) ----
     variants = measure_variants(isoq, synth, torch, dev, stream, x1, seed0) if not args.no_variants else None
     comparator = measure_rotor_comparison(isoq, torch, dev, stream) if not args.no_comparator else None
+    peaks_all, _ = measured_peaks()
+    prefill = (measure_prefill(isoq, synth, torch, dev, stream, seed0,
+                               float(peaks_all.get("bf16_tflops", 1590.0))) if not args.no_prefill else None)
 
     # ---- reduce over ranks: max time, summed bytes ----
     total_ms, t_decode, t_split, t_quant, t_deq, t_comb, e2e_ms, t_app, t_dstep = max_over_ranks(
@@ -650,6 +707,7 @@ def run_isoq(args):
                                 "outside the main region"},
         "variants": variants,
         "rotorquant_comparison": comparator,
+        "prefill": prefill,
         "gpu_launches": 4 * args.steps,
         "clocks": sampler.summary(),
     }
@@ -675,6 +733,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle CPU baseline (profiling runs)")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the chunked-prefill attention measurement")
     ap.add_argument("--no-comparator", action="store_true",
                     help="skip the IsoQuant vs RotorQuant stage-1 sweep")
     ap.add_argument("--no-variants", action="store_true",

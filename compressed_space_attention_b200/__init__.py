@@ -33,6 +33,7 @@ from .binding import (  # noqa: F401
     isoq_make_params,
     isoq_packed_bytes,
     isoq_params_size,
+    isoq_prefill_attention,
     isoq_quantize,
     isoq_rotor_dequantize,
     isoq_rotor_groups,

@@ -58,6 +58,8 @@ SIGNATURES = [
     ("isoq_decode_step", _I, [_P, _P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _P, _P,
                               _F, _P, _P, _SZ, _P]),
     ("isoq_check_device_error", _I, [_P]),
+    ("isoq_prefill_attention", _I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _I, _I,
+                                    _P, _P, _F, _P, _P]),
     ("isoq_rotor_groups", _I, [_I]),
     ("isoq_rotor_packed_bytes", _SZ, [_I, _I]),
     ("isoq_rotor_make_params", _I, [_I, ctypes.c_uint64, _I, _P]),
@@ -248,6 +250,31 @@ def isoq_dequantize(codes, norms, params, d: int, bits: int, variant: int, out_d
                                    in_head_stride, _ptr(params), _ptr(out), _dtype_code(out),
                                    out.stride(0), out.stride(1), _stream(dev, stream))
     _check(st, "isoq_dequantize")
+    return out
+
+
+def isoq_prefill_attention(q, packed_k, packed_v, norms_k, norms_v, seq_lens, params_k, params_v,
+                           bits: int, variant: int, scale: Optional[float] = None, out=None, stream=None):
+    """Causal attention of q [B][Tq][Hq][d] over the packed cache that holds
+    the chunk (seq_lens counts it); returns out [B][Tq][Hq][d] (dtype of q)."""
+    torch = _torch()
+    B, Tq, Hq, d = q.shape
+    _, Hkv, Tmax, pb = packed_k.shape
+    if pb != isoq_packed_bytes(d, bits):
+        raise ValueError("packed row size does not match d and bits")
+    if not q.is_contiguous():
+        raise ValueError("q must be contiguous")
+    dev = _require_cuda(q, packed_k, packed_v, norms_k, norms_v, seq_lens, params_k, params_v, out)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Tq, Hq, d), dtype=q.dtype, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().isoq_prefill_attention(
+            _ptr(q), _dtype_code(q), _ptr(packed_k), _ptr(packed_v), _ptr(norms_k), _ptr(norms_v),
+            _ptr(seq_lens), B, Tq, Hq, Hkv, Tmax, d, bits, variant, _ptr(params_k), _ptr(params_v),
+            float(scale), _ptr(out), _stream(dev, stream))
+    _check(st, "isoq_prefill_attention")
     return out
 
 

@@ -293,6 +293,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
 
 #include "decode_i8.cuh"
 #include "decode_append.cuh"
+#include "prefill.cuh"
 
 // ---------------------------------------------------------------------------
 // Host launchers
@@ -569,6 +570,56 @@ int isoq_decode_step(const void *q_dev, const void *k_new_dev, const void *v_new
   return isoq_decode_attention(q_dev, dtype, packed_k_dev, packed_v_dev, norms_k_dev, norms_v_dev,
                                seq_lens_dev, B, Hq, Hkv, Tmax, d, bits, variant, params_k_dev,
                                params_v_dev, scale, out_dev, workspace_dev, workspace_bytes, stream);
+}
+
+int isoq_prefill_attention(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
+                           const uint8_t *packed_v_dev, const uint16_t *norms_k_dev,
+                           const uint16_t *norms_v_dev, const int32_t *seq_lens_dev, int B, int Tq,
+                           int Hq, int Hkv, int64_t Tmax, int d, int bits, int variant,
+                           const float *params_k_dev, const float *params_v_dev, float scale,
+                           void *out_dev, isoq_stream_t stream) {
+  clear_error();
+  if (d != 128 && d != 256) return set_error(ISOQ_ERR_UNSUPPORTED, "prefill: d=%d (128 or 256)", d);
+  if (bits != 3) return set_error(ISOQ_ERR_UNSUPPORTED, "prefill: bits=%d (3)", bits);
+  if (!supported_decode_variant(variant)) return set_error(ISOQ_ERR_UNSUPPORTED, "variant=%d", variant);
+  if (dtype != ISOQ_F16) return set_error(ISOQ_ERR_UNSUPPORTED, "prefill: dtype=%d (float16 queries)", dtype);
+  if (B <= 0 || Tq < 0 || Hq <= 0 || Hkv <= 0 || Tmax <= 0)
+    return set_error(ISOQ_ERR_INVALID_ARG, "B, Hq, Hkv and Tmax must be positive, Tq >= 0");
+  if (Hq % Hkv) return set_error(ISOQ_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return set_error(ISOQ_ERR_UNSUPPORTED, "prefill: Hq/Hkv=%d (1, 2, 4 or 8)", G);
+  if (Tmax >= (1ll << 31) || B > 65535 || Hkv > 65535 || Tq > (1 << 24))
+    return set_error(ISOQ_ERR_INVALID_ARG, "shape too large");
+  if (Tmax % 8) return set_error(ISOQ_ERR_UNSUPPORTED, "prefill: Tmax %% 8 != 0");
+  if (!q_dev || !packed_k_dev || !packed_v_dev || !norms_k_dev || !norms_v_dev || !seq_lens_dev ||
+      !params_k_dev || !params_v_dev || !out_dev)
+    return set_error(ISOQ_ERR_INVALID_ARG, "null pointer");
+  if (!decode::aligned(packed_k_dev, 16) || !decode::aligned(packed_v_dev, 16) ||
+      !decode::aligned(params_k_dev, 16) || !decode::aligned(params_v_dev, 16) ||
+      !decode::aligned(q_dev, 4) || !decode::aligned(out_dev, 4) || !decode::aligned(norms_k_dev, 2) ||
+      !decode::aligned(norms_v_dev, 2) || !decode::aligned(seq_lens_dev, 4))
+    return set_error(ISOQ_ERR_UNSUPPORTED, "misaligned pointer");
+  if (!std::isfinite(scale)) return set_error(ISOQ_ERR_INVALID_ARG, "scale is not finite");
+  if (Tq == 0) return ISOQ_OK;
+  decode::PrefillArgs a{};
+  a.q = q_dev;
+  a.packed_k = packed_k_dev;
+  a.packed_v = packed_v_dev;
+  a.norms_k = norms_k_dev;
+  a.norms_v = norms_v_dev;
+  a.seq_lens = seq_lens_dev;
+  a.params_k = params_k_dev;
+  a.params_v = params_v_dev;
+  a.out = out_dev;
+  a.tmax = Tmax;
+  a.batch = B;
+  a.tq = Tq;
+  a.hq = Hq;
+  a.hkv = Hkv;
+  a.group = G;
+  a.score_unit = static_cast<float>(scale * 1.4426950408889634);
+  return decode::run_prefill(d, block_map_variant(variant), a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

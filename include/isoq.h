@@ -306,6 +306,30 @@ int isoq_decode_step(const void *q_dev, const void *k_new_dev, const void *v_new
                      size_t workspace_bytes, isoq_stream_t stream);
 
 /*
+ * Chunked prefill: causal attention of Tq new queries over the packed cache
+ * that already holds them ([RQ] §3.4: kernel A "benefits from early
+ * termination via causal masking"; Figure 1's compressed-space path with
+ * more than one query).  Query t of batch row b sits at position
+ * p = seq_lens[b] - Tq + t and attends to the tokens j <= p (j < Tmax);
+ * queries with p < 0 get zero rows.  Each output row is what
+ * isoq_decode_attention gives for that query over p + 1 tokens.
+ *   q_dev      [B][Tq][Hq][d] float16 (dtype ISOQ_F16; 4-byte aligned)
+ *   out_dev    [B][Tq][Hq][d] float16, written (4-byte aligned)
+ *   the cache, seq_lens, parameters, scale: as isoq_decode_attention
+ *              (seq_lens[b] counts the chunk; the chunk's K/V are written
+ *              first, e.g. by isoq_quantize into the cache rows).
+ * Tensor-core path: d in {128, 256}, bits = 3, Hq/Hkv in {1, 2, 4, 8},
+ * variants FULL, FAST and PLANAR; anything else is ISOQ_ERR_UNSUPPORTED.
+ * Tq = 0 is a no-op.  No workspace; one launch.
+ */
+int isoq_prefill_attention(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
+                           const uint8_t *packed_v_dev, const uint16_t *norms_k_dev,
+                           const uint16_t *norms_v_dev, const int32_t *seq_lens_dev, int B, int Tq,
+                           int Hq, int Hkv, int64_t Tmax, int d, int bits, int variant,
+                           const float *params_k_dev, const float *params_v_dev, float scale,
+                           void *out_dev, isoq_stream_t stream);
+
+/*
  * RotorQuant comparator (the RotorQuant page; [IQ] abstract compares
  * IsoQuant's kernels with it on the stage-1 path).  Each vector is padded
  * to 3G dimensions, G = ceil(d / 3), each group of three is rotated by its
