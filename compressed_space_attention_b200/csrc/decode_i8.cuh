@@ -120,6 +120,7 @@ __device__ __forceinline__ float lds_half(const unsigned char *p) {
 
 struct I8Lut {
   uint32_t kh0, kh1, kl0, kl1, vh0, vh1, vl0, vl1;
+  uint32_t neg1, one;     // -1 and 1, opaque to the compiler (see group_sel8_im)
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -175,6 +176,31 @@ __device__ __forceinline__ void group_sel8(uint32_t w0, uint32_t w1, uint32_t w2
   // adds, which the compiler may place on the FMA pipe) is their union.
   const uint32_t x0 = w0 - m0, x1 = w1 - m1, x2 = w2 - m2;
   const uint32_t sum = (x0 >> 2) + (x1 >> 1) + x2;   // code 24+j at bits 4j+1 .. 4j+3
+  s[0] = m0;
+  s[1] = m0 >> 16;
+  s[2] = m1;
+  s[3] = m1 >> 16;
+  s[4] = m2;
+  s[5] = m2 >> 16;
+  s[6] = sum >> 1;
+  s[7] = sum >> 17;
+}
+
+__device__ __forceinline__ uint32_t imad_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+// group_sel8 with the spare-bit planes and their sum formed by multiply-adds
+// whose factors (-1, 1) arrive as kernel parameters: the compiler cannot
+// turn them into logic ops, so that work moves from the integer (ALU) pipe,
+// which bounds the decode, to the separate multiply-add pipe.
+__device__ __forceinline__ void group_sel8_im(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t (&s)[8],
+                                              uint32_t neg1, uint32_t one) {
+  const uint32_t m0 = w0 & 0x77777777u, m1 = w1 & 0x77777777u, m2 = w2 & 0x77777777u;
+  const uint32_t x0 = imad_u32(m0, neg1, w0), x1 = imad_u32(m1, neg1, w1), x2 = imad_u32(m2, neg1, w2);
+  const uint32_t sum = imad_u32(x0 >> 2, one, imad_u32(x1 >> 1, one, x2));
   s[0] = m0;
   s[1] = m0 >> 16;
   s[2] = m1;
@@ -410,8 +436,8 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
 #pragma unroll
       for (int gq = 0; gq < C::GRP_QK; ++gq) {
         uint32_t sa[8], sb[8];
-        group_sel8(wg[3 * gq], wg[3 * gq + 1], wg[3 * gq + 2], sa);
-        group_sel8(wg8[3 * gq], wg8[3 * gq + 1], wg8[3 * gq + 2], sb);
+        group_sel8_im(wg[3 * gq], wg[3 * gq + 1], wg[3 * gq + 2], sa, lut.neg1, lut.one);
+        group_sel8_im(wg8[3 * gq], wg8[3 * gq + 1], wg8[3 * gq + 2], sb, lut.neg1, lut.one);
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
           const int kk = 4 * gq + kq;
@@ -592,7 +618,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const unsigned char *row = vc + (16 * h2 + t + 4 * r) * C::PB + goff;
-          group_sel8(lds32(row), lds32(row + 4), lds32(row + 8), vs[r]);
+          group_sel8_im(lds32(row), lds32(row + 4), lds32(row + 8), vs[r], lut.neg1, lut.one);
         }
       }
 #pragma unroll
@@ -759,7 +785,7 @@ const I8Tables &i8_tables() {
       kl[k / 4] |= (static_cast<uint32_t>(cl) & 0xFFu) << sh;
       vl[k / 4] |= (static_cast<uint32_t>(2 * cl) & 0xFFu) << sh;
     }
-    tb.lut = I8Lut{kh[0], kh[1], kl[0], kl[1], kh[0], kh[1], vl[0], vl[1]};
+    tb.lut = I8Lut{kh[0], kh[1], kl[0], kl[1], kh[0], kh[1], vl[0], vl[1], 0xFFFFFFFFu, 1u};
   });
   return tb;
 }

@@ -34,10 +34,10 @@
 // negation is folded into that group's block matrices.
 //
 // The quantiser compares the unnormalised R x with s * t_k (no division per
-// element) using the symmetry of the codebook: the sign picks the half, and
-// the magnitude is counted against the positive thresholds.  Both decisions
-// are exact 0/1 steps from saturating FMAs, so the search and the packing of
-// the codes run as float arithmetic on the FMA pipe.
+// element) using the symmetry of the codebook: the magnitude is counted
+// against the positive thresholds with exact 0/1 steps from saturating FMAs,
+// and the sign, taken by the integer pipe, signs the field weight with which
+// one FMA adds the code into its packed word.
 //
 // Data movement.  Each warp of a quantize CTA streams its own rows through a
 // ring of 128B-swizzled TMA tiles (no producer warp); each lane reads its own
@@ -262,20 +262,13 @@ __device__ __forceinline__ void wht_cross_full(uint64_t (&xp)[kPairs], int part)
 // The Lloyd-Max search runs on the FMA pipe.  With `big` a power of two that
 // scales a coordinate of the vector to about 2^40 (one float ulp of any scaled
 // threshold is then >= 1), fma.sat(|y|, big, -t big) is exactly 1.0 when
-// |y| > t and 0.0 otherwise (ties go to the lower code).  The sign step uses
-// two multiplies by 2^127, which take any nonzero y to +-inf-or-beyond-1 and
-// keep +-0 at 0.  Codes are then small exact integers in float32, and the
-// packing accumulates them as exact integers below 2^24 (offset by 2^23, so
-// that the low 16 bits of the float are the packed field).
+// |y| > t and 0.0 otherwise (ties go to the lower code).  Codes are then
+// small exact integers in float32, and the packing accumulates them as exact
+// integers below 2^24 (offset by 2^23, so that the low 16 bits of the float
+// are the packed field).
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   float r;
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-__device__ __forceinline__ float mul_sat(float a, float b) {
-  float r;
-  asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
   return r;
 }
 
@@ -290,47 +283,50 @@ __device__ __forceinline__ float search_scale(float norm) {
 // Codes of one group (16 pairs (e, e + 16) from xp[base]) packed into its
 // GB/4 words (layout in common.cuh).  tb[j] = -t_j big for the positive
 // thresholds t_j scaled by the norm.
+//
+// With m = #{j : |y| > t_j} (one saturating FMA per threshold), the code is
+// L/2 + m for y > 0 and L/2 - 1 - m otherwise, i.e. (L/2 - 1/2) + sg (m + 1/2)
+// with sg = +-1.  The packing accumulates code * w for the field weight w of
+// each position as one FMA, (sg w) (m + 1/2), onto the constant
+// 2^22 + (L/2 - 1/2) sum w; sg w is w with its sign bit set from y by the
+// integer pipe.  Every partial sum is a multiple of 1/2 in [2^22, 2^23),
+// where float32 steps by 1/2, so all of it is exact, and the packed field
+// is the float's mantissa shifted right by one bit.
 template <int BITS>
 __device__ __forceinline__ void quantize_group(const uint64_t (&xp)[kPairs], int base,
                                                const float *tb, float big, uint32_t *w) {
   constexpr int L = 1 << BITS, NPOS = L / 2 - 1;
-  const float p127 = 1.7014118346046923e38f;   // 2^127
-  const uint64_t one2 = f2_pack(1.f, 1.f), two2 = f2_pack(2.f, 2.f);
-  const uint64_t low2 = f2_pack(static_cast<float>(L / 2 - 1), static_cast<float>(L / 2 - 1));
-  uint64_t cp[kGP];   // (code of element e, code of element e + 16) per pair
-#pragma unroll
-  for (int p = 0; p < kGP; ++p) {
-    float y0, y1;
-    f2_unpack(xp[base + p], y0, y1);
-    const float a0 = fabsf(y0), a1 = fabsf(y1);
-    // m = #{j : |y| > t_j}
-    uint64_t m = f2_pack(fma_sat(a0, big, tb[0]), fma_sat(a1, big, tb[0]));
-#pragma unroll
-    for (int j = 1; j < NPOS; ++j) m = f2_add(m, f2_pack(fma_sat(a0, big, tb[j]), fma_sat(a1, big, tb[j])));
-    // s = [y > 0]
-    const uint64_t s = f2_pack(mul_sat(y0 * p127, p127), mul_sat(y1 * p127, p127));
-    // code = s ? L/2 + m : L/2 - 1 - m  =  (L/2 - 1 - m) + s (2m + 1)
-    cp[p] = f2_fma(s, f2_fma(m, two2, one2), f2_sub(low2, m));
-  }
-  // Exact integer packing: acc_q = 2^23 + sum of the pair's codes times their
-  // field weights; the low 16 bits of each float are one half word.
   constexpr int PER_HALF = 16 / BITS == 5 ? 4 : 16 / BITS;   // codes per 16-bit half (3 bits: 4-bit fields)
   constexpr int FIELD = BITS == 3 ? 4 : BITS;
   constexpr int NACC = kGP / PER_HALF;
-  const uint64_t magic2 = f2_pack(8388608.f, 8388608.f);
+  constexpr float WSUM = static_cast<float>(((1u << (FIELD * PER_HALF)) - 1u) / ((1u << FIELD) - 1u));
+  const float c0 = 4194304.f + (static_cast<float>(L / 2) - 0.5f) * WSUM;
+  const uint64_t half2 = f2_pack(0.5f, 0.5f);
   uint32_t lo[NACC], hi[NACC];
 #pragma unroll
   for (int q = 0; q < NACC; ++q) {
-    uint64_t acc = f2_add(cp[PER_HALF * q], magic2);
+    uint64_t acc = f2_pack(c0, c0);
 #pragma unroll
-    for (int j = 1; j < PER_HALF; ++j) {
-      const float wgt = static_cast<float>(1u << (FIELD * j));
-      acc = f2_fma(cp[PER_HALF * q + j], f2_pack(wgt, wgt), acc);
+    for (int j = 0; j < PER_HALF; ++j) {
+      const int p = PER_HALF * q + j;
+      float y0, y1;
+      f2_unpack(xp[base + p], y0, y1);
+      const float a0 = fabsf(y0), a1 = fabsf(y1);
+      // m + 1/2
+      uint64_t m = f2_pack(fma_sat(a0, big, tb[0]), fma_sat(a1, big, tb[0]));
+#pragma unroll
+      for (int k = 1; k < NPOS; ++k) m = f2_add(m, f2_pack(fma_sat(a0, big, tb[k]), fma_sat(a1, big, tb[k])));
+      m = f2_add(m, half2);
+      // sg w: the field weight, negative unless y > 0 (+-0 count as not positive)
+      const uint32_t wb = __float_as_uint(static_cast<float>(1u << (FIELD * j)));
+      const uint32_t s0 = static_cast<int>(__float_as_uint(y0)) > 0 ? wb : (wb | 0x80000000u);
+      const uint32_t s1 = static_cast<int>(__float_as_uint(y1)) > 0 ? wb : (wb | 0x80000000u);
+      acc = f2_fma(f2_pack(__uint_as_float(s0), __uint_as_float(s1)), m, acc);
     }
     float fl, fh;
     f2_unpack(acc, fl, fh);
-    lo[q] = __float_as_uint(fl);
-    hi[q] = __float_as_uint(fh);
+    lo[q] = __float_as_uint(fl) >> 1;
+    hi[q] = __float_as_uint(fh) >> 1;
   }
   if constexpr (BITS == 2) {
     // words: codes 0..15 (low elements), codes 16..31 (high elements)
