@@ -499,13 +499,16 @@ int launch_prefill(PrefillArgs a, cudaStream_t stream) {
   return ISOQ_OK;
 }
 
+template <typename T, int D, bool FULL, int GP>
+int launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream);
+
 template <typename T, int D, bool FULL>
 int run_prefill_g(const PrefillArgs &a, cudaStream_t st) {
   switch (a.group) {
-    case 1: return launch_prefill<T, D, FULL, 1>(a, st);
-    case 2: return launch_prefill<T, D, FULL, 2>(a, st);
-    case 4: return launch_prefill<T, D, FULL, 4>(a, st);
-    default: return launch_prefill<T, D, FULL, 8>(a, st);
+    case 1: return launch_prefill_tc<T, D, FULL, 1>(a, st);
+    case 2: return launch_prefill_tc<T, D, FULL, 2>(a, st);
+    case 4: return launch_prefill_tc<T, D, FULL, 4>(a, st);
+    default: return launch_prefill_tc<T, D, FULL, 8>(a, st);
   }
 }
 
