@@ -478,13 +478,13 @@ def measure_prefill(isoq, synth, torch, dev, stream, seed0, peak_tflops, reps=5)
         tflops = flops / (ms * 1e-3) / 1e12
         out[name] = {"ms": ms, "tflops": tflops, "frac_of_tensor_peak": tflops / peak_tflops,
                      "queries_per_s": B * tq / (ms * 1e-3), "kv_bytes": kv_bytes,
-                     "kernel": f"prefill_kernel<__half, {d}, Full, GP={Hq // Hkv}>"}
+                     "kernel": f"prefill_tc_kernel<__half, {d}, Full, GP={Hq // Hkv}>"}
         del pk, pv, nk, nv, q, o
     torch.cuda.empty_cache()
     return {"workloads": out, "peak_tflops": peak_tflops,
             "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst; float16 runs at the bf16 rate)",
             "what": "isoq_prefill_attention: one chunk of float16 queries at the end of the context, "
-                    "causal, 3-bit Full, mma.sync float16 tiles"}
+                    "causal, 3-bit Full, tcgen05.mma kind::f16 with accumulators in tensor memory"}
 
 
 def run_isoq(args):

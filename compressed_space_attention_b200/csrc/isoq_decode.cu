@@ -294,7 +294,6 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
 #include "decode_i8.cuh"
 #include "decode_append.cuh"
 #include "prefill.cuh"
-#include "prefill_tc.cuh"
 
 // ---------------------------------------------------------------------------
 // Host launchers
