@@ -204,8 +204,9 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   constexpr int BQ = kTcRows / GP;
   constexpr int QBLK = kTcRows * 128, KBLK = kTcTok * 128;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char *smem = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // Aligned by an offset from the shared array itself (not through an
+  // integer cast), so the compiler keeps the shared address space.
+  unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char *q_hi = smem, *q_lo = smem + C::OFF_QLO;
   unsigned char *kv = smem + C::OFF_KV, *pt = smem + C::OFF_P;
   float *nk_s = reinterpret_cast<float *>(smem + C::OFF_NORM), *nv_s = nk_s + kTcTok;
