@@ -487,6 +487,61 @@ def measure_prefill(isoq, synth, torch, dev, stream, seed0, peak_tflops, reps=5)
                     "causal, 3-bit Full, tcgen05.mma kind::f16 with accumulators in tensor memory"}
 
 
+DECODE_SWEEP = [
+    # (name, B, Hq, Hkv, Tmax, d, ragged)
+    ("b1_gqa32_4_d128_t32768", 1, 32, 4, 32768, 128, False),
+    ("b16_gqa32_4_d128_t8192_ragged", 16, 32, 4, 8192, 128, True),
+] + [(f"b32_gqa16_8_d256_t{t}", 32, 16, 8, t, 256, False) for t in (1024, 2048, 4096, 8192, 16384, 32768)]
+
+
+def measure_decode_sweep(isoq, synth, torch, dev, seed0, hbm, reps=20):
+    """Decode attention (query preparation + split + combine) on the small
+    decode workloads and the long-context shape at shorter contexts: each
+    call captured once in a CUDA graph and replayed `reps` times between two
+    events, so host launch overhead does not enter the small cases."""
+    out = {}
+    for name, B, Hq, Hkv, T, d, ragged in DECODE_SWEEP:
+        bits, variant, pb = 3, isoq.ISOQ_FULL, d * 3 // 8
+        prk = torch.from_numpy(isoq.isoq_make_params(d, variant, 1, Hkv)).to(dev)
+        prv = torch.from_numpy(isoq.isoq_make_params(d, variant, 2, Hkv)).to(dev)
+        k, v = synth.student_t_kv_torch(B, Hkv, T, d, seed=seed0 + 61, device=dev)
+        pk, nk = isoq.isoq_quantize(k.view(-1, T, d), prk.repeat(B, 1, 1), bits, variant)
+        pv, nv = isoq.isoq_quantize(v.view(-1, T, d), prv.repeat(B, 1, 1), bits, variant)
+        del k, v
+        pk, pv, nk, nv = pk.view(B, Hkv, T, pb), pv.view(B, Hkv, T, pb), nk.view(B, Hkv, T), nv.view(B, Hkv, T)
+        q = synth.queries_torch(B, Hq, d, seed=seed0 + 62, device=dev)
+        lens_np = synth.ragged_lengths(B, T // 2, T, seed=0) if ragged else np.full(B, T, dtype=np.int32)
+        lens = torch.from_numpy(lens_np).to(dev)
+        o = torch.empty((B, Hq, d), dtype=torch.float16, device=dev)
+        ws = torch.empty(isoq.isoq_decode_workspace_size(B, Hq, Hkv, T, d), dtype=torch.uint8, device=dev)
+        call = lambda: isoq.isoq_decode_attention(q, pk, pv, nk, nv, lens, prk, prv, bits, variant,  # noqa: E731
+                                                  out=o, workspace=ws)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        assert isoq.isoq_check_device_error() == 0
+        us = e0.elapsed_time(e1) / reps * 1e3
+        kv_bytes = int(lens_np.clip(0, T).sum()) * Hkv * kv_bytes_per_token_head(d, bits)
+        gbps = kv_bytes / (us * 1e-6) / 1e9
+        out[name] = {"us": us, "gbps": gbps, "frac": gbps / hbm, "kv_bytes": kv_bytes}
+        del g, pk, pv, nk, nv, q, o, ws
+        torch.cuda.empty_cache()
+    return {"what": "isoq_decode_attention (prep + split + combine) replayed from a CUDA graph; KV GB/s on "
+                    "the packed bytes of the valid tokens", "by_workload": out}
+
+
 def run_isoq(args):
     import torch
 
@@ -665,6 +720,8 @@ def run_isoq(args):
     variants = measure_variants(isoq, synth, torch, dev, stream, x1, seed0) if not args.no_variants else None
     comparator = measure_rotor_comparison(isoq, torch, dev, stream) if not args.no_comparator else None
     peaks_all, _ = measured_peaks()
+    sweep = (measure_decode_sweep(isoq, synth, torch, dev, seed0, float(peaks_all.get("hbm_gbs", FALLBACK_HBM_GBS)))
+             if not args.no_sweep else None)
     prefill = (measure_prefill(isoq, synth, torch, dev, stream, seed0,
                                float(peaks_all.get("bf16_tflops", 1590.0))) if not args.no_prefill else None)
 
@@ -708,6 +765,7 @@ def run_isoq(args):
         "variants": variants,
         "rotorquant_comparison": comparator,
         "prefill": prefill,
+        "decode_sweep": sweep,
         "gpu_launches": 4 * args.steps,
         "clocks": sampler.summary(),
     }
@@ -733,6 +791,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle CPU baseline (profiling runs)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the decode measurements at small batch and shorter contexts")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the chunked-prefill attention measurement")
     ap.add_argument("--no-comparator", action="store_true",

@@ -240,6 +240,7 @@ __global__ void __launch_bounds__(kI8Threads) prep_i8_kernel(const SplitArgs a, 
   const int kvh = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.group;
+  pdl_launch_dependents();   // the split kernel may start its staging now
   for (int i = tid; i < GP * D; i += kI8Threads) {
     const int gq = i / D;
     float v = 0.f;
@@ -358,7 +359,11 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
   const int g = lane >> 2, t = lane & 3;
 
   // B fragments of the fixed-point query and the per-head score factors,
-  // prepared once per (b, kvh) by prep_i8_kernel.
+  // prepared once per (b, kvh) by prep_i8_kernel (launched just before this
+  // kernel with programmatic dependent launch: wait for it here, after the
+  // staging above has started).
+  pdl_launch_dependents();
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t *qp = a.ws_qprep + pair * C::QPREP_WORDS;
   uint32_t qb[C::NQ][C::KK][2];
 #pragma unroll
@@ -811,8 +816,8 @@ int launch_split_i8(const SplitArgs &a, cudaStream_t stream) {
   dim3 grid(a.n_splits, a.hkv, a.batch);
   static_assert(C::QPREP_WORDS == decode_qprep_words(D), "prepared-query layout");
   prep_i8_kernel<D, FULL, GP><<<dim3(a.hkv, a.batch), kI8Threads, 0, stream>>>(a, score_unit);
-  kernel<<<grid, kI8Threads, C::SMEM, stream>>>(a, tb.lut, out_scale);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kernel, grid, dim3(kI8Threads), C::SMEM, stream, a, tb.lut, out_scale);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode i8 launch: %s", cudaGetErrorString(e));
   return ISOQ_OK;
 }

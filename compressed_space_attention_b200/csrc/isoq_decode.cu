@@ -38,6 +38,29 @@ using namespace isoq::dev;
 
 __device__ unsigned int g_decode_error = 0;
 
+// Launch with programmatic dependent launch: the kernel may start while the
+// previous kernel on the stream is still running (once that kernel's CTAs
+// have all started or signalled), and must execute griddepcontrol.wait
+// before reading anything the previous kernel writes.  Used only for
+// kernels whose predecessor is one of ours (prep -> split -> combine).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Barrier over the threads taking part in a shared-memory rotation: the whole
 // CTA (bar_id 0 -> __syncthreads) or a named barrier over `nthreads` threads.
 __device__ __forceinline__ void rotation_sync(int bar_id, int nthreads) {
@@ -232,17 +255,28 @@ __global__ void __launch_bounds__(kGenericThreads) split_generic_kernel(const Sp
 // ---------------------------------------------------------------------------
 // Combine + inverse rotation.
 // ---------------------------------------------------------------------------
-constexpr int kCombineThreads = 128;
+constexpr int kCombineThreads = 256;
+constexpr int kCombineWBlock = 1024;    // split weights held in shared memory per pass
 
+// One CTA per (b, qh).  The split weights w_s = exp(m_s - m*) are computed
+// once per split (not once per split and dimension) into shared memory; the
+// threads then sum acc_s[i] w_s with kCombineThreads / D threads per
+// dimension, each over every (kCombineThreads / D)-th split.
 template <typename T, int D, bool FULL>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineArgs a) {
+  constexpr int P = D >= kCombineThreads ? 1 : kCombineThreads / D;   // threads per dimension
+  constexpr int DPT = D > kCombineThreads ? D / kCombineThreads : 1;  // dimensions per thread
   __shared__ float v[D];
+  __shared__ float part[P > 1 ? P : 1][D];
+  __shared__ float wsh[kCombineWBlock];
   __shared__ float red[kCombineThreads / 32];
   __shared__ float s_mstar, s_l;
   const int qh = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kvh = qh / a.group;
   const long long base = (static_cast<long long>(b) * a.hq + qh) * a.n_splits;
+  // The partial states come from the split kernel launched just before.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   float mx = -INFINITY;
   for (int s = tid; s < a.n_splits; s += kCombineThreads) mx = fmaxf(mx, a.ws_ml[base + s].x);
@@ -257,15 +291,37 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
   }
   __syncthreads();
   const float mstar = s_mstar;
+
+  const int p = tid / (D < kCombineThreads ? D : kCombineThreads);
+  const int i0 = tid % (D < kCombineThreads ? D : kCombineThreads);
+  float acc[DPT];
+#pragma unroll
+  for (int k = 0; k < DPT; ++k) acc[k] = 0.f;
   float lsum = 0.f;
-  for (int s = tid; s < a.n_splits; s += kCombineThreads) {
-    const float2 ml = a.ws_ml[base + s];
-    if (ml.y > 0.f) lsum += ml.y * expf(ml.x - mstar);
+  for (int s0 = 0; s0 < a.n_splits; s0 += kCombineWBlock) {
+    const int ns = a.n_splits - s0 < kCombineWBlock ? a.n_splits - s0 : kCombineWBlock;
+    __syncthreads();   // the previous pass no longer reads wsh
+    for (int s = tid; s < ns; s += kCombineThreads) {
+      const float2 ml = a.ws_ml[base + s0 + s];
+      const float w = ml.y > 0.f ? expf(ml.x - mstar) : 0.f;
+      wsh[s] = w;
+      lsum += ml.y * w;
+    }
+    __syncthreads();
+    const float *accp = a.ws_acc + (base + s0) * D;
+#pragma unroll 4
+    for (int s = p; s < ns; s += P) {
+      const float w = wsh[s];
+#pragma unroll
+      for (int k = 0; k < DPT; ++k) acc[k] = fmaf(accp[static_cast<long long>(s) * D + i0 + k * kCombineThreads], w, acc[k]);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  __syncthreads();
   if (lane == 0) red[warp] = lsum;
+  if (P > 1) {
+    part[p][i0] = acc[0];
+  }
   __syncthreads();
   if (tid == 0) {
     float l = 0.f;
@@ -273,16 +329,17 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
     s_l = l;
   }
   __syncthreads();
-  const float ltot = s_l;
-  const float inv_l = ltot > 0.f ? 1.f / ltot : 0.f;
-
-  for (int i = tid; i < D; i += kCombineThreads) {
-    float acc = 0.f;
-    for (int s = 0; s < a.n_splits; ++s) {
-      const float2 ml = a.ws_ml[base + s];
-      if (ml.y > 0.f) acc = fmaf(a.ws_acc[(base + s) * D + i], expf(ml.x - mstar), acc);
+  const float inv_l = s_l > 0.f ? 1.f / s_l : 0.f;
+  if (P > 1) {
+    for (int i = tid; i < D; i += kCombineThreads) {
+      float t = 0.f;
+#pragma unroll
+      for (int q = 0; q < P; ++q) t += part[q][i];
+      v[i] = t * inv_l;
     }
-    v[i] = acc * inv_l;
+  } else {
+#pragma unroll
+    for (int k = 0; k < DPT; ++k) v[i0 + k * kCombineThreads] = acc[k] * inv_l;
   }
   __syncthreads();
   rotate_inverse_cta<D, FULL>(v, a.params_v + static_cast<size_t>(kvh) * 2 * D);
@@ -317,8 +374,8 @@ int launch_split_generic(const SplitArgs &a, cudaStream_t stream) {
 template <typename T, int D, bool FULL>
 int launch_combine(const CombineArgs &a, cudaStream_t stream) {
   dim3 grid(a.hq, a.batch);
-  combine_kernel<T, D, FULL><<<grid, kCombineThreads, 0, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(combine_kernel<T, D, FULL>, grid, dim3(kCombineThreads), 0, stream, a);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode combine launch: %s", cudaGetErrorString(e));
   return ISOQ_OK;
 }

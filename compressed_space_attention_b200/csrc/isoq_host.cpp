@@ -167,14 +167,16 @@ bool codebook_unit_f64(int bits, double *centroids) {
 
 // Each split covers a fixed number of tokens (a multiple of 64) chosen so
 // that B * Hkv * n_splits is about 8 CTAs per SM of a 148-SM B200, with
-// chunks between 256 and 4096 tokens.
+// chunks between 512 and 4096 tokens (below 512 tokens a split's fixed
+// costs, its set-up and its share of the combine, outweigh the parallelism
+// it adds: measured on a batch-1, 32K-token decode, 42 -> 33 us).
 int64_t decode_chunk_tokens(int B, int Hkv, int64_t Tmax, int d) {
   (void)d;
   const int64_t target_ctas = 148 * 8;
   int64_t work = static_cast<int64_t>(B) * Hkv * Tmax;
   int64_t chunk = (work + target_ctas - 1) / target_ctas;
   chunk = (chunk + kDecodeTokenQuantum - 1) / kDecodeTokenQuantum * kDecodeTokenQuantum;
-  if (chunk < 256) chunk = 256;
+  if (chunk < 512) chunk = 512;
   if (chunk > 4096) chunk = 4096;
   return chunk;
 }
