@@ -17,9 +17,12 @@ extern "C" int isoq_check_device_error(isoq_stream_t stream) {
   st = isoq_detail_take_decode_error(s, &d);
   if (st) return st;
   // Bit 1: a bounded wait gave up.  Bit 2: a decode append found a full row.
+  // Bit 4: the prefill kernel found its shared memory misaligned.
   if ((q | d) & 1u)
     return isoq::set_error(ISOQ_ERR_TIMEOUT, "device wait timed out (quantize=%u, decode=%u)", q, d);
   if (d & 2u)
     return isoq::set_error(ISOQ_ERR_INVALID_ARG, "decode append: a row already held Tmax tokens");
+  if (d & 4u)
+    return isoq::set_error(ISOQ_ERR_CUDA, "prefill: dynamic shared memory not 1024-byte aligned");
   return ISOQ_OK;
 }

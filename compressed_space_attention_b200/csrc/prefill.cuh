@@ -11,33 +11,42 @@
 // softmax, V accumulated as centroids, one inverse rotation per output row.
 //
 // CTA = 128 query-head rows (128 / GP positions x GP heads; heads >= G are
-// dead rows), one TMEM lane each, 4 warps; thread r owns row r for the
-// softmax (TMEM lane r lies in its warp's sub-partition).  Per 64-token tile:
-//   thread 0 has staged the tile's packed codes and norms with bulk copies
-//   (2-deep ring); the CTA expands the K codes into float16 centroids
-//   alpha c_k (alpha, searched on the host, makes them nearly exact in
-//   float16) in a 128B-swizzled tile; one thread issues
-//   S = Q~hi K~^T + Q~lo K~^T with tcgen05.mma kind::f16 (M = 128, N = 64;
-//   q~ split into float16 hi and lo parts keeps 22-bit scores) into TMEM;
-//   after the commit's mbarrier the V codes are expanded into the same tile
-//   buffer while each thread reads its S row (tcgen05.ld), scales it by
-//   s^K scale / alpha, masks it on diagonal tiles, updates its running
-//   maximum and sum, rescales its O row in TMEM when its warp's maximum
-//   moved, and writes p s^V as float16 (11 bits of each weight's own
-//   magnitude) into a K-major P tile; one thread issues O += P V~ (N = d, V~
-//   read MN-major from the same token-row tile).
+// dead rows), one TMEM lane each, 8 warps: warps w and w + 4 share TMEM
+// sub-partition w (lanes 32 w .. + 31) and split each row's S and O columns
+// in halves.  Per 64-token tile j, software-pipelined by one product:
+//   the packed codes and norms of the next tiles are loaded into registers
+//   one phase ahead; the CTA expands K tile j + 1's codes into float16
+//   centroids alpha c_k (alpha, searched on the host, makes them nearly
+//   exact in float16) in a 128B-swizzled tile, and one thread issues
+//   S(j + 1) = Q~hi K~^T + Q~lo K~^T (tcgen05.mma kind::f16, M = 128,
+//   N = 64; q~ split into float16 hi and lo parts keeps 22-bit scores) into
+//   the other of two TMEM S buffers, so it runs under the softmax of tile j;
+//   each thread reads its half row of S(j) (tcgen05.ld), scales it by
+//   s^K scale / alpha, masks it on diagonal tiles, exchanges its half-row
+//   maximum with the partner warp, writes p s^V as float16 (11 bits of each
+//   weight's own magnitude) into a K-major P tile and, when its warp's
+//   maximum moved, rescales its half of the O row in TMEM; the CTA expands
+//   V tile j into its own tile buffer and one thread issues O += P V~
+//   (N = d, V~ read MN-major from the token-row tile).
+// d = 128 keeps one P tile and fits two CTAs per SM (one CTA's thread work
+// runs under the other's products); d = 256 keeps two P tiles, one CTA.
 // The epilogue reads O from TMEM, normalises, rotates back (R_V^T) in shared
 // memory and stores float16.
 // Operand tiles use the canonical SW128 layouts: rows of 128 bytes (64
 // float16), 16-byte chunks XOR-swizzled by (row % 8), 8-row groups 1024
 // bytes apart, 64-element blocks of the row direction `blk_stride` apart.
 // Every wait is bounded; on a timeout the CTA records kErrWaitTimeout, waits
-// (bounded) for its outstanding copies and products, frees its tensor memory
-// and returns.
+// (bounded) for its outstanding products, frees its tensor memory and
+// returns.
 //
 // Requires float16 queries (float16 tiles meet the float16 output tolerance,
 // not the float32 one), 3-bit codes, d in {128, 256}, G = Hq / Hkv in
 // {1, 2, 4, 8}, Tmax % 8 == 0 and 16-byte aligned code rows.
+
+// The prefill kernel found its dynamic shared memory off a 1024-byte
+// boundary (its two-CTAs-per-SM layout keeps no slack to align it) and
+// returned without writing its output.
+constexpr unsigned kErrSmemAlign = 4u;
 
 struct PrefillArgs {
   const void *q;                  // [B][Tq][Hq][d]
@@ -87,31 +96,39 @@ __device__ void rotate_inverse_rows(float *v, int nvec, const float *params_head
   }
 }
 
-constexpr int kTcThreads = 128;
+constexpr int kTcThreads = 256;   // 8 warps: two per TMEM sub-partition, one per column half
 constexpr int kTcRows = 128;      // M: query-head rows per CTA
 constexpr int kTcTok = 64;        // N of QK, K of PV
-constexpr int kTcStages = 2;
 
 template <int D>
 struct TcCfg {
   static constexpr int PB = D * 3 / 8;
+  static constexpr int ITEMS = kTcTok * (D / 32) / kTcThreads;   // 32-code groups per thread per tile
   static constexpr int Q_BYTES = kTcRows * D * 2;         // one of hi / lo
-  static constexpr int KV_BYTES = kTcTok * D * 2;         // one tile buffer (K, then V)
-  static constexpr int P_BYTES = kTcRows * kTcTok * 2;
-  static constexpr int ST_CODES = kTcTok * PB;
-  static constexpr int ST_BYTES = 2 * ST_CODES + 2 * kTcTok * 2;
-  static constexpr int NORM_BYTES = 2 * kTcTok * 4;
+  static constexpr int KV_BYTES = kTcTok * D * 2;         // one K or V tile
+  static constexpr int P_BYTES = kTcRows * kTcTok * 2;    // one P tile
+  // d = 256: two P tiles, so PV(j - 1) (twice the work of d = 128's) runs on
+  // under the softmax of tile j; d = 128 has one, waits for PV(j - 1) before
+  // writing P(j) and fits two CTAs per SM instead.
+  static constexpr int P_BUFS = D == 128 ? 1 : 2;
+  static constexpr int NORM_BYTES = 2 * kTcTok * 4;       // s^K score_unit, s^V of one tile
   static constexpr int OFF_QLO = Q_BYTES;
-  static constexpr int OFF_KV = 2 * Q_BYTES;
-  static constexpr int OFF_P = OFF_KV + KV_BYTES;
-  static constexpr int OFF_NORM = OFF_P + P_BYTES;
-  static constexpr int OFF_STAGE = OFF_NORM + NORM_BYTES;
-  static constexpr int OFF_BAR = OFF_STAGE + kTcStages * ST_BYTES;
-  static constexpr int SMEM = OFF_BAR + 8 * (kTcStages + 2) + 16 + 1024;
-  static constexpr int TMEM_COLS = D == 128 ? 256 : 512;     // S (64) + O (D), rounded to a power of 2
+  static constexpr int OFF_K = 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_P = OFF_V + KV_BYTES;
+  static constexpr int OFF_NORM = OFF_P + P_BUFS * P_BYTES;
+  static constexpr int OFF_BAR = OFF_NORM + NORM_BYTES;
+  // Two CTAs per SM at d = 128 (the second CTA's softmax and expansion run
+  // under the first one's products).  Their layout leaves no room to align
+  // the dynamic shared memory by hand: the kernel checks that it starts on a
+  // 1024-byte boundary and reports kErrSmemAlign otherwise.
   static constexpr int MIN_BLOCKS = D == 128 ? 2 : 1;
-  static_assert(32 * D * 4 <= KV_BYTES + P_BYTES, "prep scratch (32 rows) fits the K/V and P buffers");
-  static_assert(SMEM <= 232448, "shared memory");
+  static constexpr int SLACK = MIN_BLOCKS == 2 ? 0 : 1024;
+  static constexpr int SMEM = OFF_BAR + 8 * 3 + 8 + SLACK;
+  static constexpr int TMEM_COLS = D == 128 ? 256 : 512;     // S (2 x 64) + O (D), rounded to a power of 2
+  static_assert(32 * D * 4 <= 2 * KV_BYTES, "prep scratch (32 rows) fits the K and V tiles");
+  static_assert(MIN_BLOCKS * (SMEM + 1024) <= 233472, "shared memory per SM (1 KB reserved per CTA)");
+  static_assert(MIN_BLOCKS * TMEM_COLS <= 512, "tensor memory columns");
 };
 
 __host__ __device__ __forceinline__ uint32_t tc_off(int r, int e, int blk_stride) {
@@ -170,30 +187,55 @@ __device__ __forceinline__ void tc_st16(uint32_t taddr, const float (&v)[16]) {
       : "memory");
 }
 
-// Staged codes of a tile's tokens (zeros from token nvalid on) -> float16
-// centroids in the SW128 token-row layout (64-dim blocks KV_BYTES / (D/64)
-// apart); the same layout serves K (K-major B of QK) and V (MN-major B of PV).
+// Packed codes of one tile, this thread's share (ITEMS 32-code groups),
+// loaded from global memory one phase before they are expanded.
 template <int D>
-__device__ __forceinline__ void tc_expand(const unsigned char *codes, int nvalid, unsigned char *tile,
-                                          const PrefillArgs &a, int tid) {
-  constexpr int GROUPS = D / 32, PB = D * 3 / 8, BLK = kTcTok * 128;
-  for (int idx = tid; idx < kTcTok * GROUPS; idx += kTcThreads) {
-    const int tok = idx / GROUPS, grp = idx - tok * GROUPS;
-    uint32_t w0 = 0, w1 = 0, w2 = 0;
-    if (tok < nvalid) {
-      const unsigned char *src = codes + tok * PB + 12 * grp;
-      w0 = lds32(src);
-      w1 = lds32(src + 4);
-      w2 = lds32(src + 8);
-    }
-    uint32_t s[8];
-    group_sel8(w0, w1, w2, s);
+struct TcCodes {
+  uint32_t w[TcCfg<D>::ITEMS][3];
+};
+
+template <int D>
+__device__ __forceinline__ void tc_fetch(TcCodes<D> &c, const uint8_t *base, int t0, int tend, int tid) {
+  constexpr int GROUPS = D / 32, PB = D * 3 / 8;
 #pragma unroll
-    for (int qd = 0; qd < 8; ++qd) {
-      const uint32_t lo = prmt(a.lut_lo0, a.lut_lo1, s[qd]);
-      const uint32_t hi = prmt(a.lut_hi0, a.lut_hi1, s[qd]);
-      const uint2 v = make_uint2(prmt(lo, hi, 0x5140u), prmt(lo, hi, 0x7362u));
-      *reinterpret_cast<uint2 *>(tile + tc_off(tok, 32 * grp + 4 * qd, BLK)) = v;   // dims 32 grp + 4 qd .. + 3
+  for (int k = 0; k < TcCfg<D>::ITEMS; ++k) {
+    const int idx = tid + k * kTcThreads, tok = idx / GROUPS, grp = idx % GROUPS;
+    if (t0 + tok < tend) {
+      const uint32_t *src = reinterpret_cast<const uint32_t *>(base + static_cast<long long>(t0 + tok) * PB + 12 * grp);
+      c.w[k][0] = __ldg(src);
+      c.w[k][1] = __ldg(src + 1);
+      c.w[k][2] = __ldg(src + 2);
+    } else {
+      c.w[k][0] = c.w[k][1] = c.w[k][2] = 0u;
+    }
+  }
+}
+
+// Fetched codes -> float16 centroids alpha c_k in the SW128 token-row tile
+// (64-dim blocks kTcTok * 128 bytes apart); the same layout serves K (K-major
+// B of QK) and V (MN-major B of PV).
+template <int D>
+__device__ __forceinline__ void tc_expand(const TcCodes<D> &c, unsigned char *tile, const PrefillArgs &a, int tid) {
+  constexpr int GROUPS = D / 32, BLK = kTcTok * 128;
+#pragma unroll
+  for (int k = 0; k < TcCfg<D>::ITEMS; ++k) {
+    const int idx = tid + k * kTcThreads, tok = idx / GROUPS, grp = idx % GROUPS;
+    uint32_t s[8];
+    group_sel8(c.w[k][0], c.w[k][1], c.w[k][2], s);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      uint32_t v[4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint32_t lo = prmt(a.lut_lo0, a.lut_lo1, s[2 * m + u]);
+        const uint32_t hi = prmt(a.lut_hi0, a.lut_hi1, s[2 * m + u]);
+        v[2 * u] = prmt(lo, hi, 0x5140u);
+        v[2 * u + 1] = prmt(lo, hi, 0x7362u);
+      }
+      // dims 32 grp + 8 m .. + 7, as two 8-byte stores (measured faster
+      // here than one 16-byte store, despite the latter's fewer bank conflicts)
+      *reinterpret_cast<uint2 *>(tile + tc_off(tok, 32 * grp + 8 * m, BLK)) = make_uint2(v[0], v[1]);
+      *reinterpret_cast<uint2 *>(tile + tc_off(tok, 32 * grp + 8 * m + 4, BLK)) = make_uint2(v[2], v[3]);
     }
   }
 }
@@ -206,15 +248,19 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   extern __shared__ unsigned char smem_raw[];
   // Aligned by an offset from the shared array itself (not through an
   // integer cast), so the compiler keeps the shared address space.
-  unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (pad > static_cast<uint32_t>(C::SLACK)) {   // uniform over the grid: nothing allocated yet
+    if (threadIdx.x == 0) atomicOr(&g_decode_error, kErrSmemAlign);
+    return;
+  }
+  unsigned char *smem = smem_raw + pad;
   unsigned char *q_hi = smem, *q_lo = smem + C::OFF_QLO;
-  unsigned char *kv = smem + C::OFF_KV, *pt = smem + C::OFF_P;
-  float *nk_s = reinterpret_cast<float *>(smem + C::OFF_NORM), *nv_s = nk_s + kTcTok;
-  unsigned char *stage = smem + C::OFF_STAGE;
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-  uint64_t *bar_s = full_bar + kTcStages, *bar_o = bar_s + 1;
+  unsigned char *kt = smem + C::OFF_K, *vt = smem + C::OFF_V, *pt = smem + C::OFF_P;
+  float *nrm_s = reinterpret_cast<float *>(smem + C::OFF_NORM);   // [2][kTcTok] s^K score_unit, s^V of the tile in the softmax
+  uint64_t *bar_s = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);   // [2]: S buffer b's product done
+  uint64_t *bar_o = bar_s + 2;                                          // PV product done
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_o + 1);
-  float *scratch = reinterpret_cast<float *>(kv);   // 32 rows x D floats over the K/V and P buffers
+  float *scratch = reinterpret_cast<float *>(kt);   // 32 rows x D floats over the K and V tiles (prep, epilogue)
 
   const int qt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -237,19 +283,21 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   const uint16_t *nkb = a.norms_k + pair * a.tmax;
   const uint16_t *nvb = a.norms_v + pair * a.tmax;
 
-  auto issue = [&](int i) {
-    const int t0 = i * kTcTok;
-    int n = tend - t0;
-    n = n > kTcTok ? kTcTok : n;
-    const int n8 = (n + 7) & ~7;
-    unsigned char *st = stage + (i % kTcStages) * C::ST_BYTES;
-    uint64_t *bar = &full_bar[i % kTcStages];
-    mbar_arrive_expect_tx(bar, 2u * n * C::PB + 4u * n8);
-    bulk_load(st, kb + static_cast<long long>(t0) * C::PB, n * C::PB, bar);
-    bulk_load(st + C::ST_CODES, vb + static_cast<long long>(t0) * C::PB, n * C::PB, bar);
-    bulk_load(st + 2 * C::ST_CODES, nkb + t0, 2 * n8, bar);
-    bulk_load(st + 2 * C::ST_CODES + 2 * kTcTok, nvb + t0, 2 * n8, bar);
+  // Codes and norms of upcoming tiles, one phase ahead, in registers:
+  // kc = the next K tile to expand, vc = the next V tile, nrm = the norm
+  // (K for tid < 64, V for tid < 128) of the next tile to enter the softmax.
+  TcCodes<D> kc, vc;
+  uint16_t nrm = 0;
+  auto fetch_norm = [&](int j) {
+    const int t0 = j * kTcTok, tok = tid & (kTcTok - 1);
+    nrm = (tid < 2 * kTcTok && t0 + tok < tend) ? __ldg(((tid < kTcTok) ? nkb : nvb) + t0 + tok)
+                                                : static_cast<uint16_t>(0);
   };
+  if (n_tiles > 0) {
+    tc_fetch<D>(kc, kb, 0, tend, tid);
+    tc_fetch<D>(vc, vb, 0, tend, tid);
+    fetch_norm(0);
+  }
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -257,11 +305,10 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    for (int k = 0; k < kTcStages; ++k) mbar_init(&full_bar[k], 1);
-    mbar_init(bar_s, 1);
+    mbar_init(&bar_s[0], 1);
+    mbar_init(&bar_s[1], 1);
     mbar_init(bar_o, 1);
     mbar_fence_init();
-    if (n_tiles > 0) issue(0);
   }
 
   // ---- prep, 32 rows per pass: rotate, split into float16 hi / lo (SW128 K-major) ----
@@ -299,126 +346,180 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_s = tmem, t_o = tmem + 64;                 // S columns [0, 64), O columns [64, 64 + D)
-  const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+  const uint32_t t_o = tmem + 128;                           // S buffers at columns [0, 64), [64, 128); O after
+  // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (its sub-partition) and
+  // handles column half w / 4 of those rows' S and O.
+  const int sub = warp & 3, half = warp >> 2, lane = tid & 31;
+  const uint32_t lane_off = static_cast<uint32_t>(32 * sub) << 16;
+  const uint32_t qh_s = smem_u32(q_hi), ql_s = smem_u32(q_lo), k_s = smem_u32(kt), v_s = smem_u32(vt),
+                 p_s = smem_u32(pt);
 
-  const int r = tid;                                          // this thread's row / TMEM lane
-  const int pr = p_first + r / GP;
-  const int pw_min = p_first + (32 * warp) / GP;
-  float mx = -INFINITY, l = 0.f;
-  const uint32_t qh_s = smem_u32(q_hi), ql_s = smem_u32(q_lo), kv_s = smem_u32(kv), p_s = smem_u32(pt);
-
-  bool failed = false;
-  int consumed = 0, s_done = 0, o_done = 0, o_issued = 0;
-  for (int it = 0; it < n_tiles; ++it) {
-    const int t0 = it * kTcTok;
-    // Staged codes of this tile, and the previous PV product (it reads the
-    // tile buffer and P) must be complete.
-    bool ok = mbar_wait_bounded(&full_bar[it % kTcStages], (it / kTcStages) & 1);
-    if (ok && o_issued > o_done) {
-      ok = mbar_wait_bounded(bar_o, o_done & 1);
-      if (ok) ++o_done;
-    }
-    if (__syncthreads_or(!ok)) {
-      failed = true;
-      break;
-    }
-    tc_fence_after();
-    consumed = it + 1;
-    if (tid == 0 && it + 1 < n_tiles) {
-      fence_proxy_async_smem();
-      issue(it + 1);
-    }
-    const unsigned char *st = stage + (it % kTcStages) * C::ST_BYTES;
-    const int nvalid = tend - t0 < kTcTok ? tend - t0 : kTcTok;
-    tc_expand<D>(st, nvalid, kv, a, tid);
-    if (tid < kTcTok) {
-      const bool in = tid < nvalid;
-      const unsigned char *nks = st + 2 * C::ST_CODES, *nvs = nks + 2 * kTcTok;
-      nk_s[tid] = in ? lds_half(nks + 2 * tid) * a.score_unit : 0.f;
-      nv_s[tid] = in ? lds_half(nvs + 2 * tid) : 0.f;
-    }
+  // Expands K tile j (codes and norms from the registers), then issues its QK
+  // product into S buffer j % 2.  The caller has made sure the K tile and
+  // that S buffer are free.
+  auto store_norm = [&]() {
+    if (tid < 2 * kTcTok) nrm_s[tid] = __half2float(__ushort_as_half(nrm)) * (tid < kTcTok ? a.score_unit : 1.f);
+  };
+  auto stage_qk = [&](int j) {
+    tc_expand<D>(kc, kt, a, tid);
+    if (j + 1 < n_tiles) tc_fetch<D>(kc, kb, (j + 1) * kTcTok, tend, tid);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (tid == 0) {
       constexpr uint32_t idesc = tc_idesc(kTcRows, kTcTok, 0);
+      const uint32_t t_s = tmem + (j & 1) * 64;
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t ko = (ks >> 2) * KBLK + (ks & 3) * 32, qo = (ks >> 2) * QBLK + (ks & 3) * 32;
-        const uint64_t bd = tc_desc(kv_s + ko, 16, 1024);
+        const uint64_t bd = tc_desc(k_s + ko, 16, 1024);
         tc_mma(t_s, tc_desc(qh_s + qo, 16, 1024), bd, idesc, ks > 0 ? 1u : 0u);
         tc_mma(t_s, tc_desc(ql_s + qo, 16, 1024), bd, idesc, 1u);
       }
-      tc_commit(bar_s);
+      tc_commit(&bar_s[j & 1]);
     }
-    ok = mbar_wait_bounded(bar_s, s_done & 1);
+  };
+
+  const int r = 32 * sub + lane;                              // this thread's row / TMEM lane
+  const int pr = p_first + r / GP;
+  const int pw_min = p_first + (32 * sub) / GP;
+  constexpr int HC = kTcTok / 2;                               // score columns per thread
+  constexpr int OH = D / 2;                                    // output columns per thread
+  float mx = -INFINITY;
+  uint64_t l2 = f2_pack(0.f, 0.f);                             // running row sum, two partial lanes
+  bool failed = false;
+  int qk_issued = 0, qk_done = 0, o_issued = 0, o_done = 0;
+
+  if (n_tiles > 0) {
+    store_norm();
+    if (n_tiles > 1) fetch_norm(1);
+    stage_qk(0);
+    ++qk_issued;
+  }
+  for (int it = 0; it < n_tiles; ++it) {
+    const int t0 = it * kTcTok;
+    // QK(it) must be complete: its S buffer is read below and the K tile is free.
+    bool ok = mbar_wait_bounded(&bar_s[it & 1], (it >> 1) & 1);
     if (__syncthreads_or(!ok)) {
       failed = true;
       break;
     }
-    ++s_done;
+    ++qk_done;
     tc_fence_after();
-
-    // V codes into the tile buffer (the QK product no longer reads it).
-    tc_expand<D>(st + C::ST_CODES, nvalid, kv, a, tid);
-
-    // ---- softmax on this thread's row ----
-    float x[64];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float v[16];
-      tc_ld16(t_s + lane_off + 16 * c, v);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) x[16 * c + j] = v[j] * nk_s[16 * c + j];
+    // The next tile's QK runs on the tensor cores under this tile's softmax.
+    if (it + 1 < n_tiles) {
+      stage_qk(it + 1);
+      ++qk_issued;
     }
-    if (t0 + kTcTok - 1 > pw_min || t0 + kTcTok > tend) {   // warp-uniform
+
+    // ---- softmax on this thread's half row of S(it) ----
+    // Arithmetic on float pairs (f32x2: one instruction per two columns);
+    // the norms are read as 16-byte broadcasts.
+    const ulonglong2 *nk4 = reinterpret_cast<const ulonglong2 *>(nrm_s + HC * half);
+    const ulonglong2 *nv4 = reinterpret_cast<const ulonglong2 *>(nrm_s + kTcTok + HC * half);
+    const int c0 = t0 + HC * half;                             // token of this thread's first column
+    float x[HC];
 #pragma unroll
-      for (int j = 0; j < 64; ++j)
-        if (t0 + j > pr || t0 + j >= tend) x[j] = -INFINITY;
+    for (int c = 0; c < HC / 16; ++c) {
+      float v[16];
+      tc_ld16(tmem + (it & 1) * 64 + HC * half + lane_off + 16 * c, v);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const ulonglong2 n = nk4[4 * c + k];
+        f2_unpack(f2_mul(f2_pack(v[4 * k], v[4 * k + 1]), n.x), x[16 * c + 4 * k], x[16 * c + 4 * k + 1]);
+        f2_unpack(f2_mul(f2_pack(v[4 * k + 2], v[4 * k + 3]), n.y), x[16 * c + 4 * k + 2], x[16 * c + 4 * k + 3]);
+      }
+    }
+    if (t0 + kTcTok - 1 > pw_min || t0 + kTcTok > tend) {   // uniform over the warp pair
+#pragma unroll
+      for (int j = 0; j < HC; ++j)
+        if (c0 + j > pr || c0 + j >= tend) x[j] = -INFINITY;
     }
     float tmx = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) tmx = fmaxf(tmx, x[j]);
+    for (int j = 0; j < HC; ++j) tmx = fmaxf(tmx, x[j]);
+
+    // PV(it - 1) must be complete before O is rescaled and the V tile
+    // reused; with one P tile, already before P(it) is written.
+    auto wait_pv = [&]() -> bool {
+      if (o_issued > o_done) {
+        const bool done = mbar_wait_bounded(bar_o, o_done & 1);
+        if (__syncthreads_or(!done)) return false;
+        ++o_done;
+        tc_fence_after();
+      }
+      return true;
+    };
+    if (C::P_BUFS == 1 && !wait_pv()) {
+      failed = true;
+      break;
+    }
+    unsigned char *pb = pt + (it % C::P_BUFS) * C::P_BYTES;   // free: PV(it - P_BUFS) is complete
+    // The row maximum over both column halves, exchanged with the partner
+    // warp through the free P tile: each thread leaves its value in the
+    // partner's part of row r and reads the partner's from its own part,
+    // which only it overwrites afterwards.
+    *reinterpret_cast<float *>(pb + tc_off(r, HC * (half ^ 1), 0)) = tmx;
+    named_barrier(1 + sub, 64);
+    tmx = fmaxf(tmx, *reinterpret_cast<const float *>(pb + tc_off(r, HC * half, 0)));
     const float nm = fmaxf(mx, tmx);
     const float base = nm == -INFINITY ? 0.f : nm;
     const float f = ex2f(mx - base);                            // 0 while mx = -inf
-    if (__any_sync(0xffffffffu, nm > mx) && it > 0) {
-      // rescale this warp's O rows in tensor memory (the last PV product is complete)
-#pragma unroll 1
-      for (int c = 0; c < D / 16; ++c) {
-        float v[16];
-        tc_ld16(t_o + lane_off + 16 * c, v);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] *= f;
-        tc_st16(t_o + lane_off + 16 * c, v);
-      }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-    }
+    const bool moved = __any_sync(0xffffffffu, nm > mx);       // the same in both warps of the pair
     mx = nm;
-    l *= f;
+    const uint64_t base2 = f2_pack(base, base);
+    l2 = f2_mul(l2, f2_pack(f, f));
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < HC / 8; ++c) {
       uint32_t w[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int j = 8 * c + 2 * k;
-        const float p0 = ex2f(x[j] - base), p1 = ex2f(x[j + 1] - base);
-        l += p0 + p1;
-        w[k] = pack_f16x2(p0 * nv_s[j], p1 * nv_s[j + 1]);
+        float p0, p1;
+        f2_unpack(f2_sub(f2_pack(x[j], x[j + 1]), base2), p0, p1);
+        const uint64_t p2 = f2_pack(ex2f(p0), ex2f(p1));
+        l2 = f2_add(l2, p2);
+        const ulonglong2 n = nv4[j >> 2];
+        f2_unpack(f2_mul(p2, (k & 1) ? n.y : n.x), p0, p1);
+        w[k] = pack_f16x2(p0, p1);
       }
-      *reinterpret_cast<uint4 *>(pt + tc_off(r, 8 * c, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4 *>(pb + tc_off(r, HC * half + 8 * c, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
+    if (C::P_BUFS == 2 && !wait_pv()) {
+      failed = true;
+      break;
+    }
+
+    if (moved && it > 0) {
+#pragma unroll 1
+      for (int c = 0; c < OH / 16; ++c) {
+        float v[16];
+        tc_ld16(t_o + OH * half + lane_off + 16 * c, v);
+        const uint64_t f2 = f2_pack(f, f);
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), f2), v[j], v[j + 1]);
+        tc_st16(t_o + OH * half + lane_off + 16 * c, v);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    tc_expand<D>(vc, vt, a, tid);
+    if (it + 1 < n_tiles) tc_fetch<D>(vc, vb, (it + 1) * kTcTok, tend, tid);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Every thread is past the softmax of tile it: its norms can be replaced.
+    if (it + 1 < n_tiles) {
+      store_norm();
+      if (it + 2 < n_tiles) fetch_norm(it + 2);
+    }
     if (tid == 0) {
       constexpr uint32_t idesc = tc_idesc(kTcRows, D, 1);
+      const uint32_t pbs = p_s + (it % C::P_BUFS) * C::P_BYTES;
 #pragma unroll
       for (int ks = 0; ks < kTcTok / 16; ++ks)
-        tc_mma(t_o, tc_desc(p_s + ks * 32, 16, 1024), tc_desc(kv_s + ks * 2048, KBLK, 1024), idesc,
+        tc_mma(t_o, tc_desc(pbs + ks * 32, 16, 1024), tc_desc(v_s + ks * 2048, KBLK, 1024), idesc,
                (it > 0 || ks > 0) ? 1u : 0u);
       tc_commit(bar_o);
     }
@@ -435,28 +536,36 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   if (failed) {
     if (tid == 0) {
       atomicOr(&g_decode_error, kErrWaitTimeout);
-      for (int k = consumed; k < n_tiles && k < consumed + kTcStages; ++k)
-        if (!mbar_wait_bounded(&full_bar[k % kTcStages], (k / kTcStages) & 1)) break;
+      for (int j = qk_done; j < qk_issued; ++j)
+        if (!mbar_wait_bounded(&bar_s[j & 1], (j >> 1) & 1)) break;
       if (o_issued > o_done) mbar_wait_bounded(bar_o, o_done & 1);
     }
   } else {
     // ---- epilogue, 32 rows per pass: O / l from TMEM, rotate back, store ----
     tc_fence_after();
-    const float inv = l > 0.f ? a.out_unit / l : 0.f;
+    __syncthreads();
+    float *xchg = reinterpret_cast<float *>(pt);   // [2][kTcRows] row sums; the P tile is free
+    float l0, l1;
+    f2_unpack(l2, l0, l1);
+    const float l = l0 + l1;
+    xchg[half * kTcRows + r] = l;
+    __syncthreads();
+    const float lt = l + xchg[(half ^ 1) * kTcRows + r];
+    const float inv = lt > 0.f ? a.out_unit / lt : 0.f;
     for (int pass = 0; pass < kTcRows / 32; ++pass) {
-      __syncthreads();   // scratch (over the K/V and P buffers) is free
-      if (warp == pass) {
+      __syncthreads();   // scratch (over the K and V tiles) is free
+      if (sub == pass) {
 #pragma unroll 1
-        for (int c = 0; c < D / 16; ++c) {
+        for (int c = 0; c < OH / 16; ++c) {
           float v[16];
           if (n_tiles > 0) {
-            tc_ld16(t_o + lane_off + 16 * c, v);
+            tc_ld16(t_o + OH * half + lane_off + 16 * c, v);
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
           }
 #pragma unroll
-          for (int j = 0; j < 16; ++j) scratch[(r - 32 * pass) * D + 16 * c + j] = v[j] * inv;
+          for (int j = 0; j < 16; ++j) scratch[lane * D + OH * half + 16 * c + j] = v[j] * inv;
         }
       }
       __syncthreads();

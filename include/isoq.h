@@ -367,7 +367,9 @@ int isoq_rotor_dequantize(const uint8_t *codes_dev, const uint16_t *norms_dev, i
  * `stream`.  Returns ISOQ_OK, ISOQ_ERR_TIMEOUT if a kernel's bounded wait
  * gave up since the last check (the kernel then stopped early and its
  * outputs are incomplete), ISOQ_ERR_INVALID_ARG if a decode append met a
- * row that already held Tmax tokens, or ISOQ_ERR_CUDA.
+ * row that already held Tmax tokens, or ISOQ_ERR_CUDA (among others when
+ * the prefill kernel found its dynamic shared memory off a 1024-byte
+ * boundary and returned without output).
  */
 int isoq_check_device_error(isoq_stream_t stream);
 
