@@ -165,20 +165,36 @@ bool codebook_unit_f64(int bits, double *centroids) {
   return true;
 }
 
-// Each split covers a fixed number of tokens (a multiple of 64) chosen so
-// that B * Hkv * n_splits is about 8 CTAs per SM of a 148-SM B200, with
-// chunks between 512 and 4096 tokens (below 512 tokens a split's fixed
-// costs, its set-up and its share of the combine, outweigh the parallelism
-// it adds: measured on a batch-1, 32K-token decode, 42 -> 33 us).
+// Each split covers a fixed number of tokens: a multiple of 64 between 512
+// and 4096 (below 512 tokens a split's fixed costs, its set-up and its share
+// of the combine, outweigh the parallelism it adds).  Among those the chunk
+// c minimises the wave model of the split kernel on a 148-SM B200:
+//   time ~ max(ceil(n_ctas / 148), 4) * (min(c, Tmax) + 128),
+// with n_ctas = B Hkv ceil(Tmax / c): the busiest SM runs ceil(n_ctas / 148)
+// CTAs one after another (an SM is issue-bound once a few CTAs share it),
+// an SM with fewer than 4 CTAs is not faster per CTA for it (too few warps
+// to hide latency), and each CTA costs about 128 tokens' worth of set-up
+// and merge.  Ties go to the larger chunk (fewer partial states to combine).
+// On the decode sweep (batch 32, GQA 16/8, d = 256, contexts 1K..64K, and
+// the batch-1 and ragged batch-16 GQA 32/4 cases) the model picks the
+// fastest of the chunks 512..4096 timed, or one within 0.2 %, where a fixed
+// target of 8 CTAs per SM lost up to 11 % to a nearly empty last wave.
 int64_t decode_chunk_tokens(int B, int Hkv, int64_t Tmax, int d) {
   (void)d;
-  const int64_t target_ctas = 148 * 8;
-  int64_t work = static_cast<int64_t>(B) * Hkv * Tmax;
-  int64_t chunk = (work + target_ctas - 1) / target_ctas;
-  chunk = (chunk + kDecodeTokenQuantum - 1) / kDecodeTokenQuantum * kDecodeTokenQuantum;
-  if (chunk < 512) chunk = 512;
-  if (chunk > 4096) chunk = 4096;
-  return chunk;
+  constexpr int64_t kSms = 148, kMinPerSm = 4, kCtaCost = 128;
+  const int64_t pairs = static_cast<int64_t>(B) * Hkv;
+  int64_t best_chunk = 4096, best_cost = -1;
+  for (int64_t c = 4096; c >= 512; c -= kDecodeTokenQuantum) {
+    const int64_t n_ctas = pairs * ((Tmax + c - 1) / c);
+    int64_t per_sm = (n_ctas + kSms - 1) / kSms;
+    if (per_sm < kMinPerSm) per_sm = kMinPerSm;
+    const int64_t cost = per_sm * ((c < Tmax ? c : Tmax) + kCtaCost);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_chunk = c;
+    }
+  }
+  return best_chunk;
 }
 
 size_t decode_qprep_bytes(int B, int Hkv, int d) {

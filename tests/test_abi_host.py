@@ -73,6 +73,20 @@ def test_split_policy_and_workspace():
     assert isoq.isoq_decode_workspace_size(1, 3, 2, 100, 128) == 0  # Hq % Hkv != 0
 
 
+def test_split_policy_wave_model():
+    """The chunk is a multiple of 64 in [512, 4096]; on the decode sweep's
+    shapes it is the one the timed sweep found fastest (batch 32 x 8 KV heads:
+    1K and 2K contexts 512 tokens, 4K 1024, 8K 2048, 32K and 64K 4096; batch 1
+    x 4 KV heads at 32K: 512)."""
+    expect = {(32, 8, 1024): 2, (32, 8, 2048): 4, (32, 8, 4096): 4, (32, 8, 8192): 4,
+              (32, 8, 32768): 8, (32, 8, 65536): 16, (1, 4, 32768): 64}
+    for (B, hkv, tmax), n in expect.items():
+        assert isoq.isoq_decode_num_splits(B, hkv, tmax, 256) == n, (B, hkv, tmax)
+    for B, hkv, tmax in [(1, 1, 100), (7, 3, 5000), (64, 8, 131072), (2, 16, 300000)]:
+        n = isoq.isoq_decode_num_splits(B, hkv, tmax, 128)
+        assert -(-tmax // 4096) <= n <= max(1, -(-tmax // 512)), (B, hkv, tmax, n)
+
+
 def _call_quantize(**kw):
     args = dict(x=1, dtype=isoq.ISOQ_F16, n_heads=1, n_vec=10, d=128, bits=3,
                 variant=isoq.ISOQ_FULL, hs=1280, vs=128, params=16, codes=16, norms=16,
