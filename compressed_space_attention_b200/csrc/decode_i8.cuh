@@ -129,6 +129,12 @@ __device__ __forceinline__ float ex2f(float x) {
   return r;
 }
 
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // c += A B (s8 x s8), and the same with a zero accumulator.
 __device__ __forceinline__ void mma_s8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -581,7 +587,9 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     // p s^V r + 2^23; one unit of 256 E1 + E2 is then 2^7 pm / kWMax of
     // sum p s^V C (dinv, in the PV layout).  u[T][hh]: (W head 2t, W head
     // 2t+1) of token 16T + 8hh + g.
-    const float r0 = pm0 > 0.f ? kWMax / pm0 : 0.f, r1 = pm1 > 0.f ? kWMax / pm1 : 0.f;
+    // (r needs no IEEE division: any r <= kWMax (1 + 2^-22) / pm keeps W_q
+    // within 16 bits, and dinv below uses pm itself.)
+    const float r0 = pm0 > 0.f ? kWMax * rcp_approx(pm0) : 0.f, r1 = pm1 > 0.f ? kWMax * rcp_approx(pm1) : 0.f;
     uint32_t u[2][2];
 #pragma unroll
     for (int T = 0; T < 2; ++T) {
