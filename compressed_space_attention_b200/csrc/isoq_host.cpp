@@ -165,30 +165,37 @@ bool codebook_unit_f64(int bits, double *centroids) {
   return true;
 }
 
-// Each split covers a fixed number of tokens: a multiple of 64 between 512
-// and 4096 (below 512 tokens a split's fixed costs, its set-up and its share
-// of the combine, outweigh the parallelism it adds).  Among those the chunk
-// c minimises the wave model of the split kernel on a 148-SM B200:
-//   time ~ max(ceil(n_ctas / 148), 4) * (min(c, Tmax) + 128),
-// with n_ctas = B Hkv ceil(Tmax / c): the busiest SM runs ceil(n_ctas / 148)
-// CTAs one after another (an SM is issue-bound once a few CTAs share it),
-// an SM with fewer than 4 CTAs is not faster per CTA for it (too few warps
-// to hide latency), and each CTA costs about 128 tokens' worth of set-up
-// and merge.  Ties go to the larger chunk (fewer partial states to combine).
-// On the decode sweep (batch 32, GQA 16/8, d = 256, contexts 1K..64K, and
-// the batch-1 and ragged batch-16 GQA 32/4 cases) the model picks the
-// fastest of the chunks 512..4096 timed, or one within 0.2 %, where a fixed
-// target of 8 CTAs per SM lost up to 11 % to a nearly empty last wave.
+// Each split covers a fixed number of tokens, one of 512, 768, 1024, 1536,
+// 2048, 3072 or 4096 (below 512 tokens a split's fixed costs, its set-up and
+// its share of the combine, outweigh the parallelism it adds).  The chunk c
+// minimises a wave model of the split kernel on a 148-SM B200 with 4 CTAs
+// resident per SM:
+//   the busiest SM runs m = ceil(n_ctas / 148) CTAs, n_ctas = B Hkv
+//   ceil(Tmax / c), in phases of k = min(4, remaining) concurrent CTAs; a
+//   phase costs (k + 0.7) (min(c, Tmax) + 160)
+// (an SM with k CTAs moves k / (k + 0.7) of its full rate: one CTA's four
+// warps hide little latency; each CTA costs about 160 tokens' worth of
+// set-up and merge).  Ties go to the larger chunk (fewer partial states to
+// combine).  The constants are fitted to the split time over these chunks
+// on 17 shapes (batch 1..32, 8 or 4 KV heads, d = 128 and 256, contexts
+// 1K..64K): the chunk the model picks is within 7 % of the fastest one on
+// every shape, where a fixed target of 8 CTAs per SM lost up to 11 % to a
+// nearly empty last wave.
 int64_t decode_chunk_tokens(int B, int Hkv, int64_t Tmax, int d) {
   (void)d;
-  constexpr int64_t kSms = 148, kMinPerSm = 4, kCtaCost = 128;
+  static constexpr int64_t kChunks[] = {4096, 3072, 2048, 1536, 1024, 768, 512};
+  constexpr int64_t kSms = 148, kSlots = 4, kCtaCost = 160;
   const int64_t pairs = static_cast<int64_t>(B) * Hkv;
   int64_t best_chunk = 4096, best_cost = -1;
-  for (int64_t c = 4096; c >= 512; c -= kDecodeTokenQuantum) {
+  for (const int64_t c : kChunks) {
     const int64_t n_ctas = pairs * ((Tmax + c - 1) / c);
-    int64_t per_sm = (n_ctas + kSms - 1) / kSms;
-    if (per_sm < kMinPerSm) per_sm = kMinPerSm;
-    const int64_t cost = per_sm * ((c < Tmax ? c : Tmax) + kCtaCost);
+    int64_t m = (n_ctas + kSms - 1) / kSms, phases10 = 0;   // sum of 10 (k + 0.7)
+    while (m > 0) {
+      const int64_t k = m < kSlots ? m : kSlots;
+      phases10 += 10 * k + 7;
+      m -= k;
+    }
+    const int64_t cost = phases10 * ((c < Tmax ? c : Tmax) + kCtaCost);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best_chunk = c;
