@@ -238,40 +238,104 @@ __device__ __forceinline__ uint32_t pack_s8x4(int v0, int v1, int v2, int v3) {
 // tile p, column h (GP = 8); the four int8 values are the dims of quad
 // 2 (kk mod 4) + half of lane t's 32-code group (D = 128: group t; D = 256:
 // group 2t + kk / 4).
+//
+// One warp per query head h (GP warps), lane j holding dims E j .. E j + E - 1
+// (E = d / 32) in registers: the Walsh-Hadamard stages h < E inside the
+// lane, the others by shuffles with lane j ^ (h / E), in the same stage
+// order and with the same sums as the shared-memory rotation (so q~ is the
+// same to the bit), then 1/sqrt(d) and the block map on the lane's own 4-dim
+// blocks.  The part words go through shared memory once to their fragment
+// positions.
 template <int D, bool FULL, int GP>
-__global__ void __launch_bounds__(kI8Threads) prep_i8_kernel(const SplitArgs a, float score_unit) {
+__global__ void __launch_bounds__(32 * GP) prep_i8_kernel(const SplitArgs a, float score_unit) {
   using C = I8Cfg<D, GP>;
-  __shared__ float qs[GP * D];
-  __shared__ float qinv[8];
+  constexpr int E = D / 32, NQUAD = D / 4;
+  __shared__ uint32_t pw[3][GP][NQUAD];   // part p of head h, dims 4 quad .. + 3
+  __shared__ float qinv_s[8];
   const int kvh = blockIdx.x, b = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, h = tid >> 5, lane = tid & 31;
   const int G = a.group;
   pdl_launch_dependents();   // the split kernel may start its staging now
-  for (int i = tid; i < GP * D; i += kI8Threads) {
-    const int gq = i / D;
-    float v = 0.f;
-    if (gq < G) {
-      const __half *qp = static_cast<const __half *>(a.q) +
-                         (static_cast<long long>(b) * a.hq + kvh * G + gq) * D;
-      v = __half2float(qp[i % D]);
-    }
-    qs[i] = v;
-  }
-  __syncthreads();
-  rotate_forward_smem<D, FULL>(qs, G, a.params_k + static_cast<size_t>(kvh) * 2 * D, tid, kI8Threads, 0);
-  for (int h = warp; h < 8; h += kI8Warps) {
-    float mx = 0.f;
-    if (h < G)
-      for (int i = lane; i < D; i += 32) mx = fmaxf(mx, fabsf(qs[h * D + i]));
+
+  float x[E];
+  if (h < G) {
+    const __half *qp = static_cast<const __half *>(a.q) + (static_cast<long long>(b) * a.hq + kvh * G + h) * D + E * lane;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) qinv[h] = mx / static_cast<float>(kQueryIntMax);
+    for (int e = 0; e < E; e += 2) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(qp + e));
+      x[e] = f.x;
+      x[e + 1] = f.y;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[e] = 0.f;
+  }
+  // Walsh-Hadamard stages (a, b) -> (a + b, a - b), h = 1, 2, ..., d/2.
+#pragma unroll
+  for (int hs = 1; hs < E; hs <<= 1) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if (!(e & hs)) {
+        const float u = x[e], v = x[e + hs];
+        x[e] = u + v;
+        x[e + hs] = u - v;
+      }
+    }
+  }
+#pragma unroll
+  for (int lm = 1; lm < 32; lm <<= 1) {
+    const bool upper = (lane & lm) != 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[e], lm);
+      x[e] = upper ? o - x[e] : x[e] + o;
+    }
+  }
+  const float inv = rsqrtf(static_cast<float>(D));
+  const float *prm = a.params_k + static_cast<size_t>(kvh) * 2 * D;
+  float mx = 0.f;
+#pragma unroll
+  for (int u = 0; u < E / 4; ++u) {
+    const int bi = (E / 4) * lane + u;
+    const Quat v{x[4 * u] * inv, x[4 * u + 1] * inv, x[4 * u + 2] * inv, x[4 * u + 3] * inv};
+    const Quat r = block_forward(load_quat(prm + 8 * bi), load_quat(prm + 8 * bi + 4), v, FULL);
+    x[4 * u] = r.w;
+    x[4 * u + 1] = r.x;
+    x[4 * u + 2] = r.y;
+    x[4 * u + 3] = r.z;
+  }
+  if (h < G) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) mx = fmaxf(mx, fabsf(x[e]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float qi = mx / static_cast<float>(kQueryIntMax);
+  const float qsc = qi > 0.f ? 1.f / qi : 0.f;
+  if (lane == 0) qinv_s[h] = qi;
+  if (h == 0 && lane >= GP && lane < 8) qinv_s[lane] = 0.f;
+#pragma unroll
+  for (int u = 0; u < E / 4; ++u) {
+    int v[3][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int q = h < G ? __float2int_rn(x[4 * u + i] * qsc) : 0;
+      q = q > kQueryIntMax ? kQueryIntMax : (q < -kQueryIntMax ? -kQueryIntMax : q);
+      const int r1 = (q + 64) >> 7, ql = q - 128 * r1;     // arithmetic shifts: floor
+      const int r2 = (r1 + 64) >> 7, qm = r1 - 128 * r2;
+      v[0][i] = r2;
+      v[1][i] = qm;
+      v[2][i] = ql;
+    }
+#pragma unroll
+    for (int p = 0; p < 3; ++p) pw[p][h][(E / 4) * lane + u] = pack_s8x4(v[p][0], v[p][1], v[p][2], v[p][3]);
   }
   __syncthreads();
 
+  // Word ((nq KK + kk) 2 + half) 32 + lane of the B fragments (see above).
   uint32_t *out = a.ws_qprep + (static_cast<long long>(b) * a.hkv + kvh) * C::QPREP_WORDS;
   constexpr int NWORDS = C::NQ * C::KK * 2 * 32;
-  for (int idx = tid; idx < NWORDS; idx += kI8Threads) {
+  for (int idx = tid; idx < NWORDS; idx += 32 * GP) {
     const int ln = idx & 31, half = (idx >> 5) & 1, kk = (idx >> 6) % C::KK, nq = (idx >> 6) / C::KK;
     const int g = ln >> 2, t = ln & 3;
     int head, part;
@@ -286,22 +350,10 @@ __global__ void __launch_bounds__(kI8Threads) prep_i8_kernel(const SplitArgs a, 
       head = g;
     }
     const bool live = part < 3 && head < G;
-    const float qi = live ? qinv[head] : 0.f;
-    const float qsc = qi > 0.f ? 1.f / qi : 0.f;
     const int grp = (D == 256 ? 2 * t : t) + kk / 4;
-    const int base = 32 * grp + 4 * (2 * (kk & 3) + half);
-    int v[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int q = live ? __float2int_rn(qs[head * D + base + i] * qsc) : 0;
-      q = q > kQueryIntMax ? kQueryIntMax : (q < -kQueryIntMax ? -kQueryIntMax : q);
-      const int r1 = (q + 64) >> 7, ql = q - 128 * r1;     // arithmetic shifts: floor
-      const int r2 = (r1 + 64) >> 7, qm = r1 - 128 * r2;
-      v[i] = part == 0 ? r2 : (part == 1 ? qm : ql);
-    }
-    out[idx] = pack_s8x4(v[0], v[1], v[2], v[3]);
+    out[idx] = live ? pw[part][head][8 * grp + 2 * (kk & 3) + half] : 0u;
   }
-  if (tid < 8) out[3 * C::KK * 2 * 32 + tid] = __float_as_uint(tid < G ? qinv[tid] * score_unit : 0.f);
+  if (tid < 8) out[3 * C::KK * 2 * 32 + tid] = __float_as_uint(tid < G ? qinv_s[tid] * score_unit : 0.f);
 }
 
 // GP: query heads per KV head rounded up to 1, 2, 4 or 8 (padded heads carry
@@ -823,7 +875,7 @@ int launch_split_i8(const SplitArgs &a, cudaStream_t stream) {
   const float out_scale = static_cast<float>(unit);
   dim3 grid(a.n_splits, a.hkv, a.batch);
   static_assert(C::QPREP_WORDS == decode_qprep_words(D), "prepared-query layout");
-  prep_i8_kernel<D, FULL, GP><<<dim3(a.hkv, a.batch), kI8Threads, 0, stream>>>(a, score_unit);
+  prep_i8_kernel<D, FULL, GP><<<dim3(a.hkv, a.batch), 32 * GP, 0, stream>>>(a, score_unit);
   cudaError_t e = launch_pdl(kernel, grid, dim3(kI8Threads), C::SMEM, stream, a, tb.lut, out_scale);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode i8 launch: %s", cudaGetErrorString(e));
