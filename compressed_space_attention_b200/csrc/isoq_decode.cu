@@ -103,31 +103,6 @@ __device__ void rotate_forward_smem(float *v, int nvec, const float *params_head
   rotation_sync(bar_id, nthreads);
 }
 
-// Inverse rotation x = H_d R_SO4^T u / sqrt(d) of one vector in shared memory.
-template <int D, bool FULL>
-__device__ void rotate_inverse_cta(float *v, const float *params_head) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  for (int bi = tid; bi < D / 4; bi += nt) {
-    const Quat u{v[4 * bi], v[4 * bi + 1], v[4 * bi + 2], v[4 * bi + 3]};
-    const Quat x = block_inverse(load_quat(params_head + 8 * bi), load_quat(params_head + 8 * bi + 4), u, FULL);
-    v[4 * bi] = x.w;
-    v[4 * bi + 1] = x.x;
-    v[4 * bi + 2] = x.y;
-    v[4 * bi + 3] = x.z;
-  }
-  __syncthreads();
-#pragma unroll 1
-  for (int h = 1; h < D; h <<= 1) {
-    for (int p = tid; p < D / 2; p += nt) {
-      const int i = (p / h) * 2 * h + (p % h);
-      const float a = v[i], b = v[i + h];
-      v[i] = a + b;
-      v[i + h] = a - b;
-    }
-    __syncthreads();
-  }
-}
-
 template <typename T>
 __device__ __forceinline__ float to_f32(T v);
 template <>
@@ -261,16 +236,20 @@ constexpr int kCombineWBlock = 1024;    // split weights held in shared memory p
 // One CTA per (b, qh).  The split weights w_s = exp(m_s - m*) are computed
 // once per split (not once per split and dimension) into shared memory; the
 // threads then sum acc_s[i] w_s with kCombineThreads / D threads per
-// dimension, each over every (kCombineThreads / D)-th split.
+// dimension, each over every (kCombineThreads / D)-th split.  Warp 0 then
+// normalises and rotates back in registers, lane j holding dims E j .. + E - 1
+// (E = D / 32): x = H_d R_SO4^T u / sqrt(d), the block maps on its own
+// 4-dim blocks first, then the Walsh-Hadamard stages h = 1, 2, ..., D/2
+// ((a, b) -> (a + b, a - b)), those with h < E inside the lane and the others
+// by shuffles.  Three block barriers in all.
 template <typename T, int D, bool FULL>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineArgs a) {
   constexpr int P = D >= kCombineThreads ? 1 : kCombineThreads / D;   // threads per dimension
   constexpr int DPT = D > kCombineThreads ? D / kCombineThreads : 1;  // dimensions per thread
-  __shared__ float v[D];
-  __shared__ float part[P > 1 ? P : 1][D];
+  constexpr int NW = kCombineThreads / 32, E = D / 32;
+  __shared__ float part[P][D];
   __shared__ float wsh[kCombineWBlock];
-  __shared__ float red[kCombineThreads / 32];
-  __shared__ float s_mstar, s_l;
+  __shared__ float red_m[NW], red_l[NW];
   const int qh = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kvh = qh / a.group;
@@ -282,15 +261,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
   for (int s = tid; s < a.n_splits; s += kCombineThreads) mx = fmaxf(mx, a.ws_ml[base + s].x);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) red[warp] = mx;
+  if (lane == 0) red_m[warp] = mx;
   __syncthreads();
-  if (tid == 0) {
-    float m = red[0];
-    for (int w = 1; w < kCombineThreads / 32; ++w) m = fmaxf(m, red[w]);
-    s_mstar = m;
-  }
-  __syncthreads();
-  const float mstar = s_mstar;
+  float mstar = red_m[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) mstar = fmaxf(mstar, red_m[w]);
 
   const int p = tid / (D < kCombineThreads ? D : kCombineThreads);
   const int i0 = tid % (D < kCombineThreads ? D : kCombineThreads);
@@ -300,7 +275,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
   float lsum = 0.f;
   for (int s0 = 0; s0 < a.n_splits; s0 += kCombineWBlock) {
     const int ns = a.n_splits - s0 < kCombineWBlock ? a.n_splits - s0 : kCombineWBlock;
-    __syncthreads();   // the previous pass no longer reads wsh
+    if (s0 > 0) __syncthreads();   // the previous pass no longer reads wsh
     for (int s = tid; s < ns; s += kCombineThreads) {
       const float2 ml = a.ws_ml[base + s0 + s];
       const float w = ml.y > 0.f ? expf(ml.x - mstar) : 0.f;
@@ -318,34 +293,59 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  if (lane == 0) red[warp] = lsum;
-  if (P > 1) {
-    part[p][i0] = acc[0];
-  }
-  __syncthreads();
-  if (tid == 0) {
-    float l = 0.f;
-    for (int w = 0; w < kCombineThreads / 32; ++w) l += red[w];
-    s_l = l;
-  }
-  __syncthreads();
-  const float inv_l = s_l > 0.f ? 1.f / s_l : 0.f;
-  if (P > 1) {
-    for (int i = tid; i < D; i += kCombineThreads) {
-      float t = 0.f;
+  if (lane == 0) red_l[warp] = lsum;
 #pragma unroll
-      for (int q = 0; q < P; ++q) t += part[q][i];
-      v[i] = t * inv_l;
+  for (int k = 0; k < DPT; ++k) part[p][i0 + k * kCombineThreads] = acc[k];
+  __syncthreads();
+  if (warp != 0) return;
+
+  float l = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) l += red_l[w];
+  const float inv_l = l > 0.f ? 1.f / l : 0.f;
+  float x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    float t = 0.f;
+#pragma unroll
+    for (int q = 0; q < P; ++q) t += part[q][E * lane + e];
+    x[e] = t * inv_l;
+  }
+  const float *prm = a.params_v + static_cast<size_t>(kvh) * 2 * D;
+#pragma unroll
+  for (int u = 0; u < E / 4; ++u) {
+    const int bi = (E / 4) * lane + u;
+    const Quat r = block_inverse(load_quat(prm + 8 * bi), load_quat(prm + 8 * bi + 4),
+                                 Quat{x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]}, FULL);
+    x[4 * u] = r.w;
+    x[4 * u + 1] = r.x;
+    x[4 * u + 2] = r.y;
+    x[4 * u + 3] = r.z;
+  }
+#pragma unroll
+  for (int hs = 1; hs < E; hs <<= 1) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if (!(e & hs)) {
+        const float u = x[e], v = x[e + hs];
+        x[e] = u + v;
+        x[e + hs] = u - v;
+      }
     }
-  } else {
-#pragma unroll
-    for (int k = 0; k < DPT; ++k) v[i0 + k * kCombineThreads] = acc[k] * inv_l;
   }
-  __syncthreads();
-  rotate_inverse_cta<D, FULL>(v, a.params_v + static_cast<size_t>(kvh) * 2 * D);
+#pragma unroll
+  for (int lm = 1; lm < 32; lm <<= 1) {
+    const bool upper = (lane & lm) != 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[e], lm);
+      x[e] = upper ? o - x[e] : x[e] + o;
+    }
+  }
   const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
-  T *out = static_cast<T *>(a.out) + (static_cast<long long>(b) * a.hq + qh) * D;
-  for (int i = tid; i < D; i += kCombineThreads) out[i] = from_f32<T>(v[i] * inv_sqrt_d);
+  T *out = static_cast<T *>(a.out) + (static_cast<long long>(b) * a.hq + qh) * D + E * lane;
+#pragma unroll
+  for (int e = 0; e < E; ++e) out[e] = from_f32<T>(x[e] * inv_sqrt_d);
 }
 
 #include "decode_i8.cuh"
