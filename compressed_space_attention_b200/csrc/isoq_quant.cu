@@ -92,10 +92,14 @@ struct Cfg : Lanes<D> {
   using Lanes<D>::VPW;
   static constexpr int NV = kQuantWarps * VPW;  // vectors per CTA tile
   static constexpr int ES = sizeof(T);
-  static constexpr int BOX_ELEMS = 128 / ES;    // elements in one 128-byte box row
-  static constexpr int NBOX = D * ES / 128;     // boxes per row
-  static constexpr int BOX_BYTES = VPW * 128;   // one warp's rows of one box
-  // 128B-swizzled boxes start on 1024-byte boundaries.
+  static constexpr int BOX_ELEMS = 128 / ES;    // elements in one 128-byte chunk of a row
+  // A box holds CPB consecutive 128-byte chunks of each of the warp's VPW
+  // rows, so that it fills the 1024 bytes a 128B-swizzled box is aligned to
+  // (d = 512: 4 rows x 2 chunks; the rows are then viewed as [chunk][elem]
+  // by a 4-D tensor map).
+  static constexpr int CPB = VPW >= 8 ? 1 : 8 / VPW;
+  static constexpr int NBOX = D * ES / 128 / CPB;   // boxes per row
+  static constexpr int BOX_BYTES = VPW * CPB * 128; // one warp's rows of one box
   static constexpr int BOX_STRIDE = BOX_BYTES < 1024 ? 1024 : BOX_BYTES;
   static constexpr int STAGE_BYTES = NBOX * BOX_STRIDE;
   static constexpr int STAGES = STAGE_BYTES >= 8192 ? 2 : 3;
@@ -123,6 +127,25 @@ struct QuantArgs {
 // ---------------------------------------------------------------------------
 // Register-level pieces
 // ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+// Shared address of chunk ch (128 bytes of a row) of the warp's row vl in a
+// ring stage, and the row's swizzle phase there: inside a box the 128-byte
+// lines run (row, chunk) with the chunk fastest.
+template <typename C>
+__device__ __forceinline__ uint32_t stage_line(uint32_t stage, int ch, int vl, uint32_t &sw) {
+  const int line = vl * C::CPB + ch % C::CPB;
+  sw = static_cast<uint32_t>(line & 7);
+  return stage + (ch / C::CPB) * C::BOX_STRIDE + line * 128;
+}
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -390,8 +413,12 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     const int s = i % C::STAGES;
     unsigned char *st = ring + s * C::STAGE_BYTES;
     mbar_arrive_expect_tx(&full_bar[s], C::NBOX * C::BOX_BYTES);
-    for (int b = 0; b < C::NBOX; ++b)
-      tma_load_3d(st + b * C::BOX_STRIDE, &xmap, &full_bar[s], b * C::BOX_ELEMS, v0, head);
+    for (int b = 0; b < C::NBOX; ++b) {
+      if constexpr (C::CPB == 1)
+        tma_load_3d(st + b * C::BOX_STRIDE, &xmap, &full_bar[s], b * C::BOX_ELEMS, v0, head);
+      else
+        tma_load_4d(st + b * C::BOX_STRIDE, &xmap, &full_bar[s], 0, b * C::CPB, v0, head);
+    }
   };
   int issued = 0;
   if (lane == 0)
@@ -443,9 +470,9 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     // doing the h = 16 butterfly on the way.
     uint64_t xp[kPairs];
     const uint32_t stage = smem_u32(ring + s * C::STAGE_BYTES);
-    const uint32_t sw = static_cast<uint32_t>(vl & 7);
     if constexpr (C::ES == 2) {
-      const uint32_t row = stage + part * C::BOX_STRIDE + vl * 128;
+      uint32_t sw;
+      const uint32_t row = stage_line<C>(stage, part, vl, sw);
 #pragma unroll
       for (int G = 0; G < 2; ++G) {
 #pragma unroll
@@ -471,7 +498,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     } else {
 #pragma unroll
       for (int G = 0; G < 2; ++G) {
-        const uint32_t row = stage + (2 * part + G) * C::BOX_STRIDE + vl * 128;
+        uint32_t sw;
+        const uint32_t row = stage_line<C>(stage, 2 * part + G, vl, sw);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint4 ulo = lds128(row + ((c ^ sw) << 4));
@@ -775,11 +803,24 @@ int launch_quantize(const void *x, int n_heads, long long n_vec, long long head_
   const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(vec_stride * C::ES),
                                  static_cast<cuuint64_t>(hs * C::ES)};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(C::BOX_ELEMS), static_cast<cuuint32_t>(C::VPW), 1u};
-  const cuuint32_t estride[3] = {1u, 1u, 1u};
-  CUresult r = encode(&map, C::ES == 2 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                      3, const_cast<void *>(x), gdim, gstride, box, estride,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
+  const CUtensorMapDataType dt = C::ES == 2 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUresult r;
+  if constexpr (C::CPB == 1) {
+    r = encode(&map, dt, 3, const_cast<void *>(x), gdim, gstride, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    // Rows as [D / BOX_ELEMS chunks][BOX_ELEMS], the box CPB chunks x VPW rows.
+    const cuuint64_t gdim4[4] = {static_cast<cuuint64_t>(C::BOX_ELEMS), static_cast<cuuint64_t>(D / C::BOX_ELEMS),
+                                 static_cast<cuuint64_t>(n_vec), static_cast<cuuint64_t>(n_heads)};
+    const cuuint64_t gstride4[3] = {128u, gstride[0], gstride[1]};
+    const cuuint32_t box4[4] = {static_cast<cuuint32_t>(C::BOX_ELEMS), static_cast<cuuint32_t>(C::CPB),
+                                static_cast<cuuint32_t>(C::VPW), 1u};
+    r = encode(&map, dt, 4, const_cast<void *>(x), gdim4, gstride4, box4, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
   if (r != CUDA_SUCCESS) return set_error(ISOQ_ERR_UNSUPPORTED, "quantize: tensor map encode failed (%d)", (int)r);
 
   QuantArgs a;

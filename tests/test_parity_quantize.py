@@ -110,15 +110,17 @@ def test_empty_is_noop():
     assert codes.shape == (2, 0, 48) and norms.shape == (2, 0)
 
 
-def test_token_major_input_into_larger_cache():
+@pytest.mark.parametrize("d,dtype", [(128, np.float16), (512, np.float16), (512, np.float32)])
+def test_token_major_input_into_larger_cache(d, dtype):
     """x in token-major [T][Hkv][d] layout written into a [Hkv][Tmax] cache at
-    an offset: strided input and out_head_stride > n_vec."""
-    hkv, t, d, tmax, off = 3, 200, 128, 512, 40
-    xt = synth.unit_vectors(t * hkv, d, seed=9, dtype=np.float16).reshape(t, hkv, d)
+    an offset: strided input and out_head_stride > n_vec (at d = 512 the rows
+    are staged through a 4-D tensor map of 128-byte chunks)."""
+    hkv, t, tmax, off = 3, 200, 512, 40
+    xt = synth.unit_vectors(t * hkv, d, seed=9, dtype=dtype).reshape(t, hkv, d)
     params = O.make_params(d, O.FULL, seed=6, n_heads=hkv)
     x_dev = torch.from_numpy(xt).to(DEV)
     view = x_dev.permute(1, 0, 2)                     # [Hkv][T][d], strides (d, Hkv*d, 1)
-    cache_codes = torch.full((hkv, tmax, 48), 0xAB, dtype=torch.uint8, device=DEV)
+    cache_codes = torch.full((hkv, tmax, d * 3 // 8), 0xAB, dtype=torch.uint8, device=DEV)
     cache_norms = torch.full((hkv, tmax), 7.0, dtype=torch.float16, device=DEV)
     isoq.isoq_quantize(view, torch.from_numpy(params).to(DEV), 3, O.FULL,
                        codes=cache_codes[:, off:], norms=cache_norms[:, off:], out_head_stride=tmax)
