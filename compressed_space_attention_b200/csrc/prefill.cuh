@@ -260,6 +260,9 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   uint64_t *bar_s = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);   // [2]: S buffer b's product done
   uint64_t *bar_o = bar_s + 2;                                          // PV product done
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_o + 1);
+  // A product wait that gave up in iteration j sets fail_s[j % 2]; it is read
+  // after the iteration's last block barrier (see the loop).
+  volatile uint8_t *fail_s = reinterpret_cast<volatile uint8_t *>(tmem_slot + 1);
   float *scratch = reinterpret_cast<float *>(kt);   // 32 rows x D floats over the K and V tiles (prep, epilogue)
 
   const int qt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -308,6 +311,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
     mbar_init(&bar_s[0], 1);
     mbar_init(&bar_s[1], 1);
     mbar_init(bar_o, 1);
+    fail_s[0] = fail_s[1] = 0;
     mbar_fence_init();
   }
 
@@ -399,18 +403,27 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   }
   for (int it = 0; it < n_tiles; ++it) {
     const int t0 = it * kTcTok;
-    // QK(it) must be complete: its S buffer is read below and the K tile is free.
-    bool ok = mbar_wait_bounded(&bar_s[it & 1], (it >> 1) & 1);
-    if (__syncthreads_or(!ok)) {
-      failed = true;
-      break;
-    }
-    ++qk_done;
+    // QK(it) must be complete: its S buffer is read below and the K tile is
+    // free.  Every thread waits on the mbarrier itself, so no block barrier
+    // follows: a wait that gave up is recorded in fail_s[it % 2], which all
+    // threads read after the block barrier that ends the iteration and leave
+    // the loop together.  (A flag per iteration parity: the writes of
+    // iteration it + 2 come after every thread has passed the barrier that
+    // ends iteration it + 1, i.e. after every read of iteration it.)
+    if (mbar_wait_bounded(&bar_s[it & 1], (it >> 1) & 1))
+      ++qk_done;
+    else
+      fail_s[it & 1] = 1;
     tc_fence_after();
     // The next tile's QK runs on the tensor cores under this tile's softmax.
+    // Its block barrier also publishes this tile's norms, stored after the
+    // previous iteration's last barrier; the last tile needs a barrier of
+    // its own for that.
     if (it + 1 < n_tiles) {
       stage_qk(it + 1);
       ++qk_issued;
+    } else {
+      __syncthreads();
     }
 
     // ---- softmax on this thread's half row of S(it) ----
@@ -442,19 +455,16 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
 
     // PV(it - 1) must be complete before O is rescaled and the V tile
     // reused; with one P tile, already before P(it) is written.
-    auto wait_pv = [&]() -> bool {
+    auto wait_pv = [&]() {
       if (o_issued > o_done) {
-        const bool done = mbar_wait_bounded(bar_o, o_done & 1);
-        if (__syncthreads_or(!done)) return false;
-        ++o_done;
+        if (mbar_wait_bounded(bar_o, o_done & 1))
+          ++o_done;
+        else
+          fail_s[it & 1] = 1;
         tc_fence_after();
       }
-      return true;
     };
-    if (C::P_BUFS == 1 && !wait_pv()) {
-      failed = true;
-      break;
-    }
+    if (C::P_BUFS == 1) wait_pv();
     unsigned char *pb = pt + (it % C::P_BUFS) * C::P_BYTES;   // free: PV(it - P_BUFS) is complete
     // The row maximum over both column halves, exchanged with the partner
     // warp through the free P tile: each thread leaves its value in the
@@ -486,10 +496,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
       }
       *reinterpret_cast<uint4 *>(pb + tc_off(r, HC * half + 8 * c, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    if (C::P_BUFS == 2 && !wait_pv()) {
-      failed = true;
-      break;
-    }
+    if (C::P_BUFS == 2) wait_pv();
 
     if (moved && it > 0) {
 #pragma unroll 1
@@ -509,6 +516,10 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (fail_s[it & 1]) {   // the same value for every thread
+      failed = true;
+      break;
+    }
     // Every thread is past the softmax of tile it: its norms can be replaced.
     if (it + 1 < n_tiles) {
       store_norm();
