@@ -84,8 +84,10 @@ struct I8Cfg {
   static constexpr int MB = D / 64;                         // PV M-blocks (64 dims each)
   static constexpr int NQ = GP <= 2 ? 1 : (GP == 4 ? 2 : 3);  // QK N tiles (3 parts x GP columns)
   static constexpr int NV = (GP + 1) / 2;                   // PV N tiles (2 heads each)
-  static constexpr int SCRATCH_FLOATS = GP * D;             // the warp merge
+  static constexpr int SCRATCH_FLOATS = GP * D;             // the sequential warp merge
+  static constexpr int MERGE_FLOATS = kI8Warps * GP * D;    // the sliced warp merge, over the rings
   static constexpr int QPREP_WORDS = 3 * KK * 2 * 32 + 8;   // per (b, kvh), see prep_i8_kernel
+  static_assert(MERGE_FLOATS * 4 <= kI8Warps * RING_BYTES, "merge slices fit the rings");
   static constexpr int SMEM = kI8Warps * RING_BYTES + SCRATCH_FLOATS * 4 +
                               2 * kI8Warps * 8 * 4 + kI8Warps * kI8Stages * 8 + 128;
   static constexpr int MIN_BLOCKS = (D == 256 && GP == 8) ? 2 : ((D == 256 && GP == 4) || GP == 8 ? 3 : 4);
@@ -357,8 +359,13 @@ __global__ void __launch_bounds__(32 * GP) prep_i8_kernel(const SplitArgs a, flo
 }
 
 // GP: query heads per KV head rounded up to 1, 2, 4 or 8 (padded heads carry
-// zero queries and zero weights).
-template <int D, bool FULL, int GP>
+// zero queries and zero weights).  SLICES selects the warp merge: every warp
+// into its own slice and one barrier (for short chunks, where the merge is a
+// visible share of a CTA's time: batch-1 32K-token decode 27.0 -> 22.9 us),
+// or one warp after the other into one buffer, a barrier each (for long
+// chunks, where the sliced form measured 0.7 % slower: it changes how the
+// main loop compiles).
+template <int D, bool FULL, int GP, bool SLICES>
 __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     split_i8_kernel(const SplitArgs a, const I8Lut lut, float out_scale) {
   using C = I8Cfg<D, GP>;
@@ -743,64 +750,120 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
-  __syncthreads();   // all warps are done with the q~ scratch
-  if (g == 0) {
-    wm[warp * 8 + 2 * t] = m0;
-    wm[warp * 8 + 2 * t + 1] = m1;
-    wl[warp * 8 + 2 * t] = l0;
-    wl[warp * 8 + 2 * t + 1] = l1;
-  }
-  __syncthreads();
-  // Merge the warps' accumulators into scratch[head][dim] (rotated domain),
-  // one warp after the other so that the sum order is fixed.
-  {
-    const int grp = D == 256 ? g : (g >> 1);
-    const int qoff = D == 256 ? 0 : 4 * (g & 1);
-    float f[C::NV];
-#pragma unroll
-    for (int nvt = 0; nvt < C::NV; ++nvt) {
-      const int h = 2 * nvt + (t >> 1);
+  if constexpr (SLICES) {
+    __syncthreads();   // every warp is done with its ring, and its copies have landed
+    // Each warp's accumulators go raw into its own slice [warp][head][dim]
+    // (rotated domain) over the ring memory; after one barrier the slices are
+    // scaled to the common maximum and summed in warp order (a fixed order).
+    float *slices = reinterpret_cast<float *>(smem);
+    if (g == 0) {
+      wm[warp * 8 + 2 * t] = m0;
+      wm[warp * 8 + 2 * t + 1] = m1;
+      wl[warp * 8 + 2 * t] = l0;
+      wl[warp * 8 + 2 * t + 1] = l1;
+    }
+    {
+      const int grp = D == 256 ? g : (g >> 1);
+      const int qoff = D == 256 ? 0 : 4 * (g & 1);
+  #pragma unroll
+      for (int nvt = 0; nvt < C::NV; ++nvt) {
+        const int h = 2 * nvt + (t >> 1);
+        if (h < G) {
+          float *dst = slices + (warp * GP + h) * D;
+  #pragma unroll
+          for (int mb = 0; mb < C::MB; ++mb)
+  #pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[32 * grp + 4 * (2 * mb + (e >> 1) + qoff) + 2 * (t & 1) + (e & 1)] = acc[nvt][mb][e];
+        }
+      }
+    }
+    __syncthreads();
+
+    // One partial state per query head: natural-log max, sum, acc (unscaled).
+    for (int h = 0; h < G; ++h) {
       float mstar = -INFINITY;
       for (int w2 = 0; w2 < kI8Warps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
-      const float mine = wm[warp * 8 + h];
-      f[nvt] = (mine == -INFINITY) ? 0.f : exp2f(mine - mstar);
+      float f[kI8Warps];
+  #pragma unroll
+      for (int w2 = 0; w2 < kI8Warps; ++w2) {
+        const float mw = wm[w2 * 8 + h];
+        f[w2] = mw == -INFINITY ? 0.f : exp2f(mw - mstar);
+      }
+      const long long slot = (static_cast<long long>(b) * a.hq + kvh * G + h) * a.n_splits + split;
+      float *acc_out = a.ws_acc + slot * D;
+      for (int i = tid; i < D; i += kI8Threads) {
+        float sum = 0.f;
+  #pragma unroll
+        for (int w2 = 0; w2 < kI8Warps; ++w2) sum += slices[(w2 * GP + h) * D + i] * f[w2];
+        acc_out[i] = sum * out_scale;
+      }
+      if (tid == 0) {
+        float l = 0.f;
+        for (int w2 = 0; w2 < kI8Warps; ++w2) l += wl[w2 * 8 + h] * f[w2];
+        a.ws_ml[slot] = make_float2(mstar == -INFINITY ? -INFINITY : mstar * 0.69314718055994531f, l);
+      }
     }
-    for (int w2 = 0; w2 < kI8Warps; ++w2) {
-      if (warp == w2) {
-#pragma unroll
-        for (int nvt = 0; nvt < C::NV; ++nvt) {
-          const int h = 2 * nvt + (t >> 1);
-          if (h < G) {
-#pragma unroll
-            for (int mb = 0; mb < C::MB; ++mb) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int dim = 32 * grp + 4 * (2 * mb + (e >> 1) + qoff) + 2 * (t & 1) + (e & 1);
-                float *dst = scratch + h * D + dim;
-                const float v = acc[nvt][mb][e] * f[nvt];
-                *dst = (w2 == 0) ? v : *dst + v;
+  } else {
+    __syncthreads();   // all warps are done with the q~ scratch
+    if (g == 0) {
+      wm[warp * 8 + 2 * t] = m0;
+      wm[warp * 8 + 2 * t + 1] = m1;
+      wl[warp * 8 + 2 * t] = l0;
+      wl[warp * 8 + 2 * t + 1] = l1;
+    }
+    __syncthreads();
+    // Merge the warps' accumulators into scratch[head][dim] (rotated domain),
+    // one warp after the other so that the sum order is fixed.
+    {
+      const int grp = D == 256 ? g : (g >> 1);
+      const int qoff = D == 256 ? 0 : 4 * (g & 1);
+      float f[C::NV];
+  #pragma unroll
+      for (int nvt = 0; nvt < C::NV; ++nvt) {
+        const int h = 2 * nvt + (t >> 1);
+        float mstar = -INFINITY;
+        for (int w2 = 0; w2 < kI8Warps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
+        const float mine = wm[warp * 8 + h];
+        f[nvt] = (mine == -INFINITY) ? 0.f : exp2f(mine - mstar);
+      }
+      for (int w2 = 0; w2 < kI8Warps; ++w2) {
+        if (warp == w2) {
+  #pragma unroll
+          for (int nvt = 0; nvt < C::NV; ++nvt) {
+            const int h = 2 * nvt + (t >> 1);
+            if (h < G) {
+  #pragma unroll
+              for (int mb = 0; mb < C::MB; ++mb) {
+  #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int dim = 32 * grp + 4 * (2 * mb + (e >> 1) + qoff) + 2 * (t & 1) + (e & 1);
+                  float *dst = scratch + h * D + dim;
+                  const float v = acc[nvt][mb][e] * f[nvt];
+                  *dst = (w2 == 0) ? v : *dst + v;
+                }
               }
             }
           }
         }
+        __syncthreads();
       }
-      __syncthreads();
     }
-  }
 
-  // One partial state per query head: natural-log max, sum, acc (unscaled).
-  for (int h = 0; h < G; ++h) {
-    const long long slot = (static_cast<long long>(b) * a.hq + kvh * G + h) * a.n_splits + split;
-    float *acc_out = a.ws_acc + slot * D;
-    for (int i = tid; i < D; i += kI8Threads) acc_out[i] = scratch[h * D + i] * out_scale;
-    if (tid == 0) {
-      float mstar = -INFINITY, l = 0.f;
-      for (int w2 = 0; w2 < kI8Warps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
-      for (int w2 = 0; w2 < kI8Warps; ++w2) {
-        const float mw = wm[w2 * 8 + h];
-        if (mw != -INFINITY) l += wl[w2 * 8 + h] * exp2f(mw - mstar);
+    // One partial state per query head: natural-log max, sum, acc (unscaled).
+    for (int h = 0; h < G; ++h) {
+      const long long slot = (static_cast<long long>(b) * a.hq + kvh * G + h) * a.n_splits + split;
+      float *acc_out = a.ws_acc + slot * D;
+      for (int i = tid; i < D; i += kI8Threads) acc_out[i] = scratch[h * D + i] * out_scale;
+      if (tid == 0) {
+        float mstar = -INFINITY, l = 0.f;
+        for (int w2 = 0; w2 < kI8Warps; ++w2) mstar = fmaxf(mstar, wm[w2 * 8 + h]);
+        for (int w2 = 0; w2 < kI8Warps; ++w2) {
+          const float mw = wm[w2 * 8 + h];
+          if (mw != -INFINITY) l += wl[w2 * 8 + h] * exp2f(mw - mstar);
+        }
+        a.ws_ml[slot] = make_float2(mstar == -INFINITY ? -INFINITY : mstar * 0.69314718055994531f, l);
       }
-      a.ws_ml[slot] = make_float2(mstar == -INFINITY ? -INFINITY : mstar * 0.69314718055994531f, l);
     }
   }
 }
@@ -858,14 +921,18 @@ const I8Tables &i8_tables() {
 template <int D, bool FULL, int GP>
 int launch_split_i8(const SplitArgs &a, cudaStream_t stream) {
   using C = I8Cfg<D, GP>;
-  auto kernel = split_i8_kernel<D, FULL, GP>;
+  // The sliced warp merge for chunks up to 2048 tokens (see split_i8_kernel).
+  const bool slices = a.chunk <= 2048;
+  auto kernel = slices ? split_i8_kernel<D, FULL, GP, true> : split_i8_kernel<D, FULL, GP, false>;
   static bool configured = false;
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!configured) {
-      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-      if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode i8: %s", cudaGetErrorString(e));
+      for (auto k : {split_i8_kernel<D, FULL, GP, true>, split_i8_kernel<D, FULL, GP, false>}) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "decode i8: %s", cudaGetErrorString(e));
+      }
       configured = true;
     }
   }

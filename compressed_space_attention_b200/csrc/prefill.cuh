@@ -163,14 +163,22 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+// 16 columns of this warp's 32 TMEM lanes; tc_ld16_nowait leaves the wait
+// (tcgen05.wait::ld) to the caller, so that several loads can be in flight.
+__device__ __forceinline__ void tc_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  tc_ld16_nowait(taddr, r);
+  tc_wait_ld();
 #pragma unroll
   for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
 }
@@ -433,10 +441,15 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
     const ulonglong2 *nv4 = reinterpret_cast<const ulonglong2 *>(nrm_s + kTcTok + HC * half);
     const int c0 = t0 + HC * half;                             // token of this thread's first column
     float x[HC];
+    uint32_t sraw[HC / 16][16];
+#pragma unroll
+    for (int c = 0; c < HC / 16; ++c) tc_ld16_nowait(tmem + (it & 1) * 64 + HC * half + lane_off + 16 * c, sraw[c]);
+    tc_wait_ld();
 #pragma unroll
     for (int c = 0; c < HC / 16; ++c) {
       float v[16];
-      tc_ld16(tmem + (it & 1) * 64 + HC * half + lane_off + 16 * c, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(sraw[c][j]);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const ulonglong2 n = nk4[4 * c + k];
