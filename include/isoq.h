@@ -320,7 +320,10 @@ int isoq_decode_step(const void *q_dev, const void *k_new_dev, const void *v_new
  *              first, e.g. by isoq_quantize into the cache rows).
  * Tensor-core path: d in {128, 256}, bits = 3, Hq/Hkv in {1, 2, 4, 8},
  * variants FULL, FAST and PLANAR; anything else is ISOQ_ERR_UNSUPPORTED.
- * Tq = 0 is a no-op.  No workspace; one launch.
+ * Tq = 0 is a no-op.  No workspace; one launch.  The kernel checks that its
+ * dynamic shared memory starts on a 1024-byte boundary (its d = 128 layout
+ * keeps no room to align it); otherwise it writes nothing and the next
+ * isoq_check_device_error returns ISOQ_ERR_CUDA.
  */
 int isoq_prefill_attention(const void *q_dev, int dtype, const uint8_t *packed_k_dev,
                            const uint8_t *packed_v_dev, const uint16_t *norms_k_dev,
