@@ -2,7 +2,6 @@
 header declares, and its host-only functions (parameter generator, codebook,
 split policy, argument validation) behave as specified.  No device work."""
 
-import ctypes
 
 import numpy as np
 import pytest
