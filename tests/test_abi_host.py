@@ -72,6 +72,33 @@ def test_split_policy_and_workspace():
     assert isoq.isoq_decode_workspace_size(1, 3, 2, 100, 128) == 0  # Hq % Hkv != 0
 
 
+def _wave_model_chunk(B, hkv, tmax):
+    """The split policy restated: the chunk in {4096, ..., 512} minimising
+    the busiest SM's phases of up to 4 CTAs, (k + 0.7)(min(c, Tmax) + 160)
+    each, ties to the larger chunk."""
+    best, best_cost = None, None
+    for c in (4096, 3072, 2048, 1536, 1024, 768, 512):
+        n_ctas = B * hkv * -(-tmax // c)
+        m, cost = -(-n_ctas // 148), 0.0
+        while m > 0:
+            k = min(m, 4)
+            cost += k + 0.7
+            m -= k
+        cost *= min(c, tmax) + 160
+        if best_cost is None or cost < best_cost - 1e-9:
+            best, best_cost = c, cost
+    return best
+
+
+def test_split_policy_matches_its_model():
+    rng = np.random.default_rng(5)
+    for _ in range(300):
+        B, hkv = int(rng.integers(1, 65)), int(rng.choice([1, 2, 4, 8, 16]))
+        tmax = int(rng.integers(1, 300000))
+        n = isoq.isoq_decode_num_splits(B, hkv, tmax, 128)
+        assert n == -(-tmax // _wave_model_chunk(B, hkv, tmax)), (B, hkv, tmax, n)
+
+
 def test_split_policy_wave_model():
     """The chunk is one of 512 .. 4096 tokens; on measured decode shapes it is
     the one the timed chunk sweep found fastest or within 7 % of it (batch 32
