@@ -766,7 +766,9 @@ def run_isoq(args):
         "rotorquant_comparison": comparator,
         "prefill": prefill,
         "decode_sweep": sweep,
-        "gpu_launches": 4 * args.steps,
+        # per step: quantize_kernel, dequantize_kernel, prep_i8_kernel +
+        # split_i8_kernel (isoq_decode_split), combine_kernel
+        "gpu_launches": 5 * args.steps,
         "clocks": sampler.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:
