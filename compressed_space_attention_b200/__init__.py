@@ -21,6 +21,7 @@ from .binding import (  # noqa: F401
     IsoqError,
     isoq_abi_version,
     isoq_check_device_error,
+    isoq_selftest_wait_timeout,
     isoq_decode_append,
     isoq_decode_attention,
     isoq_decode_combine,

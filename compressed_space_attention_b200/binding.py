@@ -58,6 +58,7 @@ SIGNATURES = [
     ("isoq_decode_step", _I, [_P, _P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _P, _P,
                               _F, _P, _P, _SZ, _P]),
     ("isoq_check_device_error", _I, [_P]),
+    ("isoq_selftest_wait_timeout", _I, [ctypes.c_uint64, _P]),
     ("isoq_prefill_attention", _I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _I, _I,
                                     _P, _P, _F, _P, _P]),
     ("isoq_rotor_groups", _I, [_I]),
@@ -439,6 +440,17 @@ def isoq_decode_combine(out, seq_lens, B: int, Hq: int, Hkv: int, Tmax: int, d: 
             _stream(dev, stream))
     _check(st, "isoq_decode_combine")
     return out
+
+
+def isoq_selftest_wait_timeout(limit_ns: int = 50_000_000, stream=None, device=None) -> None:
+    """Launches the failure-path self-test (a device wait on a barrier that
+    nothing arrives at, given up after limit_ns); the next
+    isoq_check_device_error then returns ISOQ_ERR_TIMEOUT."""
+    torch = _torch()
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(lib().isoq_selftest_wait_timeout(int(limit_ns), _stream(dev, stream)),
+               "isoq_selftest_wait_timeout")
 
 
 def isoq_check_device_error(stream=None, device=None) -> int:

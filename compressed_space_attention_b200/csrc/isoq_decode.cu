@@ -455,6 +455,33 @@ void workspace_views(void *ws, int B, int Hq, int n_splits, int d, float **acc, 
   }
 }
 
+// Self-test of the failure path: thread 0 waits on an mbarrier that nothing
+// arrives at, polling it (non-blocking test_wait) the way the pipelines'
+// bounded waits poll theirs, until limit_ns of %globaltimer have passed (or,
+// should the timer stall, 2^24 polls), then records kErrWaitTimeout in the
+// decode error word and returns.  Nothing else is touched.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+    const unsigned long long t0 = globaltimer();
+    bool done = false;
+    for (unsigned it = 0; it < (1u << 24); ++it) {
+      uint32_t ok;
+      asm volatile("{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                   "selp.u32 %0, 1, 0, p;\n\t}"
+                   : "=r"(ok) : "r"(smem_u32(&bar)), "r"(0u) : "memory");
+      if (ok) {
+        done = true;
+        break;
+      }
+      if ((it & 63u) == 63u && globaltimer() - t0 > limit_ns) break;
+    }
+    if (!done) atomicOr(&g_decode_error, kErrWaitTimeout);
+  }
+}
+
 }  // namespace decode
 }  // namespace isoq
 
@@ -549,6 +576,17 @@ int isoq_decode_attention(const void *q_dev, int dtype, const uint8_t *packed_k_
   if (st) return st;
   return isoq_decode_combine(dtype, seq_lens_dev, B, Hq, Hkv, Tmax, d, variant, params_v_dev,
                              out_dev, workspace_dev, workspace_bytes, stream);
+}
+
+int isoq_selftest_wait_timeout(uint64_t limit_ns, isoq_stream_t stream) {
+  clear_error();
+  if (limit_ns == 0 || limit_ns > 1000000000ull)
+    return set_error(ISOQ_ERR_INVALID_ARG, "limit_ns must be in (0, 1e9]");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  decode::wait_selftest_kernel<<<1, 32, 0, st>>>(static_cast<unsigned long long>(limit_ns));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
+  return ISOQ_OK;
 }
 
 __attribute__((visibility("hidden"))) int isoq_detail_take_decode_error(cudaStream_t stream, unsigned *out) {

@@ -376,6 +376,19 @@ int isoq_rotor_dequantize(const uint8_t *codes_dev, const uint16_t *norms_dev, i
  */
 int isoq_check_device_error(isoq_stream_t stream);
 
+/*
+ * Failure-path self-test: launches one thread that waits on a device
+ * mbarrier that nothing arrives at, polling it like the kernels' bounded
+ * waits, for limit_ns nanoseconds of the GPU timer (0 < limit_ns <= 1e9;
+ * at most 2^24 polls should the timer stall), and then records a timeout in
+ * the device error word, exactly as a pipeline wait that gives up does.
+ * The next isoq_check_device_error on `stream` returns ISOQ_ERR_TIMEOUT and
+ * clears the word; the context stays usable.  Returns ISOQ_OK once launched,
+ * ISOQ_ERR_INVALID_ARG for a limit out of range, ISOQ_ERR_CUDA on a launch
+ * failure.  Touches no buffer.
+ */
+int isoq_selftest_wait_timeout(uint64_t limit_ns, isoq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

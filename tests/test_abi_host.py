@@ -231,3 +231,10 @@ def test_append_and_step_validation_happens_on_host():
     # and the append half's own checks
     assert step(k=None) == isoq.ISOQ_ERR_INVALID_ARG
     assert step(bits=1) == isoq.ISOQ_ERR_UNSUPPORTED
+
+
+def test_selftest_limit_is_validated_on_the_host():
+    """Out-of-range limits are rejected before any launch (no GPU needed)."""
+    lib = isoq.lib()
+    assert lib.isoq_selftest_wait_timeout(0, None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert lib.isoq_selftest_wait_timeout(2_000_000_000, None) == isoq.ISOQ_ERR_INVALID_ARG
