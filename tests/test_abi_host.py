@@ -2,7 +2,6 @@
 header declares, and its host-only functions (parameter generator, codebook,
 split policy, argument validation) behave as specified.  No device work."""
 
-
 import numpy as np
 import pytest
 
@@ -238,3 +237,58 @@ def test_selftest_limit_is_validated_on_the_host():
     lib = isoq.lib()
     assert lib.isoq_selftest_wait_timeout(0, None) == isoq.ISOQ_ERR_INVALID_ARG
     assert lib.isoq_selftest_wait_timeout(2_000_000_000, None) == isoq.ISOQ_ERR_INVALID_ARG
+
+
+def test_prefill_validation_happens_on_host():
+    """Every rejected shape or pointer returns before any launch; an empty
+    chunk (Tq = 0) is a no-op (the fake pointers are never touched)."""
+    lib = isoq.lib()
+
+    def call(**kw):
+        a = dict(q=256, dtype=isoq.ISOQ_F16, pk=256, pv=256, nk=256, nv=256, sl=256, B=1, Tq=16,
+                 Hq=8, Hkv=2, Tmax=64, d=128, bits=3, variant=0, prk=256, prv=256, scale=0.088,
+                 out=256)
+        a.update(kw)
+        return lib.isoq_prefill_attention(a["q"], a["dtype"], a["pk"], a["pv"], a["nk"], a["nv"],
+                                          a["sl"], a["B"], a["Tq"], a["Hq"], a["Hkv"], a["Tmax"],
+                                          a["d"], a["bits"], a["variant"], a["prk"], a["prv"],
+                                          a["scale"], a["out"], None)
+
+    assert call(d=512) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(bits=2) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(variant=isoq.ISOQ_SO3) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(dtype=isoq.ISOQ_F32) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(B=0) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(Tq=-1) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(Hq=7) == isoq.ISOQ_ERR_INVALID_ARG                  # Hq % Hkv != 0
+    assert call(Hq=32, Hkv=2) == isoq.ISOQ_ERR_UNSUPPORTED          # G = 16
+    assert call(Hq=6, Hkv=2) == isoq.ISOQ_ERR_UNSUPPORTED           # G = 3
+    assert call(Tmax=60) == isoq.ISOQ_ERR_UNSUPPORTED               # Tmax % 8 != 0
+    assert call(q=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(prv=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(pk=256 + 8) == isoq.ISOQ_ERR_UNSUPPORTED            # misaligned
+    assert call(scale=float("nan")) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(Tq=0) == isoq.ISOQ_OK
+
+
+def test_rotor_validation_happens_on_host():
+    lib = isoq.lib()
+
+    def quant(**kw):
+        a = dict(x=256, dtype=isoq.ISOQ_F16, nh=1, nv=10, d=128, bits=3, hs=1280, vs=128, rot=256,
+                 codes=256, norms=256, ohs=10)
+        a.update(kw)
+        return lib.isoq_rotor_quantize(a["x"], a["dtype"], a["nh"], a["nv"], a["d"], a["bits"], a["hs"],
+                                       a["vs"], a["rot"], a["codes"], a["norms"], a["ohs"], None)
+
+    assert quant(d=96) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert quant(bits=5) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert quant(dtype=9) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert quant(nv=-1) == isoq.ISOQ_ERR_INVALID_ARG
+    assert quant(nv=0) == isoq.ISOQ_OK                                # empty: no launch
+    assert quant(x=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert quant(vs=64) == isoq.ISOQ_ERR_INVALID_ARG                  # rows overlap
+    assert quant(ohs=5) == isoq.ISOQ_ERR_INVALID_ARG                  # output rows overlap
+    assert quant(x=256 + 8) == isoq.ISOQ_ERR_UNSUPPORTED              # misaligned
+    assert isoq.isoq_rotor_groups(128) == 43 and isoq.isoq_rotor_groups(100) < 0
+
