@@ -292,3 +292,33 @@ def test_rotor_validation_happens_on_host():
     assert quant(x=256 + 8) == isoq.ISOQ_ERR_UNSUPPORTED              # misaligned
     assert isoq.isoq_rotor_groups(128) == 43 and isoq.isoq_rotor_groups(100) < 0
 
+
+
+@pytest.mark.parametrize("fn", ["isoq_dequantize", "isoq_rotor_dequantize"])
+def test_dequantize_validation_happens_on_host(fn):
+    lib = isoq.lib()
+    rotor = fn == "isoq_rotor_dequantize"
+
+    def call(**kw):
+        a = dict(codes=256, norms=256, nh=1, nv=10, d=128, bits=3, variant=isoq.ISOQ_FULL, ihs=10,
+                 par=256, out=256, dtype=isoq.ISOQ_F16, hs=1280, vs=128)
+        a.update(kw)
+        if rotor:
+            return lib.isoq_rotor_dequantize(a["codes"], a["norms"], a["nh"], a["nv"], a["d"], a["bits"],
+                                             a["ihs"], a["par"], a["out"], a["dtype"], a["hs"], a["vs"], None)
+        return lib.isoq_dequantize(a["codes"], a["norms"], a["nh"], a["nv"], a["d"], a["bits"],
+                                   a["variant"], a["ihs"], a["par"], a["out"], a["dtype"], a["hs"],
+                                   a["vs"], None)
+
+    assert call(d=64) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(bits=1) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(dtype=5) == isoq.ISOQ_ERR_UNSUPPORTED
+    if not rotor:
+        assert call(variant=9) == isoq.ISOQ_ERR_UNSUPPORTED
+    assert call(nv=-1) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(nv=0) == isoq.ISOQ_OK                                 # empty: no launch
+    assert call(out=None) == isoq.ISOQ_ERR_INVALID_ARG
+    assert call(ihs=5) == isoq.ISOQ_ERR_INVALID_ARG                   # input rows overlap
+    assert call(vs=64) == isoq.ISOQ_ERR_INVALID_ARG                   # output rows overlap
+    assert call(out=256 + 4) == isoq.ISOQ_ERR_UNSUPPORTED             # misaligned
+    assert call(vs=132) == isoq.ISOQ_ERR_UNSUPPORTED                  # 264-byte rows
