@@ -92,27 +92,45 @@ def f16_half_ulp(v):
     return 2.0 ** (e - 11)
 
 
-def check_attention(gpu_out, oracle_out, dtype):
+def check_attention(gpu_out, oracle_out, dtype, label=None):
     """Asserts the attention output is within the stated max-abs tolerance.
 
-    float16 outputs: 2e-3 max-abs in units of the output row's own scale,
-    max(1, max_i |o_i|) per (b, qh) row.  The outputs of the outlier-heavy
-    K/V workloads reach |o| ~ 30, where a float16 value's own spacing is
-    0.03; an absolute 2e-3 bar would sit below the output format's
-    resolution, so rows larger than 1 are measured relative to their maximum.
+    float16 outputs: |err| <= 2e-3 + half a float16 ulp of the oracle's value,
+    per element (the stated 2e-3 max-abs plus the output format's own
+    rounding, which matters only where |o| > 4).
     float32 outputs: 1e-5 max-abs.
+
+    Returns the largest absolute error.  When ISOQ_ATTENTION_LOG names a
+    file, one JSON line per call is appended to it with the largest absolute
+    error, the largest |o| and the smallest margin to the bar, so that a test
+    run records how close each case came.
     """
     g = np.asarray(gpu_out, dtype=np.float64)
     o = np.asarray(oracle_out, dtype=np.float64)
     err = np.abs(g - o)
     if dtype == np.float16:
-        scale = np.maximum(1.0, np.max(np.abs(o), axis=-1, keepdims=True)) if o.ndim else max(1.0, abs(o))
-        tol = ATT_F16 * scale
+        tol = ATT_F16 + f16_half_ulp(o)
     else:
-        tol = ATT_F32
+        tol = ATT_F32 + 0.0 * o
+    _record_attention(label, dtype, err, o, tol)
     worst = float(np.max(err - tol)) if err.size else 0.0
     assert np.all(err <= tol), f"attention error exceeds tolerance by {worst:.3g} (max err {err.max():.3g})"
     return float(err.max()) if err.size else 0.0
+
+
+def _record_attention(label, dtype, err, o, tol):
+    path = os.environ.get("ISOQ_ATTENTION_LOG")
+    if not path or not err.size:
+        return
+    import json
+    if label is None:
+        label = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    rec = {"case": label, "dtype": "f16" if dtype == np.float16 else "f32",
+           "max_abs_err": float(err.max()), "max_abs_o": float(np.abs(o).max()),
+           "min_margin": float(np.min(tol - err)),
+           "max_err_where_abs_o_le_1": float(err[np.abs(o) <= 1].max()) if np.any(np.abs(o) <= 1) else None}
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
 
 
 def scale_for(d):

@@ -90,9 +90,11 @@ def test_prefill_long_context_sampled():
         pos = tmax - tq + t
         ref = O.decode_attention(q[:, t], pk_h, pv_h, nk_h, nv_h, [pos + 1], prk, prv, 3, O.FULL, 1 / math.sqrt(d))
         check_attention(got[:, t], ref, np.float16)
+    # the last query sees the whole cache: the decode kernel on the same
+    # cache meets the same bar against the same oracle row
     dec = isoq.isoq_decode_attention(_t(q[:, -1]), pk, pv, nk, nv, _t(lens), _t(prk), _t(prv), bits=3,
                                      variant=isoq.ISOQ_FULL).cpu().numpy()
-    assert np.max(np.abs(dec.astype(np.float64) - got[:, -1].astype(np.float64))) < 4e-3 * max(1.0, np.abs(dec).max())
+    check_attention(dec, ref, np.float16)
 
 
 def test_prefill_host_validation():
