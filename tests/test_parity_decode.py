@@ -109,10 +109,11 @@ def test_long_context_shape_small():
 
 def test_long_context_full_size_sampled():
     """The benchmark's launch: batch 32 x 65,536 tokens, d=256, GQA 16/8.
-    K/V are drawn on the device and compressed by the CUDA path; two sampled
-    (b, kvh) rows are also compressed by the oracle (codes compared), their
-    oracle codes are written into the cache, and the decode outputs of those
-    rows' query heads are compared with the oracle."""
+    K/V are drawn on the device and compressed by the CUDA path; 16 sampled
+    (b, kvh) rows (the four corners of the grid and 12 seeded others) are
+    also compressed by the oracle (codes compared), their oracle codes are
+    written into the cache, and the decode outputs of those rows' query
+    heads are compared with the oracle."""
     b, hkv, hq, t, d = 32, 8, 16, 65536, 256
     torch.cuda.empty_cache()
     k, v = synth.student_t_kv_torch(b, hkv, t, d, seed=9, device=DEV)
@@ -122,7 +123,9 @@ def test_long_context_full_size_sampled():
     pv, nv = isoq.isoq_quantize(v.view(b * hkv, t, d), _t(np.tile(prv, (b, 1, 1))), 3, O.FULL)
     pk, pv = pk.view(b, hkv, t, 96), pv.view(b, hkv, t, 96)
     nk, nv = nk.view(b, hkv, t), nv.view(b, hkv, t)
-    samples = [(3, 5), (30, 0)]
+    pick = synth.rng(90).choice(b * hkv, size=16, replace=False)
+    samples = [(0, 0), (0, hkv - 1), (b - 1, 0), (b - 1, hkv - 1)]
+    samples += [(int(i) // hkv, int(i) % hkv) for i in pick if (int(i) // hkv, int(i) % hkv) not in samples][:12]
     rows = {}
     for (bb, kvh) in samples:
         for name, x, codes, norms, par in (("k", k, pk, nk, prk), ("v", v, pv, nv, prv)):
