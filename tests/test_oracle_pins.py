@@ -130,6 +130,50 @@ def _block_matrix(ql, qr, variant):
     return np.stack(cols, axis=1)
 
 
+def _left_matrix(q):
+    """q (x) v as a matrix acting on v = (w, x, y, z), rows typed out from
+    Hamilton's rules (RotaryQuant Appendix B; IsoQuant abstract)."""
+    w, x, y, z = q
+    return np.array([[w, -x, -y, -z],
+                     [x, w, -z, y],
+                     [y, z, w, -x],
+                     [z, -y, x, w]])
+
+
+def _right_matrix(p):
+    """v (x) p as a matrix acting on v, rows typed out from Hamilton's rules."""
+    w, x, y, z = p
+    return np.array([[w, -x, -y, -z],
+                     [x, w, z, -y],
+                     [y, -z, w, x],
+                     [z, y, -x, w]])
+
+
+@pytest.mark.parametrize("variant", [O.FULL, O.FAST, O.BLOCK_SO4, O.SO3])
+def test_block_maps_equal_explicit_4x4_matrices(variant):
+    """RotaryQuant §3.3 / Appendix B: T(v) = q_L v conj(q_R) is the 4x4 matrix
+    L(q_L) R(conj q_R) (Full, and the no-WHT block map; v1 repeats q_L in the
+    right slot), and IsoQuant-Fast keeps L(q_L) alone.  The matrices are typed
+    out independently of the oracle's Hamilton product; the inverse map is
+    their transpose.  Checked on random inputs, including non-unit
+    quaternions (the identities are algebraic)."""
+    g = np.random.default_rng(11)
+    for trial in range(40):
+        ql, qr = g.standard_normal((2, 4))
+        if trial % 2 == 0:
+            ql, qr = ql / np.linalg.norm(ql), qr / np.linalg.norm(qr)
+        if variant == O.SO3:
+            qr = ql
+        conj_qr = qr * np.array([1.0, -1.0, -1.0, -1.0])
+        m = _left_matrix(ql) if variant == O.FAST else _left_matrix(ql) @ _right_matrix(conj_qr)
+        v = g.standard_normal((7, 4))
+        fwd = O.so4_forward(v[:, None, :], ql[None, :], qr[None, :], variant)[:, 0]
+        scale = np.max(np.abs(v)) * np.sum(ql * ql) * max(1.0, np.sum(qr * qr))
+        np.testing.assert_allclose(fwd, v @ m.T, rtol=0, atol=4e-15 * scale)
+        inv = O.so4_inverse(v[:, None, :], ql[None, :], qr[None, :], variant)[:, 0]
+        np.testing.assert_allclose(inv, v @ m, rtol=0, atol=4e-15 * scale)
+
+
 def _complex_line(g, n):
     a = g.standard_normal((n, 2))
     a /= np.linalg.norm(a, axis=1, keepdims=True)
