@@ -738,23 +738,56 @@ constexpr size_t kStaticWorkspaceBytes = size_t(16) << 20;  // 16 MiB per device
 
 static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
+// Identifier of the CUDA context current on this thread (0 if none or if the
+// driver does not offer the query).  Context ids are unique for the life of
+// the process, so a context created after a device reset gets a new one.
+unsigned long long current_context_id() {
+  using CtxGetCurrentFn = int (*)(void **);
+  using CtxGetIdFn = int (*)(void *, unsigned long long *);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  void *ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+  return id;
+}
+
 // Device address of g_static_workspace on the current device.  Host code
 // sees only a host-side stand-in for the array, so the device address is
-// looked up once per device, with that device current, and cached.
+// looked up with that device current and cached per device, together with
+// the id of the context it belongs to: after a device reset the runtime
+// makes a new context, in which the array has a new address, and the first
+// call there looks it up again.
 int static_workspace_address(void **out) {
   static std::mutex mu;
   static void *addr[256] = {nullptr};
+  static unsigned long long ctx_of[256] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= 256) return set_error(ISOQ_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!addr[dev] || ctx != ctx_of[dev]) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_workspace);
     if (e != cudaSuccess || !p)
       return set_error(ISOQ_ERR_CUDA, "cudaGetSymbolAddress(static workspace): %s", cudaGetErrorString(e));
     addr[dev] = p;
+    // the lookup may have created the context: take its id now
+    ctx_of[dev] = current_context_id();
   }
   *out = addr[dev];
   return ISOQ_OK;

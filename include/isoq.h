@@ -252,8 +252,12 @@ int isoq_decode_combine(int dtype, const int32_t *seq_lens_dev, int B, int Hq, i
  *   - Shapes whose workspace (isoq_decode_workspace_size) exceeds the array
  *     are rejected with ISOQ_ERR_UNSUPPORTED before any launch.
  *   - The first call on a device looks up the array's device address with
- *     cudaGetSymbolAddress and caches it; make that first call before any
- *     stream capture on that device.
+ *     cudaGetSymbolAddress and caches it, with the id of the CUDA context it
+ *     belongs to; make that first call before any stream capture on that
+ *     device.  A device reset (cudaDeviceReset) ends that context, and the
+ *     array's contents with it: the first call in the new context notices
+ *     the new context id and looks the address up again, so that call too
+ *     belongs before any capture.
  *   - All calls share the one array and it keeps the last call's contents
  *     (nothing in it needs clearing: each call writes every slot it reads).
  *     Calls whose kernels overlap on the GPU, e.g. on two streams without an

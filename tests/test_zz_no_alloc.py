@@ -4,9 +4,10 @@ owned by another framework's allocator, or a plugin handed only its inputs
 and outputs).  Its split-K scratch is a fixed array inside the library.
 
 The test calls the entry point through the C ABI with raw device pointers,
-twice in a row on different inputs, and checks each output against the
-regular isoq_decode_attention (caller-provided workspace) on the same input,
-within the attention tolerance of the parity tests.  This file is named so
+several times in a row on different inputs (the last one with lengths that
+leave most splits empty, right after a long call), and checks each output
+against the regular isoq_decode_attention (caller-provided workspace) on the
+same input, within the attention tolerance of the parity tests.  This file is named so
 that pytest collects it last.
 """
 
@@ -56,15 +57,25 @@ def _static_call(c, out, dtype_code):
 
 
 def test_static_workspace_matches_allocating_entry_point_twice():
-    cases = [(_case(11, 4, 16, 8, 4096, 256, np.float16), isoq.ISOQ_F16, np.float16),
-             (_case(12, 3, 8, 2, 1000, 128, np.float32), isoq.ISOQ_F32, np.float32)]
+    long_case = _case(11, 4, 16, 8, 4096, 256, np.float16)
+    # the same shapes with lengths that leave most splits empty, right after
+    # the long call filled the array with partial states
+    short_case = dict(long_case, lens=torch.tensor([1, 37, 0, 300], dtype=torch.int32, device=DEV))
+    cases = [(long_case, isoq.ISOQ_F16, np.float16),
+             (_case(12, 3, 8, 2, 1000, 128, np.float32), isoq.ISOQ_F32, np.float32),
+             (long_case, isoq.ISOQ_F16, np.float16),
+             (short_case, isoq.ISOQ_F16, np.float16)]
     for c, code, dt in cases:
         b, hq, hkv, tmax, d = c["shape"]
         ref = isoq.isoq_decode_attention(c["q"], c["pk"], c["pv"], c["nk"], c["nv"], c["lens"],
                                          c["prk"], c["prv"], 3, isoq.ISOQ_FULL)
         out = torch.empty_like(ref)
+        torch.cuda.synchronize()
+        before = (torch.cuda.memory_allocated(), torch.cuda.memory_reserved())
         assert _static_call(c, out, code) == isoq.ISOQ_OK, isoq.last_error()
         torch.cuda.synchronize()
+        # nothing went through torch's allocator either
+        assert (torch.cuda.memory_allocated(), torch.cuda.memory_reserved()) == before
         check_attention(out.cpu().numpy(), ref.cpu().numpy(), dt)
     assert isoq.isoq_check_device_error() == 0
 
