@@ -28,6 +28,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "tcgen05.cuh"
 #include "decode.h"
 #include "internal.h"
 

@@ -53,6 +53,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "tcgen05.cuh"
 #include "internal.h"
 
 namespace isoq {

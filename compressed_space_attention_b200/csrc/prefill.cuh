@@ -16,20 +16,29 @@
 // in halves.  Per 64-token tile j, software-pipelined by one product:
 //   the packed codes and norms of the next tiles are loaded into registers
 //   one phase ahead; the CTA expands K tile j + 1's codes into float16
-//   centroids alpha c_k (alpha, searched on the host, makes them nearly
-//   exact in float16) in a 128B-swizzled tile, and one thread issues
-//   S(j + 1) = Q~hi K~^T + Q~lo K~^T (tcgen05.mma kind::f16, M = 128,
-//   N = 64; q~ split into float16 hi and lo parts keeps 22-bit scores) into
+//   centroids alpha c_k in a 128B-swizzled tile, and their float16
+//   residuals alpha c_k - fp16(alpha c_k) into a second tile (alpha is
+//   searched on the host; the residuals are below 2^-15 of the centroids,
+//   so hi + lo keeps them to about 2^-26), and one thread issues
+//   S(j + 1) = Q~hi K~hi^T + Q~lo K~hi^T + Q~hi K~lo^T (tcgen05.mma
+//   kind::f16, M = 128, N = 64; q~ split into float16 hi and lo parts) into
 //   the other of two TMEM S buffers, so it runs under the softmax of tile j;
 //   each thread reads its half row of S(j) (tcgen05.ld), scales it by
 //   s^K scale / alpha, masks it on diagonal tiles, exchanges its half-row
-//   maximum with the partner warp, writes p s^V as float16 (11 bits of each
-//   weight's own magnitude) into a K-major P tile and, when its warp's
-//   maximum moved, rescales its half of the O row in TMEM; the CTA expands
-//   V tile j into its own tile buffer and one thread issues O += P V~
-//   (N = d, V~ read MN-major from the token-row tile).
-// d = 128 keeps one P tile and fits two CTAs per SM (one CTA's thread work
-// runs under the other's products); d = 256 keeps two P tiles, one CTA.
+//   maximum with the partner warp through the consumed S buffer, writes
+//   P = p s^V as float16 hi and lo parts (22 bits of each weight) over that
+//   S buffer in TMEM and, when its warp's maximum moved, rescales its half
+//   of the O row in TMEM; the CTA expands V tile j into its own tile buffer
+//   and one thread issues O += P_hi V~ + P_lo V~ (A = P from tensor memory,
+//   N = d, V~ read MN-major from the token-row tile).  The next product into
+//   that S buffer (QK of tile j + 2) is issued after the PV product, and the
+//   tensor core runs one CTA's products in issue order.
+// Both the hi/lo query and the hi/lo centroid residual are needed for the
+// float16 output bar on outlier-heavy K/V: float16 centroids alone (relative
+// error 1.9e-5) or float16 weights alone (2^-12) move scores or weights
+// enough to shift outputs of magnitude 30-80 by several 1e-3.
+// d = 128 fits two CTAs per SM (one CTA's thread work runs under the
+// other's products); d = 256 one.
 // The epilogue reads O from TMEM, normalises, rotates back (R_V^T) in shared
 // memory and stores float16.
 // Operand tiles use the canonical SW128 layouts: rows of 128 bytes (64
@@ -60,6 +69,7 @@ struct PrefillArgs {
   float score_unit;               // scale * log2(e) / (alpha sqrt(d))
   float out_unit;                 // 1 / (alpha * d)
   uint32_t lut_lo0, lut_lo1, lut_hi0, lut_hi1;   // float16 alpha c_k, low / high bytes
+  uint32_t res_lo0, res_lo1, res_hi0, res_hi1;   // float16 alpha c_k - fp16(alpha c_k), low / high bytes
 };
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -105,18 +115,13 @@ struct TcCfg {
   static constexpr int PB = D * 3 / 8;
   static constexpr int ITEMS = kTcTok * (D / 32) / kTcThreads;   // 32-code groups per thread per tile
   static constexpr int Q_BYTES = kTcRows * D * 2;         // one of hi / lo
-  static constexpr int KV_BYTES = kTcTok * D * 2;         // one K or V tile
-  static constexpr int P_BYTES = kTcRows * kTcTok * 2;    // one P tile
-  // d = 256: two P tiles, so PV(j - 1) (twice the work of d = 128's) runs on
-  // under the softmax of tile j; d = 128 has one, waits for PV(j - 1) before
-  // writing P(j) and fits two CTAs per SM instead.
-  static constexpr int P_BUFS = D == 128 ? 1 : 2;
+  static constexpr int KV_BYTES = kTcTok * D * 2;         // one K, K-residual or V tile
   static constexpr int NORM_BYTES = 2 * kTcTok * 4;       // s^K score_unit, s^V of one tile
   static constexpr int OFF_QLO = Q_BYTES;
   static constexpr int OFF_K = 2 * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KV_BYTES;
-  static constexpr int OFF_P = OFF_V + KV_BYTES;
-  static constexpr int OFF_NORM = OFF_P + P_BUFS * P_BYTES;
+  static constexpr int OFF_KLO = OFF_K + KV_BYTES;
+  static constexpr int OFF_V = OFF_KLO + KV_BYTES;
+  static constexpr int OFF_NORM = OFF_V + KV_BYTES;
   static constexpr int OFF_BAR = OFF_NORM + NORM_BYTES;
   // Two CTAs per SM at d = 128 (the second CTA's softmax and expansion run
   // under the first one's products).  Their layout leaves no room to align
@@ -126,74 +131,10 @@ struct TcCfg {
   static constexpr int SLACK = MIN_BLOCKS == 2 ? 0 : 1024;
   static constexpr int SMEM = OFF_BAR + 8 * 3 + 8 + SLACK;
   static constexpr int TMEM_COLS = D == 128 ? 256 : 512;     // S (2 x 64) + O (D), rounded to a power of 2
-  static_assert(32 * D * 4 <= 2 * KV_BYTES, "prep scratch (32 rows) fits the K and V tiles");
+  static_assert(32 * D * 4 <= 2 * KV_BYTES, "prep scratch (32 rows) fits the K and K-residual tiles");
   static_assert(MIN_BLOCKS * (SMEM + 1024) <= 233472, "shared memory per SM (1 KB reserved per CTA)");
   static_assert(MIN_BLOCKS * TMEM_COLS <= 512, "tensor memory columns");
 };
-
-__host__ __device__ __forceinline__ uint32_t tc_off(int r, int e, int blk_stride) {
-  return static_cast<uint32_t>((e >> 6) * blk_stride + (r >> 3) * 1024 + (r & 7) * 128 +
-                               ((((e & 63) >> 3) ^ (r & 7)) << 4) + (e & 7) * 2);
-}
-
-__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// kind::f16 instruction descriptor: D float32, A and B float16, A K-major,
-// B K-major (b_mn = 0) or MN-major (1), M x N.
-__host__ __device__ constexpr uint32_t tc_idesc(int M, int N, int b_mn) {
-  return (1u << 4) | (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
-      ::"r"(tmem_d), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0));
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// 16 columns of this warp's 32 TMEM lanes; tc_ld16_nowait leaves the wait
-// (tcgen05.wait::ld) to the caller, so that several loads can be in flight.
-__device__ __forceinline__ void tc_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  tc_ld16_nowait(taddr, r);
-  tc_wait_ld();
-#pragma unroll
-  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-__device__ __forceinline__ void tc_st16(uint32_t taddr, const float (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-        "r"(__float_as_uint(v[15]))
-      : "memory");
-}
 
 // Packed codes of one tile, this thread's share (ITEMS 32-code groups),
 // loaded from global memory one phase before they are expanded.
@@ -221,9 +162,11 @@ __device__ __forceinline__ void tc_fetch(TcCodes<D> &c, const uint8_t *base, int
 
 // Fetched codes -> float16 centroids alpha c_k in the SW128 token-row tile
 // (64-dim blocks kTcTok * 128 bytes apart); the same layout serves K (K-major
-// B of QK) and V (MN-major B of PV).
-template <int D>
-__device__ __forceinline__ void tc_expand(const TcCodes<D> &c, unsigned char *tile, const PrefillArgs &a, int tid) {
+// B of QK) and V (MN-major B of PV).  With RES, the float16 residuals
+// alpha c_k - fp16(alpha c_k) go to a second tile of the same layout.
+template <int D, bool RES>
+__device__ __forceinline__ void tc_expand(const TcCodes<D> &c, unsigned char *tile, unsigned char *tile_res,
+                                          const PrefillArgs &a, int tid) {
   constexpr int GROUPS = D / 32, BLK = kTcTok * 128;
 #pragma unroll
   for (int k = 0; k < TcCfg<D>::ITEMS; ++k) {
@@ -232,18 +175,28 @@ __device__ __forceinline__ void tc_expand(const TcCodes<D> &c, unsigned char *ti
     group_sel8(c.w[k][0], c.w[k][1], c.w[k][2], s);
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      uint32_t v[4];
+      uint32_t v[4], r[4];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const uint32_t lo = prmt(a.lut_lo0, a.lut_lo1, s[2 * m + u]);
         const uint32_t hi = prmt(a.lut_hi0, a.lut_hi1, s[2 * m + u]);
         v[2 * u] = prmt(lo, hi, 0x5140u);
         v[2 * u + 1] = prmt(lo, hi, 0x7362u);
+        if constexpr (RES) {
+          const uint32_t rlo = prmt(a.res_lo0, a.res_lo1, s[2 * m + u]);
+          const uint32_t rhi = prmt(a.res_hi0, a.res_hi1, s[2 * m + u]);
+          r[2 * u] = prmt(rlo, rhi, 0x5140u);
+          r[2 * u + 1] = prmt(rlo, rhi, 0x7362u);
+        }
       }
       // dims 32 grp + 8 m .. + 7, as two 8-byte stores (measured faster
       // here than one 16-byte store, despite the latter's fewer bank conflicts)
       *reinterpret_cast<uint2 *>(tile + tc_off(tok, 32 * grp + 8 * m, BLK)) = make_uint2(v[0], v[1]);
       *reinterpret_cast<uint2 *>(tile + tc_off(tok, 32 * grp + 8 * m + 4, BLK)) = make_uint2(v[2], v[3]);
+      if constexpr (RES) {
+        *reinterpret_cast<uint2 *>(tile_res + tc_off(tok, 32 * grp + 8 * m, BLK)) = make_uint2(r[0], r[1]);
+        *reinterpret_cast<uint2 *>(tile_res + tc_off(tok, 32 * grp + 8 * m + 4, BLK)) = make_uint2(r[2], r[3]);
+      }
     }
   }
 }
@@ -263,7 +216,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   }
   unsigned char *smem = smem_raw + pad;
   unsigned char *q_hi = smem, *q_lo = smem + C::OFF_QLO;
-  unsigned char *kt = smem + C::OFF_K, *vt = smem + C::OFF_V, *pt = smem + C::OFF_P;
+  unsigned char *kt = smem + C::OFF_K, *klt = smem + C::OFF_KLO, *vt = smem + C::OFF_V;
   float *nrm_s = reinterpret_cast<float *>(smem + C::OFF_NORM);   // [2][kTcTok] s^K score_unit, s^V of the tile in the softmax
   uint64_t *bar_s = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);   // [2]: S buffer b's product done
   uint64_t *bar_o = bar_s + 2;                                          // PV product done
@@ -271,7 +224,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   // A product wait that gave up in iteration j sets fail_s[j % 2]; it is read
   // after the iteration's last block barrier (see the loop).
   volatile uint8_t *fail_s = reinterpret_cast<volatile uint8_t *>(tmem_slot + 1);
-  float *scratch = reinterpret_cast<float *>(kt);   // 32 rows x D floats over the K and V tiles (prep, epilogue)
+  float *scratch = reinterpret_cast<float *>(kt);   // 32 rows x D floats over the K tiles (prep, epilogue)
 
   const int qt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -363,8 +316,8 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
   // handles column half w / 4 of those rows' S and O.
   const int sub = warp & 3, half = warp >> 2, lane = tid & 31;
   const uint32_t lane_off = static_cast<uint32_t>(32 * sub) << 16;
-  const uint32_t qh_s = smem_u32(q_hi), ql_s = smem_u32(q_lo), k_s = smem_u32(kt), v_s = smem_u32(vt),
-                 p_s = smem_u32(pt);
+  const uint32_t qh_s = smem_u32(q_hi), ql_s = smem_u32(q_lo), k_s = smem_u32(kt), kl_s = smem_u32(klt),
+                 v_s = smem_u32(vt);
 
   // Expands K tile j (codes and norms from the registers), then issues its QK
   // product into S buffer j % 2.  The caller has made sure the K tile and
@@ -373,7 +326,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
     if (tid < 2 * kTcTok) nrm_s[tid] = __half2float(__ushort_as_half(nrm)) * (tid < kTcTok ? a.score_unit : 1.f);
   };
   auto stage_qk = [&](int j) {
-    tc_expand<D>(kc, kt, a, tid);
+    tc_expand<D, true>(kc, kt, klt, a, tid);
     if (j + 1 < n_tiles) tc_fetch<D>(kc, kb, (j + 1) * kTcTok, tend, tid);
     fence_proxy_async_smem();
     tc_fence_before();
@@ -385,9 +338,10 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t ko = (ks >> 2) * KBLK + (ks & 3) * 32, qo = (ks >> 2) * QBLK + (ks & 3) * 32;
-        const uint64_t bd = tc_desc(k_s + ko, 16, 1024);
-        tc_mma(t_s, tc_desc(qh_s + qo, 16, 1024), bd, idesc, ks > 0 ? 1u : 0u);
+        const uint64_t bd = tc_desc(k_s + ko, 16, 1024), ad = tc_desc(qh_s + qo, 16, 1024);
+        tc_mma(t_s, ad, bd, idesc, ks > 0 ? 1u : 0u);
         tc_mma(t_s, tc_desc(ql_s + qo, 16, 1024), bd, idesc, 1u);
+        tc_mma(t_s, ad, tc_desc(kl_s + ko, 16, 1024), idesc, 1u);
       }
       tc_commit(&bar_s[j & 1]);
     }
@@ -467,7 +421,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
     for (int j = 0; j < HC; ++j) tmx = fmaxf(tmx, x[j]);
 
     // PV(it - 1) must be complete before O is rescaled and the V tile
-    // reused; with one P tile, already before P(it) is written.
+    // reused (P(it) goes to the other S buffer, which PV(it - 1) does not read).
     auto wait_pv = [&]() {
       if (o_issued > o_done) {
         if (mbar_wait_bounded(bar_o, o_done & 1))
@@ -477,15 +431,20 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
         tc_fence_after();
       }
     };
-    if (C::P_BUFS == 1) wait_pv();
-    unsigned char *pb = pt + (it % C::P_BUFS) * C::P_BYTES;   // free: PV(it - P_BUFS) is complete
     // The row maximum over both column halves, exchanged with the partner
-    // warp through the free P tile: each thread leaves its value in the
-    // partner's part of row r and reads the partner's from its own part,
-    // which only it overwrites afterwards.
-    *reinterpret_cast<float *>(pb + tc_off(r, HC * (half ^ 1), 0)) = tmx;
+    // warp through the consumed S buffer: each thread leaves its value in a
+    // column of its own half of S (already read) that the partner overwrites
+    // with its P later, and reads the partner's from a column that it
+    // overwrites itself later.  Half 0 reads S columns 0..31 and writes P
+    // into 0..15 and 32..47; half 1 reads 32..63 and writes 16..31, 48..63.
+    const uint32_t s_col = tmem + (it & 1) * 64 + lane_off;
+    tc_st1(s_col + 16 + 16 * half, __float_as_uint(tmx));
+    tc_wait_st();
+    tc_fence_before();
     named_barrier(1 + sub, 64);
-    tmx = fmaxf(tmx, *reinterpret_cast<const float *>(pb + tc_off(r, HC * half, 0)));
+    tc_fence_after();
+    tmx = fmaxf(tmx, __uint_as_float(tc_ld1(s_col + 16 + 16 * (half ^ 1))));
+    tc_wait_ld();
     const float nm = fmaxf(mx, tmx);
     const float base = nm == -INFINITY ? 0.f : nm;
     const float f = ex2f(mx - base);                            // 0 while mx = -inf
@@ -493,9 +452,11 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
     mx = nm;
     const uint64_t base2 = f2_pack(base, base);
     l2 = f2_mul(l2, f2_pack(f, f));
+    // P = p s^V as float16 hi and lo parts: tokens 2i, 2i + 1 of the tile in
+    // column i of the hi block (columns 0..31) and of the lo block (32..63).
+    uint32_t phi[HC / 2], plo[HC / 2];
 #pragma unroll
     for (int c = 0; c < HC / 8; ++c) {
-      uint32_t w[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int j = 8 * c + 2 * k;
@@ -505,11 +466,16 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
         l2 = f2_add(l2, p2);
         const ulonglong2 n = nv4[j >> 2];
         f2_unpack(f2_mul(p2, (k & 1) ? n.y : n.x), p0, p1);
-        w[k] = pack_f16x2(p0, p1);
+        const __half2 h = __floats2half2_rn(p0, p1);
+        const float2 hf = __half22float2(h);
+        phi[4 * c + k] = *reinterpret_cast<const uint32_t *>(&h);
+        plo[4 * c + k] = pack_f16x2(p0 - hf.x, p1 - hf.y);
       }
-      *reinterpret_cast<uint4 *>(pb + tc_off(r, HC * half + 8 * c, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    if (C::P_BUFS == 2) wait_pv();
+    tc_st16u(s_col + 16 * half, phi);
+    tc_st16u(s_col + 32 + 16 * half, plo);
+    tc_wait_st();
+    wait_pv();
 
     if (moved && it > 0) {
 #pragma unroll 1
@@ -523,7 +489,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
-    tc_expand<D>(vc, vt, a, tid);
+    tc_expand<D, false>(vc, vt, nullptr, a, tid);
     if (it + 1 < n_tiles) tc_fetch<D>(vc, vb, (it + 1) * kTcTok, tend, tid);
     fence_proxy_async_smem();
     tc_fence_before();
@@ -540,11 +506,13 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
     }
     if (tid == 0) {
       constexpr uint32_t idesc = tc_idesc(kTcRows, D, 1);
-      const uint32_t pbs = p_s + (it % C::P_BUFS) * C::P_BYTES;
+      const uint32_t pa = tmem + (it & 1) * 64;               // P(it): hi in columns 0..31, lo in 32..63
 #pragma unroll
-      for (int ks = 0; ks < kTcTok / 16; ++ks)
-        tc_mma(t_o, tc_desc(pbs + ks * 32, 16, 1024), tc_desc(v_s + ks * 2048, KBLK, 1024), idesc,
-               (it > 0 || ks > 0) ? 1u : 0u);
+      for (int ks = 0; ks < kTcTok / 16; ++ks) {
+        const uint64_t bd = tc_desc(v_s + ks * 2048, KBLK, 1024);
+        tc_mma_ts(t_o, pa + 8 * ks, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+        tc_mma_ts(t_o, pa + 32 + 8 * ks, bd, idesc, 1u);
+      }
       tc_commit(bar_o);
     }
     ++o_issued;
@@ -568,7 +536,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::MIN_BLOCKS) prefill_tc_k
     // ---- epilogue, 32 rows per pass: O / l from TMEM, rotate back, store ----
     tc_fence_after();
     __syncthreads();
-    float *xchg = reinterpret_cast<float *>(pt);   // [2][kTcRows] row sums; the P tile is free
+    float *xchg = reinterpret_cast<float *>(q_hi);   // [2][kTcRows] row sums; the query tiles are free
     float l0, l1;
     f2_unpack(l2, l0, l1);
     const float l = l0 + l1;
@@ -642,10 +610,13 @@ inline uint16_t pf_half_bits(double v) {
 }
 
 // alpha in [1, 2) minimising the largest relative float16 rounding error of
-// alpha c_k over the unit-variance 3-bit centroids (searched once).
+// alpha c_k over the unit-variance 3-bit centroids (searched once), the
+// float16 tables of alpha c_k and of its residual alpha c_k - fp16(alpha c_k)
+// (below 2^-15 of the centroid; subnormal float16 values where small).
 struct PfTables {
   double alpha;
   uint32_t lo0, lo1, hi0, hi1;
+  uint32_t rlo0, rlo1, rhi0, rhi1;
 };
 
 inline const PfTables &pf_tables() {
@@ -671,11 +642,17 @@ inline const PfTables &pf_tables() {
     }
     tb.alpha = best;
     tb.lo0 = tb.lo1 = tb.hi0 = tb.hi1 = 0;
+    tb.rlo0 = tb.rlo1 = tb.rhi0 = tb.rhi1 = 0;
     for (int k = 0; k < 8; ++k) {
-      const uint16_t hb = pf_half_bits(best * c[k]);
+      const double v = best * c[k];
+      const uint16_t hb = pf_half_bits(v);
+      const double vh = static_cast<double>(__half2float(*reinterpret_cast<const __half *>(&hb)));
+      const uint16_t rb = pf_half_bits(v - vh);
       const int sh = 8 * (k % 4);
       (k < 4 ? tb.lo0 : tb.lo1) |= static_cast<uint32_t>(hb & 0xFFu) << sh;
       (k < 4 ? tb.hi0 : tb.hi1) |= static_cast<uint32_t>(hb >> 8) << sh;
+      (k < 4 ? tb.rlo0 : tb.rlo1) |= static_cast<uint32_t>(rb & 0xFFu) << sh;
+      (k < 4 ? tb.rhi0 : tb.rhi1) |= static_cast<uint32_t>(rb >> 8) << sh;
     }
   });
   return tb;
@@ -704,6 +681,10 @@ int run_prefill(int d, int variant, PrefillArgs a, cudaStream_t st) {
   a.lut_lo1 = tb.lo1;
   a.lut_hi0 = tb.hi0;
   a.lut_hi1 = tb.hi1;
+  a.res_lo0 = tb.rlo0;
+  a.res_lo1 = tb.rlo1;
+  a.res_hi0 = tb.rhi0;
+  a.res_hi1 = tb.rhi1;
   a.out_unit = static_cast<float>(1.0 / (tb.alpha * d));
   a.score_unit = static_cast<float>(a.score_unit / (tb.alpha * std::sqrt(static_cast<double>(d))));
   return run_prefill_t<__half>(d, variant, a, st);
