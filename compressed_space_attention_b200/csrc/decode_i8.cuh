@@ -88,7 +88,11 @@ struct I8Cfg {
   static constexpr int MERGE_FLOATS = kI8Warps * GP * D;    // the sliced warp merge, over the rings
   static constexpr int QPREP_WORDS = 3 * KK * 2 * 32 + 8;   // per (b, kvh), see prep_i8_kernel
   static_assert(MERGE_FLOATS * 4 <= kI8Warps * RING_BYTES, "merge slices fit the rings");
-  static constexpr int SMEM = kI8Warps * RING_BYTES + SCRATCH_FLOATS * 4 +
+  // GP <= 2: the block's scores go through shared memory to one token per
+  // lane (see the softmax), kBlk tokens x 2 heads per warp.
+  static constexpr bool COMPACT = GP <= 2;
+  static constexpr int ZX_FLOATS = COMPACT ? kI8Warps * kBlk * 2 : 0;
+  static constexpr int SMEM = kI8Warps * RING_BYTES + SCRATCH_FLOATS * 4 + ZX_FLOATS * 4 +
                               2 * kI8Warps * 8 * 4 + kI8Warps * kI8Stages * 8 + 128;
   static constexpr int MIN_BLOCKS = (D == 256 && GP == 8) ? 2 : ((D == 256 && GP == 4) || GP == 8 ? 3 : 4);
 };
@@ -378,7 +382,8 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
 
   unsigned char *ring = smem + warp * C::RING_BYTES;
   float *scratch = reinterpret_cast<float *>(smem + kI8Warps * C::RING_BYTES);
-  float *wm = scratch + C::SCRATCH_FLOATS;          // [warps][8]
+  float *zx = scratch + C::SCRATCH_FLOATS;          // [warps][kBlk * 2] (GP <= 2)
+  float *wm = zx + C::ZX_FLOATS;                    // [warps][8]
   float *wl = wm + kI8Warps * 8;                    // [warps][8]
   uint64_t *full_bar = reinterpret_cast<uint64_t *>(wl + kI8Warps * 8) + warp * kI8Stages;
 
@@ -437,8 +442,10 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     for (int kk = 0; kk < C::KK; ++kk)
 #pragma unroll
       for (int half = 0; half < 2; ++half) qb[nq][kk][half] = qp[((nq * C::KK + kk) * 2 + half) * 32 + lane];
-  const float qk0 = __uint_as_float(qp[3 * C::KK * 2 * 32 + 2 * t]);       // 0 for padded heads
-  const float qk1 = __uint_as_float(qp[3 * C::KK * 2 * 32 + 2 * t + 1]);
+  // score factors of the lane's two heads: 2t, 2t + 1, or with the compact
+  // softmax (GP <= 2) heads 0, 1 in every lane; 0 for padded heads
+  const float qk0 = __uint_as_float(qp[3 * C::KK * 2 * 32 + (C::COMPACT ? 0 : 2 * t)]);
+  const float qk1 = __uint_as_float(qp[3 * C::KK * 2 * 32 + (C::COMPACT ? 1 : 2 * t + 1)]);
 
   // prmt selectors that move byte k of a packed (W_a, W_b) word to byte g&3
   // of a PV B register (zeros elsewhere): lo / hi byte of head parity g>>2.
@@ -568,6 +575,67 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     }
 
     // ---- softmax bookkeeping (log2 domain) ----
+    // u[T][hh]: (W head a, W head b) packed as two 16-bit fields; dinv: one
+    // unit of 256 E1 + E2 in the PV layout (heads 2nv + (t >> 1)).
+    uint32_t u[2][2];
+    float dinv[C::NV];
+    if constexpr (C::COMPACT) {
+      // One token per lane: the scores (valid in the t = 0 lanes) go through
+      // shared memory so that lane L holds token L's scores of heads 0, 1,
+      // and every softmax step below runs on 2 values per lane instead of 8
+      // (of which 6 belong to padded heads at GP <= 2).  Slot of token
+      // 16 T + 8 hh + g, head h: g 8 + T 4 + hh 2 + h.
+      float *zw = zx + warp * (kBlk * 2);
+      if (t == 0) {
+        *reinterpret_cast<float4 *>(zw + 8 * g) = make_float4(sc[0][0], sc[0][1], sc[0][2], sc[0][3]);
+        *reinterpret_cast<float4 *>(zw + 8 * g + 4) = make_float4(sc[1][0], sc[1][1], sc[1][2], sc[1][3]);
+      }
+      __syncwarp();
+      const float2 z = *reinterpret_cast<const float2 *>(zw + 8 * (lane & 7) + 4 * (lane >> 4) + 2 * ((lane >> 3) & 1));
+      const float sk = lds_half(nk + 2 * lane);
+      float svl = lds_half(nv + 2 * lane);
+      float x0 = z.x * sk * qk0, x1 = z.y * sk * qk1;
+      if (nvalid < kBlk && lane >= nvalid) {   // the chunk's partial last block
+        x0 = x1 = -INFINITY;
+        svl = 0.f;
+      }
+      // Move the reference maximum only when a score passes m_ref + 1.
+      if (__any_sync(0xffffffffu, x0 > m0 + 1.f || x1 > m1 + 1.f)) {
+        float mx0 = x0, mx1 = x1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float mn0 = mx0 > m0 + 1.f ? mx0 : m0, mn1 = mx1 > m1 + 1.f ? mx1 : m1;
+        const float f0 = ex2f(m0 - mn0), f1 = ex2f(m1 - mn1);   // 0 on the first block
+        l0 *= f0;
+        l1 *= f1;
+        m0 = mn0;
+        m1 = mn1;
+        const float F = (t >> 1) ? f1 : f0;
+#pragma unroll
+        for (int mb = 0; mb < C::MB; ++mb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[0][mb][e] *= F;
+      }
+      const float p0 = ex2f(x0 - m0), p1 = ex2f(x1 - m1);
+      l0 += p0;
+      l1 += p1;
+      const float pw0 = p0 * svl, pw1 = p1 * svl;
+      float pm0 = pw0, pm1 = pw1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, o));
+        pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, o));
+      }
+      // W_q = rint(p s^V kWMax / pm) <= kWMax from the low 16 bits of
+      // p s^V r + 2^23 (r needs no IEEE division: any r <= kWMax (1 + 2^-22)
+      // / pm keeps W_q within 16 bits, and dinv below uses pm itself).
+      const float r0 = pm0 > 0.f ? kWMax * rcp_approx(pm0) : 0.f, r1 = pm1 > 0.f ? kWMax * rcp_approx(pm1) : 0.f;
+      u[0][0] = pack_lo16(__float_as_uint(fmaf(pw0, r0, 8388608.f)), __float_as_uint(fmaf(pw1, r1, 8388608.f)));
+      dinv[0] = ((t >> 1) ? pm1 : pm0) * (128.f / kWMax);
+    } else {
     // x[T][e]: token 16T + 8(e >> 1) + g, head 2t + (e & 1).  Padded heads
     // (qk = 0) score 0 and never move a maximum; their weights only reach
     // accumulators that are never stored.
@@ -649,7 +717,6 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     // (r needs no IEEE division: any r <= kWMax (1 + 2^-22) / pm keeps W_q
     // within 16 bits, and dinv below uses pm itself.)
     const float r0 = pm0 > 0.f ? kWMax * rcp_approx(pm0) : 0.f, r1 = pm1 > 0.f ? kWMax * rcp_approx(pm1) : 0.f;
-    uint32_t u[2][2];
 #pragma unroll
     for (int T = 0; T < 2; ++T) {
 #pragma unroll
@@ -658,26 +725,37 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
         u[T][hh] = pack_lo16(__float_as_uint(wq0), __float_as_uint(wq1));
       }
     }
-    float dinv[C::NV];
 #pragma unroll
     for (int nvt = 0; nvt < C::NV; ++nvt) {
       const float da = __shfl_sync(0xffffffffu, pm0, nvt), db = __shfl_sync(0xffffffffu, pm1, nvt);
       dinv[nvt] = ((t >> 1) ? db : da) * (128.f / kWMax);
     }
+    }
 
     // ---- PV, per 16-token half: this lane's tokens t, t+4, t+8, t+12 ----
+    // With GP <= 2 the int32 sums of both halves accumulate in one pair of
+    // registers per element and are converted once per block (both halves
+    // share the block's scale); otherwise once per half.
+    int e1c[C::COMPACT ? C::MB : 1][4], e2c[C::COMPACT ? C::MB : 1][4];
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       // B fragments of W for each N tile nv (heads 2nv, 2nv+1): column g =
       // (head 2nv + (g >> 2), parity g & 3); MMA c covers tokens 16 h2 + 8c +
-      // {t, t+4}, held by the QK lanes (t or t+4, nv) in u[h2][c].
+      // {t, t+4}: held by lanes 16 h2 + 8c + t and + 4 (compact layout, in
+      // u[0][0]) or by the QK lanes (t or t+4, nv) in u[h2][c].
       uint32_t bh[C::NV][2][2], bl[C::NV][2][2];
 #pragma unroll
       for (int nvt = 0; nvt < C::NV; ++nvt) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const uint32_t xa = __shfl_sync(0xffffffffu, u[h2][c], 4 * t + nvt);
-          const uint32_t xb = __shfl_sync(0xffffffffu, u[h2][c], 4 * t + 16 + nvt);
+          uint32_t xa, xb;
+          if constexpr (C::COMPACT) {
+            xa = __shfl_sync(0xffffffffu, u[0][0], 16 * h2 + 8 * c + t);
+            xb = __shfl_sync(0xffffffffu, u[0][0], 16 * h2 + 8 * c + t + 4);
+          } else {
+            xa = __shfl_sync(0xffffffffu, u[h2][c], 4 * t + nvt);
+            xb = __shfl_sync(0xffffffffu, u[h2][c], 4 * t + 16 + nvt);
+          }
           bh[nvt][c][0] = prmt(xa, 0u, sel_hi);
           bh[nvt][c][1] = prmt(xb, 0u, sel_hi);
           bl[nvt][c][0] = prmt(xa, 0u, sel_lo);
@@ -713,6 +791,27 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
           al[r][0] = prmt(lut.vl0, lut.vl1, s0);
           al[r][1] = prmt(lut.vl0, lut.vl1, s1);
         }
+        if constexpr (C::COMPACT) {
+          // |256 E1 + E2| < 32 x 2^15 x 255 < 2^31 over the whole block.
+          int(&e1)[4] = e1c[mb];
+          int(&e2)[4] = e2c[mb];
+          if (h2 == 0) {
+            mma_s8u8_z(e1, ah[0][0], ah[0][1], ah[1][0], ah[1][1], bh[0][0][0], bh[0][0][1]);
+            mma_s8u8_z(e2, ah[0][0], ah[0][1], ah[1][0], ah[1][1], bl[0][0][0], bl[0][0][1]);
+          } else {
+            mma_s8u8(e1, ah[0][0], ah[0][1], ah[1][0], ah[1][1], bh[0][0][0], bh[0][0][1]);
+            mma_s8u8(e2, ah[0][0], ah[0][1], ah[1][0], ah[1][1], bl[0][0][0], bl[0][0][1]);
+          }
+          mma_s8u8(e1, ah[2][0], ah[2][1], ah[3][0], ah[3][1], bh[0][1][0], bh[0][1][1]);
+          mma_s8u8(e2, ah[2][0], ah[2][1], ah[3][0], ah[3][1], bl[0][1][0], bl[0][1][1]);
+          mma_s8u8(e2, al[0][0], al[0][1], al[1][0], al[1][1], bh[0][0][0], bh[0][0][1]);
+          mma_s8u8(e2, al[2][0], al[2][1], al[3][0], al[3][1], bh[0][1][0], bh[0][1][1]);
+          if (h2 == 1) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              acc[0][mb][e] = fmaf(static_cast<float>(256 * e1[e] + e2[e]), dinv[0], acc[0][mb][e]);
+          }
+        } else {
 #pragma unroll
         for (int nvt = 0; nvt < C::NV; ++nvt) {
           // This half's sums: |256 E1 + E2| < 16 x 2^15 x 255 < 2^31.
@@ -726,6 +825,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             acc[nvt][mb][e] = fmaf(static_cast<float>(256 * e1[e] + e2[e]), dinv[nvt], acc[nvt][mb][e]);
+        }
         }
       }
     }
@@ -744,9 +844,10 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
       if (!mbar_wait_bounded(&full_bar[k % kI8Stages], (k / kI8Stages) & 1)) break;
   }
 
-  // Per-warp totals over the 8 lanes sharing t.
+  // Per-warp totals over the 8 lanes sharing t (over all 32 lanes with
+  // the compact softmax, where m0, m1 are the same in every lane).
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
+  for (int o = C::COMPACT ? 1 : 4; o < 32; o <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
@@ -756,11 +857,12 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     // (rotated domain) over the ring memory; after one barrier the slices are
     // scaled to the common maximum and summed in warp order (a fixed order).
     float *slices = reinterpret_cast<float *>(smem);
-    if (g == 0) {
-      wm[warp * 8 + 2 * t] = m0;
-      wm[warp * 8 + 2 * t + 1] = m1;
-      wl[warp * 8 + 2 * t] = l0;
-      wl[warp * 8 + 2 * t + 1] = l1;
+    if (C::COMPACT ? lane == 0 : g == 0) {
+      const int h0 = C::COMPACT ? 0 : 2 * t;
+      wm[warp * 8 + h0] = m0;
+      wm[warp * 8 + h0 + 1] = m1;
+      wl[warp * 8 + h0] = l0;
+      wl[warp * 8 + h0 + 1] = l1;
     }
     {
       const int grp = D == 256 ? g : (g >> 1);
@@ -806,11 +908,12 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     }
   } else {
     __syncthreads();   // all warps are done with the q~ scratch
-    if (g == 0) {
-      wm[warp * 8 + 2 * t] = m0;
-      wm[warp * 8 + 2 * t + 1] = m1;
-      wl[warp * 8 + 2 * t] = l0;
-      wl[warp * 8 + 2 * t + 1] = l1;
+    if (C::COMPACT ? lane == 0 : g == 0) {
+      const int h0 = C::COMPACT ? 0 : 2 * t;
+      wm[warp * 8 + h0] = m0;
+      wm[warp * 8 + h0 + 1] = m1;
+      wl[warp * 8 + h0] = l0;
+      wl[warp * 8 + h0 + 1] = l1;
     }
     __syncthreads();
     // Merge the warps' accumulators into scratch[head][dim] (rotated domain),
