@@ -41,11 +41,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "packed-3-bit decode attn KV GB/s (% of HBM peak); quantize Mvec/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0      # B200's nominal HBM3e bandwidth (~8 TB/s), reported beside the measured copy peak
 # The files holding the decode split kernel's device code (its traffic in the
 # committed ncu summary is valid only while they are unchanged).
 KERNEL_SOURCES = ["compressed_space_attention_b200/csrc/decode_i8.cuh",
                   "compressed_space_attention_b200/csrc/common.cuh"]
-TRAFFIC_PROFILE = "profiles/decode_split_b32_gqa16_8_d256_t65536.md"
+TRAFFIC_FILE = "profiles/decode_split_traffic.json"
 
 WORKLOADS = {
     # name: (B, Hq, Hkv, T, d)
@@ -77,17 +78,52 @@ def source_hash():
 
 
 def read_traffic():
-    """Per-launch DRAM bytes of the decode split kernel from the committed ncu
-    summary, if that summary was taken on the current kernel source."""
-    path = os.path.join(ROOT, TRAFFIC_PROFILE)
+    """Per-launch DRAM bytes of the decode split kernel, from the data file
+    that ``--record-traffic`` wrote out of an ncu capture, if that capture
+    was taken on the current kernel source."""
+    path = os.path.join(ROOT, TRAFFIC_FILE)
     if not os.path.exists(path):
         return None
-    text = open(path).read()
-    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-    m_val = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_val or m_hash.group(1) != source_hash():
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("source_hash") != source_hash():
         return None
-    return float(m_val.group(1))
+    return float(rec["traffic_bytes_per_launch"])
+
+
+def record_traffic(csv_path, kernel_regex, scale, note):
+    """Writes TRAFFIC_FILE from an ncu ``--page raw --csv`` export: the
+    dram__bytes_read.sum + dram__bytes_write.sum of the launches whose name
+    matches kernel_regex (averaged), times `scale` (the full launch's units
+    over the captured launch's), with the current kernel source hash."""
+    import csv
+
+    with open(csv_path, newline="") as f:
+        rows = list(csv.reader(f))
+    header = rows[0]
+    idx_name = header.index("Kernel Name")
+    units = {}
+    for unit_row in rows[1:2]:
+        units = dict(zip(header, unit_row))
+    cols = {m: header.index(m) for m in ("dram__bytes_read.sum", "dram__bytes_write.sum")}
+    mult = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+    vals = []
+    for r in rows[2:]:
+        if len(r) <= max(cols.values()) or not re.search(kernel_regex, r[idx_name]):
+            continue
+        tot = 0.0
+        for m, i in cols.items():
+            tot += float(r[i].replace(",", "")) * mult.get(units.get(m, "byte"), 1.0)
+        vals.append(tot)
+    if not vals:
+        raise SystemExit(f"no launch of {kernel_regex} in {csv_path}")
+    rec = {"kernel": kernel_regex, "source_hash": source_hash(),
+           "captured_bytes_per_launch": sum(vals) / len(vals), "scale": scale,
+           "traffic_bytes_per_launch": sum(vals) / len(vals) * scale, "launches": len(vals), "note": note}
+    with open(os.path.join(ROOT, TRAFFIC_FILE), "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    print(json.dumps(rec))
 
 
 def measured_peaks():
@@ -247,6 +283,164 @@ def oracle_quantize_rate(n=4096, seed=77):
 
 
 # ---------------------------------------------------------------------------
+# The oracle on all host cores: spawned worker processes (no CUDA in them),
+# BLAS threads 1 each, released together by a barrier so that the timed parts
+# overlap; the rate is the bytes (or vectors) of all workers over the
+# slowest worker's timed seconds.
+# ---------------------------------------------------------------------------
+
+_POOL_BARRIER = None
+
+
+def _pool_init(barrier):
+    global _POOL_BARRIER
+    _POOL_BARRIER = barrier
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _pool_run(fn, tasks, sync, workers=None):
+    """Runs fn over tasks in spawned processes.  With sync, one task per
+    worker, each waiting on a shared barrier before its timed part."""
+    import multiprocessing as mp
+
+    ctx = mp.get_context("spawn")
+    n = len(tasks) if sync else max(1, min(len(tasks), workers or len(tasks)))
+    barrier = ctx.Barrier(n) if sync else None
+    with ctx.Pool(n, initializer=_pool_init, initargs=(barrier,)) as pool:
+        return pool.map_async(fn, tasks, chunksize=1).get(timeout=900)
+
+
+def _oracle_decode_task(task):
+    """One (b, kvh) pair of the decode workload: its G query heads over
+    `tokens` tokens; oracle decodes repeated for at least min_s seconds."""
+    from threadpoolctl import threadpool_limits
+
+    import oracle as O
+    import synth
+
+    workload, seed, tokens, min_s = task
+    B, Hq, Hkv, T, d = WORKLOADS[workload]
+    g = Hq // Hkv
+    with threadpool_limits(limits=1):
+        k, v = synth.student_t_kv(1, tokens, d, seed=seed)
+        prk = O.make_params(d, O.FULL, seed=1)
+        prv = O.make_params(d, O.FULL, seed=2)
+        pk, nk = O.quantize(k[0].astype(np.float64), prk, 3, O.FULL)
+        pv, nv = O.quantize(v[0].astype(np.float64), prv, 3, O.FULL)
+        q = synth.queries(1, g, d, seed=seed + 1)
+        args = (q, pk[None], pv[None], nk[None], nv[None], [tokens], prk, prv, 3, O.FULL, 1 / math.sqrt(d))
+        if _POOL_BARRIER is not None:
+            _POOL_BARRIER.wait(timeout=600)
+        reps, elapsed = 0, 0.0
+        while elapsed < min_s:
+            t0 = time.perf_counter()
+            O.decode_attention(*args)
+            elapsed += time.perf_counter() - t0
+            reps += 1
+    return reps * tokens * kv_bytes_per_token_head(d), reps * tokens, elapsed
+
+
+def _oracle_quantize_task(task):
+    """Oracle quantize of one seeded chunk of stage-1 unit vectors, repeated
+    for at least min_s seconds."""
+    from threadpoolctl import threadpool_limits
+
+    import oracle as O
+    import synth
+
+    n, d, bits, seed, min_s = task
+    with threadpool_limits(limits=1):
+        x = synth.unit_vectors(n, d, seed=seed, dtype=np.float16).astype(np.float64)
+        p = O.make_params(d, O.FULL, seed=1)
+        if _POOL_BARRIER is not None:
+            _POOL_BARRIER.wait(timeout=600)
+        reps, elapsed = 0, 0.0
+        while elapsed < min_s:
+            t0 = time.perf_counter()
+            O.quantize(x, p, bits, O.FULL)
+            elapsed += time.perf_counter() - t0
+            reps += 1
+    return reps * n, elapsed
+
+
+def oracle_pool_rates(workload, cores, tokens=2048, min_s=6.0):
+    """The oracle on `cores` host cores: decode GB/s and token-heads/s over
+    one (b, kvh) pair per core, and quantize vectors/s over one 4,096-vector
+    chunk per core (stage-1 setting, d=128, 3-bit, float16 input)."""
+    dec = _pool_run(_oracle_decode_task, [(workload, 3000 + 7 * i, tokens, min_s) for i in range(cores)], True)
+    qnt = _pool_run(_oracle_quantize_task,
+                    [(4096, STAGE1["d"], STAGE1["bits"], 5000 + i, min_s / 2) for i in range(cores)], True)
+    t_dec = max(r[2] for r in dec)
+    t_q = max(r[1] for r in qnt)
+    B, Hq, Hkv, T, d = WORKLOADS[workload]
+    return {
+        "cores": cores,
+        "decode_gbs": sum(r[0] for r in dec) / t_dec / 1e9,
+        "decode_token_heads_per_s": sum(r[1] for r in dec) / t_dec,
+        "quantize_vec_per_s": sum(r[0] for r in qnt) / t_q,
+        "sample": (f"one (b, kvh) pair per core ({Hq // Hkv} query heads, {tokens} tokens, d={d}) and one "
+                   f"4,096-vector stage-1 chunk per core; {cores} spawned processes, BLAS threads 1 each, "
+                   f"released together; rate = all workers' work / slowest worker's seconds"),
+    }
+
+
+def _oracle_check_task(task):
+    """Oracle compression of one input chunk, compared with the GPU's codes
+    and norms for the same chunk: (vectors, code mismatches inside the 1e-5
+    boundary band, outside it, norm mismatches at an float16 midpoint, away
+    from one, oracle reconstruction squared error, GPU reconstruction
+    squared error, squared norm of the input)."""
+    from threadpoolctl import threadpool_limits
+
+    import oracle as O
+
+    x, params, bits, variant, gcodes, gnorms, grecon = task
+    with threadpool_limits(limits=1):
+        d = x.shape[-1]
+        x64 = np.asarray(x, dtype=np.float64)[None]
+        oc, on, y = O.quantize(x64, params, bits, variant, return_rotated=True)
+        _, thr = O.make_codebook(d, bits)
+        gc = O.bitunpack(np.asarray(gcodes)[None], bits, d)
+        rc = O.bitunpack(oc, bits, d)
+        mism = gc != rc
+        band = np.zeros(mism.sum(), dtype=bool)
+        if mism.any():
+            dist = np.min(np.abs(y[mism][:, None] - np.asarray(thr)[None, :]), axis=1)
+            band = dist < 1e-5
+        gn = np.asarray(gnorms, dtype=np.float16)[None]
+        nm = gn.view(np.uint16) != on.view(np.uint16)
+        s = np.sqrt(np.sum(x64 * x64, axis=-1))
+        mid = 0.5 * (gn.astype(np.float64) + on.astype(np.float64))
+        at_mid = np.abs(s - mid) <= 1e-6 * s
+        orec = O.dequantize(oc, on, params, bits, variant, d)
+        return (x64.shape[1], int(band.sum()), int((~band).sum()), int((nm & at_mid).sum()),
+                int((nm & ~at_mid).sum()), float(np.sum((orec - x64) ** 2)),
+                float(np.sum((np.asarray(grecon, dtype=np.float64)[None] - x64) ** 2)), float(np.sum(x64 * x64)))
+
+
+def oracle_checks(tasks, cores):
+    return _pool_run(_oracle_check_task, tasks, False, workers=cores) if tasks else []
+
+
+def summarize_checks(rows):
+    n = sum(r[0] for r in rows)
+    return {"vectors": n, "code_mismatches_in_band": sum(r[1] for r in rows),
+            "code_mismatches_outside_band": sum(r[2] for r in rows),
+            "norm_mismatches_at_midpoint": sum(r[3] for r in rows),
+            "norm_mismatches_elsewhere": sum(r[4] for r in rows),
+            "rel_mse_oracle": sum(r[5] for r in rows) / sum(r[7] for r in rows),
+            "rel_mse_gpu": sum(r[6] for r in rows) / sum(r[7] for r in rows)}
+
+
+# ---------------------------------------------------------------------------
 # Reference arm
 # ---------------------------------------------------------------------------
 
@@ -306,7 +500,9 @@ def workload_config(workload, n_gpus, batch=0, context=0):
         "workload": workload + "+stage1_quantize_dequantize_d128_b3_f16_n1048576",
         "batch": B, "context": T, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d, "bits": 3,
         "variant": "IsoQuant-Full", "stage1_vectors": STAGE1["n"],
-        "l2": "inputs larger than L2: each step streams the whole packed K/V cache (no explicit flush)",
+        "l2": ("inputs larger than L2: each step streams the whole 3.3 GB packed K/V cache; the stage-1 "
+               "quantize input is evicted by that stream between steps, and the dequantize reads codes "
+               "written two steps earlier (four rotating 50 MB code buffers)"),
         "parallelism": f"replicas x{n_gpus} (weak; no data-path collective)",
     }
 
@@ -338,6 +534,157 @@ def rank_seed(rank):
 # ---------------------------------------------------------------------------
 # CUDA arm
 # ---------------------------------------------------------------------------
+
+class L2Flush:
+    """Evicts the 126 MB L2 between timed repetitions: writes, then reads, a
+    buffer of four times the L2 size, so that the lines it leaves behind are
+    clean (no write-back traffic lands in the next timed launch)."""
+
+    def __init__(self, torch, dev):
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size or (126 << 20)
+        self.buf = torch.empty(4 * l2, dtype=torch.uint8, device=dev)
+        self.bytes = 4 * l2
+
+    def __call__(self):
+        self.buf.zero_()
+        self.buf.max()
+
+
+def timed_reps(torch, stream, fn, reps, flush=None):
+    """Device times (ms) of `reps` calls of fn, each after an L2 flush when
+    one is given, CUDA events on the launching stream around the call only."""
+    out = []
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1))
+    return out
+
+
+def med_cv(xs):
+    m = float(statistics.median(xs))
+    cv = float(statistics.pstdev(xs) / statistics.mean(xs)) if len(xs) > 1 and statistics.mean(xs) > 0 else 0.0
+    return m, cv
+
+
+STAGE1_SWEEP_SLICE = 4096
+
+
+def measure_stage1_sweep(isoq, torch, dev, stream, flush, hbm, cores, n=1 << 20, reps=5):
+    """The 36-setting stage-1 sweep: d in {128, 256, 512} x bits in {2, 3, 4}
+    x {float16, float32} x {Full, Fast}, N = 2^20 normalised N(0, I_d)
+    vectors.  Per setting: quantize and dequantize device time (median of
+    `reps`, L2 flushed before each), vectors/s, quantize GB/s on input +
+    packed codes + float16 norms and its fraction of HBM peak, the relative
+    reconstruction MSE over all N; and on a seeded 4,096-vector slice, the
+    codes and norms against the oracle (mismatch counts inside and outside
+    the 1e-5 boundary band) and both reconstruction MSEs."""
+    import synth
+
+    rows, checks, gen = [], [], torch.Generator(device=dev)
+    for d in (128, 256, 512):
+        for var, vname in ((isoq.ISOQ_FULL, "Full"), (isoq.ISOQ_FAST, "Fast")):
+            p_np = isoq.isoq_make_params(d, var, 1, 1)
+            p = torch.from_numpy(p_np).to(dev)
+            for dt, dname, np_dt in ((torch.float16, "f16", np.float16), (torch.float32, "f32", np.float32)):
+                gen.manual_seed(1000 + d)
+                x = torch.randn((1, n, d), generator=gen, device=dev)
+                x = (x / x.norm(dim=-1, keepdim=True)).to(dt)
+                r = torch.empty_like(x)
+                nrm = torch.empty((1, n), dtype=torch.float16, device=dev)
+                xs_np = synth.unit_vectors(STAGE1_SWEEP_SLICE, d, seed=d + var, dtype=np_dt)
+                xs = torch.from_numpy(xs_np).to(dev)
+                for bits in (2, 3, 4):
+                    pb = isoq.isoq_packed_bytes(d, bits)
+                    c = torch.empty((1, n, pb), dtype=torch.uint8, device=dev)
+                    qf = lambda: isoq.isoq_quantize(x, p, bits, var, codes=c, norms=nrm)  # noqa: E731
+                    df = lambda: isoq.isoq_dequantize(c, nrm, p, d, bits, var, out=r)  # noqa: E731
+                    qf()
+                    df()
+                    tq = timed_reps(torch, stream, qf, reps, flush)
+                    td = timed_reps(torch, stream, df, reps, flush)
+                    xf = x.float()
+                    mse = float(((r.float() - xf) ** 2).sum() / (xf * xf).sum())
+                    mq, cvq = med_cv(tq)
+                    md, cvd = med_cv(td)
+                    qbytes = n * (d * x.element_size() + pb + 2)
+                    row = {"d": d, "bits": bits, "dtype": dname, "variant": vname,
+                           "quantize_ms": mq, "quantize_cv": cvq, "quantize_mvec_s": n / (mq * 1e-3) / 1e6,
+                           "quantize_gbs": qbytes / (mq * 1e-3) / 1e9, "quantize_frac": qbytes / (mq * 1e-3) / 1e9 / hbm,
+                           "dequantize_ms": md, "dequantize_cv": cvd, "dequantize_mvec_s": n / (md * 1e-3) / 1e6,
+                           "rel_mse_gpu_all": mse}
+                    sc, sn = isoq.isoq_quantize(xs, p, bits, var)
+                    sr = isoq.isoq_dequantize(sc, sn, p, d, bits, var, out_dtype=torch.float32)
+                    checks.append((xs_np[0], p_np, bits, var, sc[0].cpu().numpy(), sn[0].cpu().numpy(),
+                                   sr[0].cpu().numpy()))
+                    rows.append(row)
+                    del c
+                del x, r, nrm, xs
+    torch.cuda.empty_cache()
+    assert isoq.isoq_check_device_error() == 0
+    results = oracle_checks(checks, cores)
+    for row, res in zip(rows, results):
+        row["oracle_slice"] = summarize_checks([res])
+    return {"workload": "stage-1 sweep: 36 settings, 2^20 normalised N(0, I_d) vectors each (device-drawn); "
+                        f"oracle comparison on a {STAGE1_SWEEP_SLICE}-vector seeded slice per setting",
+            "timing": f"median of {reps} launches, L2 flushed before each (CUDA events around the launch)",
+            "settings": rows,
+            "all_slices": summarize_checks(results)}
+
+
+def measure_prefill_compression(isoq, torch, dev, stream, flush, hbm, cores, reps=10):
+    """The KV-cache prefill-compression workload: 4 KV heads x 32,768 tokens x
+    d=128 float16 K and V (Student-t nu=4 with 4 outlier channels per head
+    x10, RoPE at base 1e6 on K), 3-bit Full, K rotation seed 1, V seed 2.
+    Throughput of isoq_quantize on K then V (80 MB, below L2: flushed before
+    each repetition), and every code and norm against the oracle."""
+    import synth
+
+    h, t, d, bits = 4, 32768, 128, 3
+    k, v = synth.student_t_kv(h, t, d, seed=3)
+    k, v = k[0], v[0]
+    pk_np = isoq.isoq_make_params(d, isoq.ISOQ_FULL, 1, h)
+    pv_np = isoq.isoq_make_params(d, isoq.ISOQ_FULL, 2, h)
+    kd, vd = torch.from_numpy(k).to(dev), torch.from_numpy(v).to(dev)
+    pk, pv = torch.from_numpy(pk_np).to(dev), torch.from_numpy(pv_np).to(dev)
+    ck = torch.empty((h, t, 48), dtype=torch.uint8, device=dev)
+    cv = torch.empty_like(ck)
+    nk = torch.empty((h, t), dtype=torch.float16, device=dev)
+    nv = torch.empty_like(nk)
+
+    def both():
+        isoq.isoq_quantize(kd, pk, bits, isoq.ISOQ_FULL, codes=ck, norms=nk)
+        isoq.isoq_quantize(vd, pv, bits, isoq.ISOQ_FULL, codes=cv, norms=nv)
+
+    both()
+    ts = timed_reps(torch, stream, both, reps, flush)
+    m, cv_ = med_cv(ts)
+    nvec = 2 * h * t
+    nbytes = nvec * (2 * d + 48 + 2)
+    rk = isoq.isoq_dequantize(ck, nk, pk, d, bits, isoq.ISOQ_FULL).cpu().numpy()
+    rv = isoq.isoq_dequantize(cv, nv, pv, d, bits, isoq.ISOQ_FULL).cpu().numpy()
+    assert isoq.isoq_check_device_error() == 0
+    tasks = []
+    step = 8192
+    for x, par, codes, norms, rec in ((k, pk_np, ck, nk, rk), (v, pv_np, cv, nv, rv)):
+        cc, nn = codes.cpu().numpy(), norms.cpu().numpy()
+        for hh in range(h):
+            for t0 in range(0, t, step):
+                tasks.append((x[hh, t0:t0 + step], par[hh:hh + 1], bits, isoq.ISOQ_FULL, cc[hh, t0:t0 + step],
+                              nn[hh, t0:t0 + step], rec[hh, t0:t0 + step]))
+    checks = summarize_checks(oracle_checks(tasks, cores))
+    return {"workload": "prefill compression: 4 KV heads x 32,768 tokens x d=128 float16 K and V (Student-t "
+                        "nu=4, 4 outlier channels x10 per head, RoPE base 1e6 on K), 3-bit Full",
+            "ms": m, "cv": cv_, "mvec_s": nvec / (m * 1e-3) / 1e6, "gbs": nbytes / (m * 1e-3) / 1e9,
+            "frac": nbytes / (m * 1e-3) / 1e9 / hbm, "vectors": nvec, "bytes": nbytes,
+            "timing": f"median of {reps} (K then V), L2 flushed before each", "oracle": checks}
+
 
 VARIANT_NAMES = {0: "Full (WHT+SO(4), v3)", 1: "Fast (WHT+q_L)", 2: "2-D special case (WHT+planar)",
                  3: "v2: block SO(4), no WHT", 4: "v1: single quaternion, no WHT"}
@@ -494,11 +841,14 @@ DECODE_SWEEP = [
 ] + [(f"b32_gqa16_8_d256_t{t}", 32, 16, 8, t, 256, False) for t in (1024, 2048, 4096, 8192, 16384, 32768)]
 
 
-def measure_decode_sweep(isoq, synth, torch, dev, seed0, hbm, reps=20):
+def measure_decode_sweep(isoq, synth, torch, dev, seed0, hbm, flush, reps=20, runs=3):
     """Decode attention (query preparation + split + combine) on the small
     decode workloads and the long-context shape at shorter contexts: each
-    call captured once in a CUDA graph and replayed `reps` times between two
-    events, so host launch overhead does not enter the small cases."""
+    call captured once in a CUDA graph, so host launch overhead does not
+    enter the small cases; every replay follows an L2 flush (these working
+    sets, 13-103 MB, fit in the 126 MB L2) and is timed alone.  `runs` runs
+    of `reps` replays: the median over all replays, and the coefficient of
+    variation of the runs' medians."""
     out = {}
     for name, B, Hq, Hkv, T, d, ragged in DECODE_SWEEP:
         bits, variant, pb = 3, isoq.ISOQ_FULL, d * 3 // 8
@@ -524,22 +874,21 @@ def measure_decode_sweep(isoq, synth, torch, dev, seed0, hbm, reps=20):
             call()
         g.replay()
         torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            g.replay()
-        e1.record()
-        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream(dev)
+        run_ms = [timed_reps(torch, stream, g.replay, reps, flush) for _ in range(runs)]
         assert isoq.isoq_check_device_error() == 0
-        us = e0.elapsed_time(e1) / reps * 1e3
+        med, _ = med_cv([t for r in run_ms for t in r])
+        _, cv = med_cv([statistics.median(r) for r in run_ms])
+        us = med * 1e3
         kv_bytes = int(lens_np.clip(0, T).sum()) * Hkv * kv_bytes_per_token_head(d, bits)
         gbps = kv_bytes / (us * 1e-6) / 1e9
-        out[name] = {"us": us, "gbps": gbps, "frac": gbps / hbm, "kv_bytes": kv_bytes}
+        out[name] = {"us": us, "gbps": gbps, "frac": gbps / hbm, "kv_bytes": kv_bytes, "cv_of_runs": cv,
+                     "min_us": min(t for r in run_ms for t in r) * 1e3}
         del g, pk, pv, nk, nv, q, o, ws
         torch.cuda.empty_cache()
-    return {"what": "isoq_decode_attention (prep + split + combine) replayed from a CUDA graph; KV GB/s on "
-                    "the packed bytes of the valid tokens", "by_workload": out}
+    return {"what": "isoq_decode_attention (prep + split + combine) replayed from a CUDA graph, L2 flushed "
+                    f"before every replay; median of {runs} x {reps} replays; KV GB/s on the packed bytes of the "
+                    "valid tokens", "by_workload": out}
 
 
 def run_isoq(args):
@@ -609,19 +958,29 @@ def run_isoq(args):
     x1 = torch.randn((1, n1, d1), generator=gen, device=dev)
     x1 = (x1 / x1.norm(dim=-1, keepdim=True)).half()
     p1 = torch.from_numpy(isoq.isoq_make_params(d1, variant, 1, 1)).to(dev)
-    c1 = torch.empty((1, n1, d1 * bits // 8), dtype=torch.uint8, device=dev)
-    s1 = torch.empty((1, n1), dtype=torch.float16, device=dev)
+    # Step i quantizes into code slot i % R and dequantizes slot (i + 2) % R,
+    # written two steps (and 6.6 GB of decode reads) earlier, so the
+    # dequantize does not read codes the quantize has just left in L2.
+    n_slots = 4
+    c1 = [torch.empty((1, n1, d1 * bits // 8), dtype=torch.uint8, device=dev) for _ in range(n_slots)]
+    s1 = [torch.empty((1, n1), dtype=torch.float16, device=dev) for _ in range(n_slots)]
+    for c_, s_ in zip(c1, s1):
+        isoq.isoq_quantize(x1, p1, bits, variant, codes=c_, norms=s_)
     r1 = torch.empty((1, n1, d1), dtype=torch.float16, device=dev)
     q_bytes = n1 * (d1 * 2 + d1 * bits // 8 + 2)
     dq_bytes = n1 * (d1 * bits // 8 + 2 + d1 * 2)
+    step_no = [0]
 
     def step(ev=None):
+        i = step_no[0]
+        step_no[0] += 1
+        qs, ds = i % n_slots, (i + 2) % n_slots
         if ev:
             ev[0].record(stream)
-        isoq.isoq_quantize(x1, p1, bits, variant, codes=c1, norms=s1)
+        isoq.isoq_quantize(x1, p1, bits, variant, codes=c1[qs], norms=s1[qs])
         if ev:
             ev[1].record(stream)
-        isoq.isoq_dequantize(c1, s1, p1, d1, bits, variant, out=r1)
+        isoq.isoq_dequantize(c1[ds], s1[ds], p1, d1, bits, variant, out=r1)
         if ev:
             ev[2].record(stream)
         isoq.isoq_decode_split(q, pk, pv, nk, nv, lens, prk, bits, variant, ws)
@@ -661,6 +1020,11 @@ def run_isoq(args):
     t_split = sum(e[2].elapsed_time(e[3]) for e in events)
     t_comb = sum(e[3].elapsed_time(e[4]) for e in events)
     t_decode = t_split + t_comb
+    # three runs: the timed steps in three consecutive groups
+    per_step_dec = [e[2].elapsed_time(e[4]) for e in events]
+    groups = [per_step_dec[i * len(per_step_dec) // 3:(i + 1) * len(per_step_dec) // 3] for i in range(3)]
+    run_gbs = [kv_bytes * len(gp) / (sum(gp) * 1e-3) / 1e9 for gp in groups if gp]
+    split_ms = [e[2].elapsed_time(e[3]) for e in events]
     assert isoq.isoq_check_device_error() == 0
 
     # ---- end to end through the API with host buffers (decode half) ----
@@ -720,8 +1084,15 @@ def run_isoq(args):
     variants = measure_variants(isoq, synth, torch, dev, stream, x1, seed0) if not args.no_variants else None
     comparator = measure_rotor_comparison(isoq, torch, dev, stream) if not args.no_comparator else None
     peaks_all, _ = measured_peaks()
-    sweep = (measure_decode_sweep(isoq, synth, torch, dev, seed0, float(peaks_all.get("hbm_gbs", FALLBACK_HBM_GBS)))
+    hbm_all = float(peaks_all.get("hbm_gbs", FALLBACK_HBM_GBS))
+    flush = L2Flush(torch, dev)
+    cores = host_cores()
+    sweep = (measure_decode_sweep(isoq, synth, torch, dev, seed0, hbm_all, flush)
              if not args.no_sweep else None)
+    stage1 = (measure_stage1_sweep(isoq, torch, dev, stream, flush, hbm_all, cores)
+              if not args.no_stage1_sweep and rank == 0 else None)
+    c3 = (measure_prefill_compression(isoq, torch, dev, stream, flush, hbm_all, cores)
+          if not args.no_stage1_sweep and rank == 0 else None)
     prefill = (measure_prefill(isoq, synth, torch, dev, stream, seed0,
                                float(peaks_all.get("bf16_tflops", 1590.0))) if not args.no_prefill else None)
 
@@ -741,8 +1112,14 @@ def run_isoq(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": workload_config(args.workload, n_ranks, args.batch, args.context),
         "frac_of_hbm_peak": value / n_ranks / hbm,
+        "frac_of_nominal_8000_gbs": value / n_ranks / NOMINAL_HBM_GBS,
+        "runs": {"what": "the timed steps in three consecutive groups: decode (split + combine) GB/s of each",
+                 "gbs": run_gbs, "median_gbs": float(statistics.median(run_gbs)),
+                 "cv": med_cv(run_gbs)[1] if len(run_gbs) > 1 else 0.0,
+                 "split_ms_median": float(statistics.median(split_ms)), "split_ms_cv": med_cv(split_ms)[1]},
         "roofline": {"bound": "hbm", "kernel": "split_i8_kernel<256,Full,GP=2> (decode split)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "frac_of_nominal_8000_gbs": achieved / NOMINAL_HBM_GBS,
                      "traffic": read_traffic(), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                      "algorithmic_bytes_per_launch": kv_bytes},
         "quantize": {"value": n_ranks * n1 * args.steps / (t_quant * 1e-3) / 1e6, "unit": "Mvec/s",
@@ -766,6 +1143,8 @@ def run_isoq(args):
         "rotorquant_comparison": comparator,
         "prefill": prefill,
         "decode_sweep": sweep,
+        "stage1_sweep": stage1,
+        "prefill_compression": c3,
         # per step: quantize_kernel, dequantize_kernel, prep_i8_kernel +
         # split_i8_kernel (isoq_decode_split), combine_kernel
         "gpu_launches": 5 * args.steps,
@@ -775,7 +1154,8 @@ def run_isoq(args):
         gbs, secs, desc = oracle_decode_sample(args.workload)
         line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                                 "sample": desc, "seconds": secs,
-                                "quantize_mvec_s": oracle_quantize_rate()}
+                                "quantize_mvec_s": oracle_quantize_rate(),
+                                "all_cores": oracle_pool_rates(args.workload, cores)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
@@ -803,11 +1183,21 @@ def main():
                     help="skip the rotation-variant measurements (2-D case, ablation v1/v2)")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (profiling runs)")
+    ap.add_argument("--no-stage1-sweep", action="store_true",
+                    help="skip the 36-setting stage-1 sweep and the prefill-compression line")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the decode batch size (smaller profiling cases)")
     ap.add_argument("--context", type=int, default=0,
                     help="override the decode context length (the long-context sweep)")
+    ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
+                    help="write the decode split's per-launch DRAM traffic from an ncu raw CSV export and exit")
+    ap.add_argument("--traffic-scale", type=float, default=1.0,
+                    help="full launch's units over the captured launch's (with --record-traffic)")
+    ap.add_argument("--traffic-note", default="", help="how the capture was taken (with --record-traffic)")
     args = ap.parse_args()
+    if args.record_traffic:
+        record_traffic(args.record_traffic, r"split_i8_kernel", args.traffic_scale, args.traffic_note)
+        return 0
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
