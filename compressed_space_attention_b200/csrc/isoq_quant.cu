@@ -51,6 +51,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "tcgen05.cuh"
@@ -222,7 +223,8 @@ __device__ void build_block_matrices(const float *params_head, float *mat, int t
 }
 
 // Applies the block matrices of one group (16 pairs starting at xp[base]).
-__device__ __forceinline__ void apply_group_matrices(uint64_t (&xp)[kPairs], int base, uint32_t mat_g) {
+template <int NP>
+__device__ __forceinline__ void apply_group_matrices(uint64_t (&xp)[NP], int base, uint32_t mat_g) {
 #pragma unroll
   for (int beta = 0; beta < 4; ++beta) {
     const uint64_t z0 = xp[base + 4 * beta], z1 = xp[base + 4 * beta + 1];
@@ -316,8 +318,8 @@ __device__ __forceinline__ float search_scale(float norm) {
 // integer pipe.  Every partial sum is a multiple of 1/2 in [2^22, 2^23),
 // where float32 steps by 1/2, so all of it is exact, and the packed field
 // is the float's mantissa shifted right by one bit.
-template <int BITS>
-__device__ __forceinline__ void quantize_group(const uint64_t (&xp)[kPairs], int base,
+template <int BITS, int NP>
+__device__ __forceinline__ void quantize_group(const uint64_t (&xp)[NP], int base,
                                                const float *tb, float big, uint32_t *w) {
   constexpr int L = 1 << BITS, NPOS = L / 2 - 1;
   constexpr int PER_HALF = 16 / BITS == 5 ? 4 : 16 / BITS;   // codes per 16-bit half (3 bits: 4-bit fields)
@@ -600,6 +602,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
   }
 }
 
+#include "quant_tc.cuh"
+
 // ---------------------------------------------------------------------------
 // Dequantize
 // ---------------------------------------------------------------------------
@@ -773,10 +777,66 @@ int num_sms() {
   return n;
 }
 
+// d = 128 float16 input with the WHT: the tensor-core compressor
+// (quant_tc.cuh), one CTA per SM.
+template <int BITS, bool FULL>
+int launch_quantize_tc(const void *x, int n_heads, long long n_vec, long long head_stride,
+                       long long vec_stride, const float *params, uint8_t *codes, uint16_t *norms,
+                       long long out_head_stride, cudaStream_t stream) {
+  auto kernel = quantize_tc_kernel<BITS, FULL>;
+  static bool configured = false;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured) {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTqSmem);
+      if (e != cudaSuccess)
+        return set_error(ISOQ_ERR_CUDA, "quantize (tcgen05): cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      configured = true;
+    }
+  }
+  EncodeTiledFn encode = encode_tiled_fn();
+  if (!encode) return set_error(ISOQ_ERR_CUDA, "quantize: cuTensorMapEncodeTiled unavailable");
+  CUtensorMap map;
+  const cuuint64_t gdim[3] = {static_cast<cuuint64_t>(kTqD), static_cast<cuuint64_t>(n_vec),
+                              static_cast<cuuint64_t>(n_heads)};
+  const long long hs = n_heads > 1 ? head_stride : vec_stride * n_vec;
+  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(vec_stride * 2), static_cast<cuuint64_t>(hs * 2)};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(kTqRows), 1u};
+  const cuuint32_t estride[3] = {1u, 1u, 1u};
+  const CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(x), gdim, gstride, box,
+                            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(ISOQ_ERR_UNSUPPORTED, "quantize: tensor map encode failed (%d)", (int)r);
+
+  QuantArgs a;
+  a.params = params;
+  a.codes = codes;
+  a.norms = norms;
+  a.out_head_stride = out_head_stride;
+  a.n_vec = n_vec;
+  a.n_heads = n_heads;
+  a.tiles_per_head = static_cast<int>((n_vec + kTqRows - 1) / kTqRows);
+  a.total_tiles = static_cast<long long>(a.tiles_per_head) * n_heads;
+  CodebookF32 cb;
+  codebook_f32(kTqD, BITS, &cb);
+  constexpr int L = 1 << BITS;
+  for (int j = 0; j < 7; ++j) a.tau[j] = j < L / 2 - 1 ? cb.threshold[L / 2 + j] : 0.f;
+  long long grid = num_sms();
+  if (grid > a.total_tiles) grid = a.total_tiles;
+  kernel<<<static_cast<unsigned>(grid), kTqThreads, kTqSmem, stream>>>(map, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "quantize (tcgen05) launch: %s", cudaGetErrorString(e));
+  return ISOQ_OK;
+}
+
 template <typename T, int D, int BITS, int RK>
 int launch_quantize(const void *x, int n_heads, long long n_vec, long long head_stride,
                     long long vec_stride, const float *params, uint8_t *codes, uint16_t *norms,
                     long long out_head_stride, cudaStream_t stream) {
+  if constexpr (std::is_same<T, __half>::value && D == 128 && RK != kRotBlock)
+    return launch_quantize_tc<BITS, RK == kRotWhtFull>(x, n_heads, n_vec, head_stride, vec_stride, params,
+                                                       codes, norms, out_head_stride, stream);
   using C = Cfg<T, D, BITS>;
   auto kernel = quantize_kernel<T, D, BITS, RK>;
   static int max_ctas_per_sm = -1;
