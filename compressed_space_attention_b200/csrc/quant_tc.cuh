@@ -1,34 +1,40 @@
-// Compressor for d = 128 float16 vectors with the Walsh-Hadamard transform on
-// the 5th-generation tensor cores (tcgen05 + TMEM).  Included by
-// isoq_quant.cu inside namespace isoq::quant, after the register-level pieces
-// (apply_group_matrices, quantize_group, search_scale).
+// Compressor for d = 128 float16 vectors with the whole rotation on the
+// 5th-generation tensor cores (tcgen05 + TMEM).  Included by isoq_quant.cu
+// inside namespace isoq::quant, after the register-level pieces
+// (quantize_group, search_scale).
 //
 // RotaryQuant §3.2 Algorithm 1 on a tile of 128 vectors x of one head:
-//   u = R_SO4 (H_128 x)      (unnormalised; R_SO4 block-diagonal 4 x 4),
-//   S = ||H_128 x|| = sqrt(128) ||x||,
+//   u = W x  with  W = R_SO4 H_128  (unnormalised; R_SO4 block-diagonal 4 x 4),
+//   S = sqrt(128) ||x||  (= ||H_128 x||),
 //   code_i = #{k : u_i > t_k S}, stored norm float16(S / sqrt(128)),
 // which are the decisions of y = R_SO4 (H x / (||x|| sqrt d)) against t_k.
 //
-// The WHT is one matrix product per tile: D[128 x 128] (float32, TMEM) =
-// X[128 x 128] (float16, TMA-loaded, 128B-swizzled K-major) . H (the +-1
-// Sylvester matrix, float16, built once per CTA; H is symmetric, so its rows
-// serve as the K-major B operand).  Every product x_j H_ij is exact, and the
-// float32 sums are the butterflies' sums in another order.  The block maps,
-// the norm, the Lloyd-Max search and the packing run on the CUDA cores, two
-// threads per vector: the threads of warps w and w + 4 of an epilogue group
-// read the same TMEM lane (row) and take columns 0..63 and 64..127 (groups
-// 0, 1 and 2, 3 of the packed layout); both read the whole row once for the
-// norm, so they exchange nothing.
+// The rotation is one matrix product per tile: D[128 x 128] (float32, TMEM)
+// = X[128 x 128] (float16, TMA-loaded, 128B-swizzled K-major) . W^T, with W
+// split into float16 hi and lo parts (W = W_hi + W_lo to about 2^-22 of each
+// entry; both are K-major B operands, two products per K step).  W depends on
+// the head: the CTA builds it in shared memory at the start of each run of
+// tiles of one head (entry W[n][k] = sum_c R_i[n mod 4][c] H[4i + c][k],
+// i = n / 4, four products in float32).  The norm, the Lloyd-Max search and
+// the packing run on the CUDA cores, two threads per vector: the threads of
+// warps w and w + 4 of an epilogue group read the same TMEM lane (row) and
+// take columns 0..63 and 64..127 (groups 0, 1 and 2, 3 of the packed
+// layout).  Both take the norm from x itself, reading the vector's row of
+// the X tile in shared memory while the product runs (not from ||u||: the
+// float32 rotation parameters make R_SO4 orthogonal only to ~1e-7), so they
+// exchange nothing; the X stage is refilled once the product and the 256
+// epilogue threads of the tile's group have all released it.
 //
 // Warp roles (one CTA per SM, a contiguous range of tiles):
 //   warp 16, lane 0: TMA loads of X tiles into a 4-deep ring and the MMAs,
 //     each into TMEM buffer (tile & 1);
 //   warps 0-7 / 8-15: epilogue of the even / odd tiles (warp w reads TMEM
-//     sub-partition w % 4, rows 32 (w % 4) .. + 31, column half (w / 4) % 2);
-//     each warp keeps its own copy of the current head's block matrices, so
-//     no barrier spans warps.
+//     sub-partition w % 4, rows 32 (w % 4) .. + 31, column half (w / 4) % 2).
+// All threads build W between runs of tiles of different heads; a block
+// barrier closes each run, after every product of the run has been read back
+// (so none still reads W).
 // mbarriers: full[s] (TMA landed), empty[s] (the MMA that read stage s is
-// done), tfull[b] (TMEM buffer b holds a finished product), tempty[b] (the
+// done and the epilogue group has read its norms there), tfull[b] (TMEM buffer b holds a finished product), tempty[b] (the
 // epilogue group has read buffer b).  Every wait is bounded; a wait that
 // gives up sets the quantize error word and a CTA-wide flag, the loops stop,
 // the producer lets its copies and products finish (bounded), and the CTA
@@ -41,36 +47,14 @@ constexpr int kTqEpiWarps = 16;
 constexpr int kTqThreads = 32 * (kTqEpiWarps + 1);
 constexpr int kTqBlk = kTqRows * 128;           // one 64-column block of a tile (16 KB)
 constexpr int kTqXBytes = 2 * kTqBlk;           // one X tile (32 KB)
-constexpr int kTqHBytes = kTqD * kTqD * 2;      // H (32 KB)
-constexpr int kTqMatBytes = kTqD * 16;          // D/4 blocks x 16 floats (one head)
-constexpr int kTqOffX = kTqHBytes;
-constexpr int kTqOffMat = kTqOffX + kTqStages * kTqXBytes;
-constexpr int kTqOffBar = kTqOffMat + kTqEpiWarps * kTqMatBytes / 2;   // per epilogue warp: its two groups' matrices
+constexpr int kTqWBytes = kTqD * kTqD * 2;      // W_hi or W_lo (32 KB each)
+constexpr int kTqOffWlo = kTqWBytes;
+constexpr int kTqOffX = 2 * kTqWBytes;
+constexpr int kTqOffRot = kTqOffX + kTqStages * kTqXBytes;    // the head's 4 x 4 blocks, 32 x 16 floats
+constexpr int kTqOffBar = kTqOffRot + kTqD / 4 * 16 * 4;
 constexpr int kTqBars = 2 * kTqStages + 4;
 constexpr int kTqSmem = kTqOffBar + 8 * kTqBars + 16 + 1024;   // + the flag words, + alignment slack
 static_assert(kTqSmem <= 232448, "shared memory per CTA");
-
-// R_i alone (no H_4 factor, no 1/sqrt(d)) for nblk consecutive blocks from
-// params_head, in the layout of build_block_matrices: group g (counted from
-// the first block), block pair beta (blocks 8g + beta, 8g + beta + 4), entry
-// (j, c) -> float pair at mat[128 g + 32 beta + 2 (4 j + c)].
-template <bool FULL>
-__device__ void build_rotation_blocks(const float *params_head, float *mat, int tid, int nthreads, int nblk) {
-  for (int b = tid; b < nblk; b += nthreads) {
-    const Quat ql = load_quat(params_head + 8 * b);
-    const Quat qr = load_quat(params_head + 8 * b + 4);
-    const int g = b >> 3, r = b & 7, beta = r & 3, half = r >> 2;
-    float *out = mat + 128 * g + 32 * beta + half;
-    for (int c = 0; c < 4; ++c) {
-      const Quat e{c == 0 ? 1.f : 0.f, c == 1 ? 1.f : 0.f, c == 2 ? 1.f : 0.f, c == 3 ? 1.f : 0.f};
-      const Quat u = block_forward(ql, qr, e, FULL);
-      out[2 * (4 * 0 + c)] = u.w;
-      out[2 * (4 * 1 + c)] = u.x;
-      out[2 * (4 * 2 + c)] = u.y;
-      out[2 * (4 * 3 + c)] = u.z;
-    }
-  }
-}
 
 __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -83,6 +67,51 @@ __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]
       : "r"(taddr));
 }
 
+// Builds W_hi, W_lo (128B-swizzled K-major, row n, column k) for one head's
+// rotation parameters; all threads of the CTA take part.
+template <bool FULL>
+__device__ void build_rotation_operand(const float *params_head, float *rot, unsigned char *whi,
+                                       unsigned char *wlo, int tid) {
+  if (tid < kTqD / 4) {
+    const Quat ql = load_quat(params_head + 8 * tid);
+    const Quat qr = load_quat(params_head + 8 * tid + 4);
+    for (int c = 0; c < 4; ++c) {
+      const Quat e{c == 0 ? 1.f : 0.f, c == 1 ? 1.f : 0.f, c == 2 ? 1.f : 0.f, c == 3 ? 1.f : 0.f};
+      const Quat u = block_forward(ql, qr, e, FULL);   // column c of R_i
+      rot[16 * tid + 4 * 0 + c] = u.w;
+      rot[16 * tid + 4 * 1 + c] = u.x;
+      rot[16 * tid + 4 * 2 + c] = u.y;
+      rot[16 * tid + 4 * 3 + c] = u.z;
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < kTqD * kTqD / 8; idx += kTqThreads) {
+    const int n = idx / (kTqD / 8), k0 = 8 * (idx % (kTqD / 8));
+    const float *rr = rot + 16 * (n >> 2) + 4 * (n & 3);
+    const int j0 = n & ~3;
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      float w[2];
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int k = k0 + j + jj;
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc += (__popc((j0 + c) & k) & 1) ? -rr[c] : rr[c];
+        w[jj] = acc;
+      }
+      const __half2 h = __floats2half2_rn(w[0], w[1]);
+      const float2 hf = __half22float2(h);
+      const __half2 l = __floats2half2_rn(w[0] - hf.x, w[1] - hf.y);
+      hw[j / 2] = *reinterpret_cast<const uint32_t *>(&h);
+      lw[j / 2] = *reinterpret_cast<const uint32_t *>(&l);
+    }
+    *reinterpret_cast<uint4 *>(whi + tc_off(n, k0, kTqBlk)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4 *>(wlo + tc_off(n, k0, kTqBlk)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
 template <int BITS, bool FULL>
 __global__ void __launch_bounds__(kTqThreads, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap xmap, const QuantArgs args) {
@@ -91,9 +120,9 @@ __global__ void __launch_bounds__(kTqThreads, 1)
   extern __shared__ unsigned char smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char *smem = smem_raw + pad;
-  unsigned char *hmat = smem;
+  unsigned char *whi = smem, *wlo = smem + kTqOffWlo;
   unsigned char *xs = smem + kTqOffX;
-  float *mats = reinterpret_cast<float *>(smem + kTqOffMat);
+  float *rot = reinterpret_cast<float *>(smem + kTqOffRot);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTqOffBar);
   uint64_t *empty = full + kTqStages;
   uint64_t *tfull = empty + kTqStages;
@@ -102,28 +131,17 @@ __global__ void __launch_bounds__(kTqThreads, 1)
   volatile uint32_t *fail = tmem_slot + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = warp == kTqEpiWarps;
   const long long per_cta = (args.total_tiles + gridDim.x - 1) / gridDim.x;
   const long long tile_begin = static_cast<long long>(blockIdx.x) * per_cta;
   long long tile_end = tile_begin + per_cta;
   if (tile_end > args.total_tiles) tile_end = args.total_tiles;
   const int n_mine = tile_end > tile_begin ? static_cast<int>(tile_end - tile_begin) : 0;
 
-  // H_128 as float16 +-1 in the 128B-swizzled K-major layout (row n, column k).
-  for (int i = tid; i < kTqD * kTqD / 8; i += kTqThreads) {
-    const int n = i / (kTqD / 8), k0 = 8 * (i % (kTqD / 8));
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = (__popc(n & (k0 + 2 * j)) & 1) ? 0xBC00u : 0x3C00u;   // -1 / +1
-      const uint32_t hi = (__popc(n & (k0 + 2 * j + 1)) & 1) ? 0xBC00u : 0x3C00u;
-      w[j] = lo | (hi << 16);
-    }
-    *reinterpret_cast<uint4 *>(hmat + tc_off(n, k0, kTqBlk)) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
   if (tid == 0) {
     for (int s = 0; s < kTqStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 1 + 8 * 32);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -132,156 +150,181 @@ __global__ void __launch_bounds__(kTqThreads, 1)
     *fail = 0u;
     mbar_fence_init();
   }
-  if (warp == kTqEpiWarps) {
+  if (producer) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(256));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  fence_proxy_async_smem();   // H is read by the tensor core (async proxy)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kTqEpiWarps) {
-    // ---- producer: TMA loads and MMAs ----
-    if (lane == 0) {
-      auto load = [&](int i) {
-        const long long t = tile_begin + i;
-        const int head = static_cast<int>(t / args.tiles_per_head);
-        const int v0 = static_cast<int>((t % args.tiles_per_head) * kTqRows);
-        unsigned char *st = xs + (i % kTqStages) * kTqXBytes;
-        uint64_t *bar = &full[i % kTqStages];
-        mbar_arrive_expect_tx(bar, kTqXBytes);
-        tma_load_3d(st, &xmap, bar, 0, v0, head);
-        tma_load_3d(st + kTqBlk, &xmap, bar, 64, v0, head);
-      };
-      int loaded = 0, mma_done = 0;
-      for (; loaded < n_mine && loaded < kTqStages; ++loaded) load(loaded);
-      constexpr uint32_t idesc = tc_idesc(kTqRows, kTqD, 0);
-      const uint32_t h_s = smem_u32(hmat);
-      bool ok = true;
-      for (int i = 0; i < n_mine && ok; ++i) {
-        const int s = i % kTqStages, b = i & 1;
-        ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / kTqStages) & 1u);
-        if (ok && i >= 2) ok = mbar_wait_bounded(&tempty[b], static_cast<uint32_t>((i >> 1) - 1) & 1u);
-        if (*fail) ok = false;
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t x_s = smem_u32(xs + s * kTqXBytes);
+  // Producer state (lane 0 of the producer warp).
+  auto load = [&](int i) {
+    const long long t = tile_begin + i;
+    const int head = static_cast<int>(t / args.tiles_per_head);
+    const int v0 = static_cast<int>((t % args.tiles_per_head) * kTqRows);
+    unsigned char *st = xs + (i % kTqStages) * kTqXBytes;
+    uint64_t *bar = &full[i % kTqStages];
+    mbar_arrive_expect_tx(bar, kTqXBytes);
+    tma_load_3d(st, &xmap, bar, 0, v0, head);
+    tma_load_3d(st + kTqBlk, &xmap, bar, 64, v0, head);
+  };
+  int loaded = 0, mma_done = 0;
+  if (producer && lane == 0)
+    for (; loaded < n_mine && loaded < kTqStages; ++loaded) load(loaded);
+
+  // Epilogue geometry.
+  const int grp = warp >> 3, sub = warp & 3, half = (warp >> 2) & 1;
+  const int r = 32 * sub + lane;
+  const uint32_t t_row = tmem + 128 * grp + (static_cast<uint32_t>(32 * sub) << 16);
+
+  int i_seg = 0;
+  while (i_seg < n_mine) {
+    // One run of tiles of one head.
+    const int head = static_cast<int>((tile_begin + i_seg) / args.tiles_per_head);
+    long long seg_end_ll = static_cast<long long>(head + 1) * args.tiles_per_head - tile_begin;
+    const int seg_end = seg_end_ll < n_mine ? static_cast<int>(seg_end_ll) : n_mine;
+    build_rotation_operand<FULL>(args.params + static_cast<size_t>(head) * 2 * kTqD, rot, whi, wlo, tid);
+    fence_proxy_async_smem();   // W is read by the tensor core (async proxy)
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (producer) {
+      // ---- producer: MMAs of this run (TMA loads run ahead across runs) ----
+      if (lane == 0 && !*fail) {
+        constexpr uint32_t idesc = tc_idesc(kTqRows, kTqD, 0);
+        const uint32_t wh_s = smem_u32(whi), wl_s = smem_u32(wlo);
+        bool ok = true;
+        for (int i = i_seg; i < seg_end && ok; ++i) {
+          const int s = i % kTqStages, b = i & 1;
+          ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / kTqStages) & 1u);
+          if (ok && i >= 2) ok = mbar_wait_bounded(&tempty[b], static_cast<uint32_t>((i >> 1) - 1) & 1u);
+          if (*fail) ok = false;
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t x_s = smem_u32(xs + s * kTqXBytes);
 #pragma unroll
-        for (int ks = 0; ks < kTqD / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * kTqBlk + (ks & 3) * 32;
-          tc_mma(tmem + 128 * b, tc_desc(x_s + off, 16, 1024), tc_desc(h_s + off, 16, 1024), idesc,
-                 ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < kTqD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * kTqBlk + (ks & 3) * 32;
+            const uint64_t ad = tc_desc(x_s + off, 16, 1024);
+            tc_mma(tmem + 128 * b, ad, tc_desc(wh_s + off, 16, 1024), idesc, ks > 0 ? 1u : 0u);
+            tc_mma(tmem + 128 * b, ad, tc_desc(wl_s + off, 16, 1024), idesc, 1u);
+          }
+          tc_commit(&tfull[b]);
+          tc_commit(&empty[s]);
+          mma_done = i + 1;
+          // Refill the stage of tile i - 1 (its product was issued a step ago).
+          if (i >= 1 && loaded < n_mine) {
+            const int sp = (i - 1) % kTqStages;
+            ok = mbar_wait_bounded(&empty[sp], static_cast<uint32_t>((i - 1) / kTqStages) & 1u);
+            if (ok) load(loaded++);
+          }
         }
-        tc_commit(&tfull[b]);
-        tc_commit(&empty[s]);
-        mma_done = i + 1;
-        // Refill the stage of tile i - 1 (its product was issued a step ago).
-        if (i >= 1 && loaded < n_mine) {
-          const int sp = (i - 1) % kTqStages;
-          ok = mbar_wait_bounded(&empty[sp], static_cast<uint32_t>((i - 1) / kTqStages) & 1u);
-          if (ok) load(loaded++);
-        }
-      }
-      if (!ok) {
-        *fail = 1u;
-        atomicOr(&g_quant_error, kErrWaitTimeout);
-      }
-      // Let every copy and product this CTA issued finish before it exits.
-      for (int i = mma_done; i < loaded; ++i)
-        if (!mbar_wait_bounded(&full[i % kTqStages], static_cast<uint32_t>(i / kTqStages) & 1u)) break;
-      if (mma_done > 0)
-        mbar_wait_bounded(&empty[(mma_done - 1) % kTqStages], static_cast<uint32_t>((mma_done - 1) / kTqStages) & 1u);
-    }
-    __syncwarp();
-  } else {
-    // ---- epilogue: two threads per vector ----
-    const int grp = warp >> 3, sub = warp & 3, half = (warp >> 2) & 1;
-    const int r = 32 * sub + lane;
-    float *mat = mats + warp * (kTqMatBytes / 8);   // this warp's copy of groups 2 half, 2 half + 1
-    const uint32_t mat_s = smem_u32(mat);
-    const uint32_t t_row = tmem + 128 * grp + (static_cast<uint32_t>(32 * sub) << 16);
-    int cur_head = -1;
-    for (int i = grp; i < n_mine; i += 2) {
-      const long long t = tile_begin + i;
-      const int head = static_cast<int>(t / args.tiles_per_head);
-      if (head != cur_head) {
-        __syncwarp();   // the warp is done with the previous head's matrices
-        build_rotation_blocks<FULL>(args.params + static_cast<size_t>(head) * 2 * kTqD + 8 * 16 * half, mat,
-                                    lane, 32, kTqD / 8);
-        __syncwarp();
-        cur_head = head;
-      }
-      const bool ok = mbar_wait_bounded(&tfull[grp], static_cast<uint32_t>(i >> 1) & 1u);
-      if (__any_sync(0xffffffffu, !ok) || *fail) {
-        if (lane == 0) {
+        if (!ok) {
           *fail = 1u;
           atomicOr(&g_quant_error, kErrWaitTimeout);
         }
-        break;
       }
-      tc_fence_after();
-      // Pass 1: the norm, S^2 = sum (H x)_i^2 over the whole row.
-      uint64_t ss2 = f2_pack(0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tc_ld32_nowait(t_row + 32 * c, v);
-        tc_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const uint64_t p = f2_pack(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-          ss2 = f2_fma(p, p, ss2);
+      __syncwarp();
+    } else {
+      // ---- epilogue of this run's tiles of parity grp: two threads per vector ----
+      for (int i = i_seg + ((i_seg & 1) != grp ? 1 : 0); i < seg_end; i += 2) {
+        const long long t = tile_begin + i;
+        const int s = i % kTqStages;
+        // The norm from the X tile (row r), while the product runs.
+        bool ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / kTqStages) & 1u);
+        if (__any_sync(0xffffffffu, !ok) || *fail) {
+          if (lane == 0) {
+            *fail = 1u;
+            atomicOr(&g_quant_error, kErrWaitTimeout);
+          }
+          break;
         }
-      }
-      float s_lo, s_hi;
-      f2_unpack(ss2, s_lo, s_hi);
-      const float S2 = s_lo + s_hi;
-      const float S = sqrtf(S2);
-      const float big = search_scale(S);
-      float tb[NPOS];
+        const uint32_t xrow = smem_u32(xs + s * kTqXBytes);
+        uint64_t ss2 = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < NPOS; ++j) tb[j] = -(args.tau[j] * S) * big;
-      const long long v = (t % args.tiles_per_head) * kTqRows + r;
-      const bool live = v < args.n_vec;
-      const long long idx = static_cast<long long>(head) * args.out_head_stride + v;
-      // Pass 2: this thread's two 32-element groups, one at a time, held as
-      // pairs (e, e + 16).
+        for (int c = 0; c < kTqD / 8; ++c) {
+          const uint4 q = lds128(xrow + tc_off(r, 8 * c, kTqBlk));
+          const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-      for (int G = 0; G < 2; ++G) {
-        const int gi = 2 * half + G;
-        uint32_t va[32];
-        tc_ld32_nowait(t_row + 32 * gi, va);
-        tc_wait_ld();
-        if (G == 1) {
-          // every read of this buffer is done: it is free for tile i + 2
-          tc_fence_before();
-          mbar_arrive(&tempty[grp]);
-        }
-        uint64_t xp[kGP];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) xp[e] = f2_pack(__uint_as_float(va[e]), __uint_as_float(va[e + 16]));
-        apply_group_matrices(xp, 0, mat_s + 512 * G);
-        if (live) {
-          uint32_t w[GB / 4];
-          quantize_group<BITS>(xp, 0, tb, big, w);
-          uint8_t *gd = args.codes + idx * PB + gi * GB;
-          if constexpr (GB == 16) {
-            *reinterpret_cast<uint4 *>(gd) = make_uint4(w[0], w[1], w[2], w[3]);
-          } else if constexpr (GB == 8) {
-            *reinterpret_cast<uint2 *>(gd) = make_uint2(w[0], w[1]);
-          } else {
-#pragma unroll
-            for (int k = 0; k < GB / 4; ++k) reinterpret_cast<uint32_t *>(gd)[k] = w[k];
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&qw[j]));
+            const uint64_t p = f2_pack(f.x, f.y);
+            ss2 = f2_fma(p, p, ss2);
           }
         }
+        mbar_arrive(&empty[s]);   // this thread is done with the stage
+        float s_lo, s_hi;
+        f2_unpack(ss2, s_lo, s_hi);
+        const float ssq = s_lo + s_hi;                 // ||x||^2
+        const float S = sqrtf(ssq * static_cast<float>(kTqD));
+        const float big = search_scale(S);
+        float tb[NPOS];
+#pragma unroll
+        for (int j = 0; j < NPOS; ++j) tb[j] = -(args.tau[j] * S) * big;
+        ok = mbar_wait_bounded(&tfull[grp], static_cast<uint32_t>(i >> 1) & 1u);
+        if (__any_sync(0xffffffffu, !ok) || *fail) {
+          if (lane == 0) {
+            *fail = 1u;
+            atomicOr(&g_quant_error, kErrWaitTimeout);
+          }
+          break;
+        }
+        tc_fence_after();
+        const long long v = (t % args.tiles_per_head) * kTqRows + r;
+        const bool live = v < args.n_vec;
+        const long long idx = static_cast<long long>(head) * args.out_head_stride + v;
+        // Pass 2: this thread's two 32-element groups, one at a time, held as
+        // pairs (e, e + 16).
+#pragma unroll
+        for (int G = 0; G < 2; ++G) {
+          const int gi = 2 * half + G;
+          uint32_t va[32];
+          tc_ld32_nowait(t_row + 32 * gi, va);
+          tc_wait_ld();
+          if (G == 1) {
+            // every read of this buffer is done: it is free for tile i + 2
+            tc_fence_before();
+            mbar_arrive(&tempty[grp]);
+          }
+          if (live) {
+            uint64_t xp[kGP];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xp[e] = f2_pack(__uint_as_float(va[e]), __uint_as_float(va[e + 16]));
+            uint32_t w[GB / 4];
+            quantize_group<BITS>(xp, 0, tb, big, w);
+            uint8_t *gd = args.codes + idx * PB + gi * GB;
+            if constexpr (GB == 16) {
+              *reinterpret_cast<uint4 *>(gd) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else if constexpr (GB == 8) {
+              *reinterpret_cast<uint2 *>(gd) = make_uint2(w[0], w[1]);
+            } else {
+#pragma unroll
+              for (int k = 0; k < GB / 4; ++k) reinterpret_cast<uint32_t *>(gd)[k] = w[k];
+            }
+          }
+        }
+        if (live && half == 0) args.norms[idx] = __half_as_ushort(__float2half_rn(sqrtf(ssq)));
       }
-      if (live && half == 0) args.norms[idx] = __half_as_ushort(__float2half_rn(sqrtf(S2 * (1.f / kTqD))));
     }
+    // Every product of the run has been read back: W may be rebuilt.
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (*fail) break;
+    i_seg = seg_end;
+  }
+  if (producer && lane == 0) {
+    // Let every copy and product this CTA issued finish before it exits.
+    for (int i = mma_done; i < loaded; ++i)
+      if (!mbar_wait_bounded(&full[i % kTqStages], static_cast<uint32_t>(i / kTqStages) & 1u)) break;
+    if (mma_done > 0)
+      mbar_wait_bounded(&empty[(mma_done - 1) % kTqStages], static_cast<uint32_t>((mma_done - 1) / kTqStages) & 1u);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kTqEpiWarps) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+  if (producer) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
 }
