@@ -27,7 +27,8 @@
 //
 // Warp roles (one CTA per SM, a contiguous range of tiles):
 //   warp 16, lane 0: TMA loads of X tiles into a 4-deep ring and the MMAs,
-//     each into TMEM buffer (tile & 1);
+//     each into TMEM buffer (tile & 3), so that the products run up to two
+//     tiles of each group ahead of the epilogue;
 //   warps 0-7 / 8-15: epilogue of the even / odd tiles (warp w reads TMEM
 //     sub-partition w % 4, rows 32 (w % 4) .. + 31, column half (w / 4) % 2).
 // All threads build W between runs of tiles of different heads; a block
@@ -52,7 +53,8 @@ constexpr int kTqOffWlo = kTqWBytes;
 constexpr int kTqOffX = 2 * kTqWBytes;
 constexpr int kTqOffRot = kTqOffX + kTqStages * kTqXBytes;    // the head's 4 x 4 blocks, 32 x 16 floats
 constexpr int kTqOffBar = kTqOffRot + kTqD / 4 * 16 * 4;
-constexpr int kTqBars = 2 * kTqStages + 4;
+constexpr int kTqBufs = 4;                      // TMEM buffers of 128 columns
+constexpr int kTqBars = 2 * kTqStages + 2 * kTqBufs;
 constexpr int kTqSmem = kTqOffBar + 8 * kTqBars + 16 + 1024;   // + the flag words, + alignment slack
 static_assert(kTqSmem <= 232448, "shared memory per CTA");
 
@@ -126,8 +128,8 @@ __global__ void __launch_bounds__(kTqThreads, 1)
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTqOffBar);
   uint64_t *empty = full + kTqStages;
   uint64_t *tfull = empty + kTqStages;
-  uint64_t *tempty = tfull + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  uint64_t *tempty = tfull + kTqBufs;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + kTqBufs);
   volatile uint32_t *fail = tmem_slot + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1 + 8 * 32);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kTqBufs; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 8 * 32);
     }
@@ -152,7 +154,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
   }
   if (producer) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(256));
+                 "r"(128 * kTqBufs));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
   // Epilogue geometry.
   const int grp = warp >> 3, sub = warp & 3, half = (warp >> 2) & 1;
   const int r = 32 * sub + lane;
-  const uint32_t t_row = tmem + 128 * grp + (static_cast<uint32_t>(32 * sub) << 16);
+  const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * sub) << 16);
 
   int i_seg = 0;
   while (i_seg < n_mine) {
@@ -199,9 +201,9 @@ __global__ void __launch_bounds__(kTqThreads, 1)
         const uint32_t wh_s = smem_u32(whi), wl_s = smem_u32(wlo);
         bool ok = true;
         for (int i = i_seg; i < seg_end && ok; ++i) {
-          const int s = i % kTqStages, b = i & 1;
+          const int s = i % kTqStages, b = i % kTqBufs;
           ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / kTqStages) & 1u);
-          if (ok && i >= 2) ok = mbar_wait_bounded(&tempty[b], static_cast<uint32_t>((i >> 1) - 1) & 1u);
+          if (ok && i >= kTqBufs) ok = mbar_wait_bounded(&tempty[b], static_cast<uint32_t>(i / kTqBufs - 1) & 1u);
           if (*fail) ok = false;
           if (!ok) break;
           tc_fence_after();
@@ -265,7 +267,9 @@ __global__ void __launch_bounds__(kTqThreads, 1)
         float tb[NPOS];
 #pragma unroll
         for (int j = 0; j < NPOS; ++j) tb[j] = -(args.tau[j] * S) * big;
-        ok = mbar_wait_bounded(&tfull[grp], static_cast<uint32_t>(i >> 1) & 1u);
+        const int b = i % kTqBufs;
+        const uint32_t t_row = t_lane + 128 * b;
+        ok = mbar_wait_bounded(&tfull[b], static_cast<uint32_t>(i / kTqBufs) & 1u);
         if (__any_sync(0xffffffffu, !ok) || *fail) {
           if (lane == 0) {
             *fail = 1u;
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
           if (G == 1) {
             // every read of this buffer is done: it is free for tile i + 2
             tc_fence_before();
-            mbar_arrive(&tempty[grp]);
+            mbar_arrive(&tempty[b]);
           }
           if (live) {
             uint64_t xp[kGP];
@@ -326,5 +330,5 @@ __global__ void __launch_bounds__(kTqThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (producer) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+  if (producer) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128 * kTqBufs));
 }
