@@ -314,13 +314,16 @@ __device__ __forceinline__ float search_scale(float norm) {
 // L/2 + m for y > 0 and L/2 - 1 - m otherwise, i.e. (L/2 - 1/2) + sg (m + 1/2)
 // with sg = +-1.  The packing accumulates code * w for the field weight w of
 // each position as one FMA, (sg w) (m + 1/2), onto the constant
-// 2^22 + (L/2 - 1/2) sum w; sg w is w with its sign bit set from y by the
-// integer pipe.  Every partial sum is a multiple of 1/2 in [2^22, 2^23),
+// 2^22 + (L/2 - 1/2) sum w; sg w is w with y's sign bit ORed in by one
+// integer logic op.  That counts +0 as positive, which only a zero vector
+// produces (any other exact zero lies on the threshold 0 itself, where either
+// code is nearest): for a zero vector, zmask = 0x80000000 makes every weight
+// negative, so all its codes are L/2 - 1 as the rule #{k : y > t_k} gives.  Every partial sum is a multiple of 1/2 in [2^22, 2^23),
 // where float32 steps by 1/2, so all of it is exact, and the packed field
 // is the float's mantissa shifted right by one bit.
 template <int BITS, int NP>
 __device__ __forceinline__ void quantize_group(const uint64_t (&xp)[NP], int base,
-                                               const float *tb, float big, uint32_t *w) {
+                                               const float *tb, float big, uint32_t zmask, uint32_t *w) {
   constexpr int L = 1 << BITS, NPOS = L / 2 - 1;
   constexpr int PER_HALF = 16 / BITS == 5 ? 4 : 16 / BITS;   // codes per 16-bit half (3 bits: 4-bit fields)
   constexpr int FIELD = BITS == 3 ? 4 : BITS;
@@ -343,10 +346,10 @@ __device__ __forceinline__ void quantize_group(const uint64_t (&xp)[NP], int bas
 #pragma unroll
       for (int k = 1; k < NPOS; ++k) m = f2_add(m, f2_pack(fma_sat(a0, big, tb[k]), fma_sat(a1, big, tb[k])));
       m = f2_add(m, half2);
-      // sg w: the field weight, negative unless y > 0 (+-0 count as not positive)
-      const uint32_t wb = __float_as_uint(static_cast<float>(1u << (FIELD * j)));
-      const uint32_t s0 = static_cast<int>(__float_as_uint(y0)) > 0 ? wb : (wb | 0x80000000u);
-      const uint32_t s1 = static_cast<int>(__float_as_uint(y1)) > 0 ? wb : (wb | 0x80000000u);
+      // sg w: the field weight with y's sign (negative for a zero vector)
+      const uint32_t wb = __float_as_uint(static_cast<float>(1u << (FIELD * j))) | zmask;
+      const uint32_t s0 = wb | (__float_as_uint(y0) & 0x80000000u);
+      const uint32_t s1 = wb | (__float_as_uint(y1) & 0x80000000u);
       acc = f2_fma(f2_pack(__uint_as_float(s0), __uint_as_float(s1)), m, acc);
     }
     float fl, fh;
@@ -581,7 +584,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
 #pragma unroll
       for (int G = 0; G < 2; ++G) {
         uint32_t w[C::GB / 4];
-        quantize_group<BITS>(xp, kGP * G, tb, big, w);
+        quantize_group<BITS>(xp, kGP * G, tb, big, norm > 0.f ? 0u : 0x80000000u, w);
         uint8_t *gd = dst + grp[G] * C::GB;
         if constexpr (C::GB == 16) {
           *reinterpret_cast<uint4 *>(gd) = make_uint4(w[0], w[1], w[2], w[3]);

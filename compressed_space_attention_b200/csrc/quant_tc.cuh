@@ -19,11 +19,14 @@
 // the packing run on the CUDA cores, two threads per vector: the threads of
 // warps w and w + 4 of an epilogue group read the same TMEM lane (row) and
 // take columns 0..63 and 64..127 (groups 0, 1 and 2, 3 of the packed
-// layout).  Both take the norm from x itself, reading the vector's row of
+// layout).  They take the norm from x itself, reading the vector's row of
 // the X tile in shared memory while the product runs (not from ||u||: the
-// float32 rotation parameters make R_SO4 orthogonal only to ~1e-7), so they
-// exchange nothing; the X stage is refilled once the product and the 256
-// epilogue threads of the tile's group have all released it.
+// float32 rotation parameters make R_SO4 orthogonal only to ~1e-7): each
+// sums the squares of its 64 columns and the two swap their partial sums
+// through shared memory, with an mbarrier per warp and a bounded wait (both
+// add the halves in the same order, so both hold the same norm); the X stage
+// is refilled once the product and the 256 epilogue threads of the tile's
+// group have all released it.
 //
 // Warp roles (one CTA per SM, a contiguous range of tiles):
 //   warp 16, lane 0: TMA loads of X tiles into a 4-deep ring and the MMAs,
@@ -54,8 +57,10 @@ constexpr int kTqOffX = 2 * kTqWBytes;
 constexpr int kTqOffRot = kTqOffX + kTqStages * kTqXBytes;    // the head's 4 x 4 blocks, 32 x 16 floats
 constexpr int kTqOffBar = kTqOffRot + kTqD / 4 * 16 * 4;
 constexpr int kTqBufs = 4;                      // TMEM buffers of 128 columns
-constexpr int kTqBars = 2 * kTqStages + 2 * kTqBufs;
-constexpr int kTqSmem = kTqOffBar + 8 * kTqBars + 16 + 1024;   // + the flag words, + alignment slack
+constexpr int kTqOffXch = kTqOffBar;            // partial norms [group][half][sub][slot][lane]
+constexpr int kTqXchBytes = 2 * 2 * 4 * 2 * 32 * 4;
+constexpr int kTqBars = 2 * kTqStages + 2 * kTqBufs + 2 * kTqEpiWarps;   // + two per epilogue warp
+constexpr int kTqSmem = kTqOffBar + kTqXchBytes + 8 * kTqBars + 16 + 1024;   // + the flag words, + alignment slack
 static_assert(kTqSmem <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
@@ -125,11 +130,13 @@ __global__ void __launch_bounds__(kTqThreads, 1)
   unsigned char *whi = smem, *wlo = smem + kTqOffWlo;
   unsigned char *xs = smem + kTqOffX;
   float *rot = reinterpret_cast<float *>(smem + kTqOffRot);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTqOffBar);
+  float *xch = reinterpret_cast<float *>(smem + kTqOffXch);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTqOffBar + kTqXchBytes);
   uint64_t *empty = full + kTqStages;
   uint64_t *tfull = empty + kTqStages;
   uint64_t *tempty = tfull + kTqBufs;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + kTqBufs);
+  uint64_t *pbar = tempty + kTqBufs;   // [epilogue warp][slot]: its partial norms are written
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pbar + 2 * kTqEpiWarps);
   volatile uint32_t *fail = tmem_slot + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -149,6 +156,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 8 * 32);
     }
+    for (int w = 0; w < 2 * kTqEpiWarps; ++w) mbar_init(&pbar[w], 32);
     *fail = 0u;
     mbar_fence_init();
   }
@@ -248,7 +256,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
         const uint32_t xrow = smem_u32(xs + s * kTqXBytes);
         uint64_t ss2 = f2_pack(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < kTqD / 8; ++c) {
+        for (int c = 8 * half; c < 8 * half + 8; ++c) {   // this thread's 64 columns
           const uint4 q = lds128(xrow + tc_off(r, 8 * c, kTqBlk));
           const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
@@ -261,7 +269,27 @@ __global__ void __launch_bounds__(kTqThreads, 1)
         mbar_arrive(&empty[s]);   // this thread is done with the stage
         float s_lo, s_hi;
         f2_unpack(ss2, s_lo, s_hi);
-        const float ssq = s_lo + s_hi;                 // ||x||^2
+        // Swap the partial sums with the partner warp.  Slot (and mbarrier)
+        // k & 1 for the group's k-th tile: the partner reads slot k & 1 before
+        // it arrives for tile k + 1, and this warp writes that slot again only
+        // at tile k + 2, after waiting for that arrival; each mbarrier moves one
+        // phase per two tiles, so a wait cannot see a phase two ahead.
+        const int k = i >> 1, slot = k & 1;
+        float *mine = xch + (((grp * 2 + half) * 4 + sub) * 2 + slot) * 32;
+        const float *theirs = xch + (((grp * 2 + (half ^ 1)) * 4 + sub) * 2 + slot) * 32;
+        mine[lane] = s_lo + s_hi;
+        mbar_arrive(&pbar[2 * warp + slot]);
+        ok = mbar_wait_bounded(&pbar[2 * (warp ^ 4) + slot], static_cast<uint32_t>(k >> 1) & 1u);
+        if (__any_sync(0xffffffffu, !ok) || *fail) {
+          if (lane == 0) {
+            *fail = 1u;
+            atomicOr(&g_quant_error, kErrWaitTimeout);
+          }
+          break;
+        }
+        const float other = theirs[lane];
+        const float ssq = half == 0 ? mine[lane] + other : other + mine[lane];   // ||x||^2, same order in both
+        const uint32_t zmask = ssq > 0.f ? 0u : 0x80000000u;
         const float S = sqrtf(ssq * static_cast<float>(kTqD));
         const float big = search_scale(S);
         float tb[NPOS];
@@ -299,7 +327,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) xp[e] = f2_pack(__uint_as_float(va[e]), __uint_as_float(va[e + 16]));
             uint32_t w[GB / 4];
-            quantize_group<BITS>(xp, 0, tb, big, w);
+            quantize_group<BITS>(xp, 0, tb, big, zmask, w);
             uint8_t *gd = args.codes + idx * PB + gi * GB;
             if constexpr (GB == 16) {
               *reinterpret_cast<uint4 *>(gd) = make_uint4(w[0], w[1], w[2], w[3]);

@@ -103,6 +103,27 @@ def test_edge_cases_sizes_zeros_magnitudes():
         assert gn[0, 0] == 0
 
 
+@pytest.mark.parametrize("d,dtype", [(128, np.float16), (128, np.float32), (256, np.float16)])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("variant", [O.FULL, O.FAST])
+def test_zero_vectors_get_the_middle_negative_code(d, dtype, bits, variant):
+    """A zero vector has y = 0, so code = #{k : 0 > t_k} = L/2 - 1 at every
+    coordinate (RotaryQuant Algorithm 1 with the threshold rule; the oracle's
+    reading for a zero norm), and a zero norm: on every kernel path, next to
+    ordinary vectors in the same tile."""
+    params = O.make_params(d, variant, seed=3)
+    x = synth.unit_vectors(200, d, seed=d + bits, dtype=dtype)
+    for j in (0, 37, 128, 199):
+        x[0, j] = 0
+    gc, gn = _gpu_quantize(x, params, bits, variant)
+    codes = O.bitunpack(gc, bits, d)
+    for j in (0, 37, 128, 199):
+        np.testing.assert_array_equal(codes[0, j], (1 << bits) // 2 - 1)
+        assert gn[0, j] == 0
+    oc, on, y = O.quantize(x.astype(np.float64), params, bits, variant, return_rotated=True)
+    assert check_codes(gc, oc, y, bits, d) <= 2
+
+
 def test_empty_is_noop():
     x = torch.zeros((2, 0, 128), dtype=torch.float16, device=DEV)
     p = torch.from_numpy(O.make_params(128, O.FULL, 1, 2)).to(DEV)
