@@ -29,14 +29,15 @@
 // group have all released it.
 //
 // Warp roles (one CTA per SM, a contiguous range of tiles):
-//   warp 16, lane 0: TMA loads of X tiles into a 4-deep ring and the MMAs,
-//     each into TMEM buffer (tile & 3), so that the products run up to two
-//     tiles of each group ahead of the epilogue;
+//   warp 17, lane 0: TMA loads of X tiles into a 4-deep ring, running ahead
+//     across runs of heads (it takes no part in the run barriers);
+//   warp 16, lane 0: the MMAs, each tile into TMEM buffer (tile & 3), so that
+//     the products run up to two tiles of each group ahead of the epilogue;
 //   warps 0-7 / 8-15: epilogue of the even / odd tiles (warp w reads TMEM
 //     sub-partition w % 4, rows 32 (w % 4) .. + 31, column half (w / 4) % 2).
-// All threads build W between runs of tiles of different heads; a block
-// barrier closes each run, after every product of the run has been read back
-// (so none still reads W).
+// The epilogue and MMA warps build W between runs of tiles of different heads;
+// a barrier of those 17 warps closes each run, after every product of the
+// run has been read back (so none still reads W).
 // mbarriers: full[s] (TMA landed), empty[s] (the MMA that read stage s is
 // done and the epilogue group has read its norms there), tfull[b] (TMEM buffer b holds a finished product), tempty[b] (the
 // epilogue group has read buffer b).  Every wait is bounded; a wait that
@@ -48,7 +49,9 @@ constexpr int kTqRows = 128;                    // vectors per tile (M, one TMEM
 constexpr int kTqD = 128;
 constexpr int kTqStages = 4;
 constexpr int kTqEpiWarps = 16;
-constexpr int kTqThreads = 32 * (kTqEpiWarps + 1);
+constexpr int kTqMmaWarp = kTqEpiWarps, kTqTmaWarp = kTqEpiWarps + 1;
+constexpr int kTqThreads = 32 * (kTqEpiWarps + 2);
+constexpr int kTqRunThreads = 32 * (kTqEpiWarps + 1);   // the run barrier: epilogue and MMA warps
 constexpr int kTqBlk = kTqRows * 128;           // one 64-column block of a tile (16 KB)
 constexpr int kTqXBytes = 2 * kTqBlk;           // one X tile (32 KB)
 constexpr int kTqWBytes = kTqD * kTqD * 2;      // W_hi or W_lo (32 KB each)
@@ -78,7 +81,7 @@ __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]
 // rotation parameters; all threads of the CTA take part.
 template <bool FULL>
 __device__ void build_rotation_operand(const float *params_head, float *rot, unsigned char *whi,
-                                       unsigned char *wlo, int tid) {
+                                       unsigned char *wlo, int tid) {   // tid < kTqRunThreads
   if (tid < kTqD / 4) {
     const Quat ql = load_quat(params_head + 8 * tid);
     const Quat qr = load_quat(params_head + 8 * tid + 4);
@@ -91,8 +94,8 @@ __device__ void build_rotation_operand(const float *params_head, float *rot, uns
       rot[16 * tid + 4 * 3 + c] = u.z;
     }
   }
-  __syncthreads();
-  for (int idx = tid; idx < kTqD * kTqD / 8; idx += kTqThreads) {
+  named_barrier(1, kTqRunThreads);
+  for (int idx = tid; idx < kTqD * kTqD / 8; idx += kTqRunThreads) {
     const int n = idx / (kTqD / 8), k0 = 8 * (idx % (kTqD / 8));
     const float *rr = rot + 16 * (n >> 2) + 4 * (n & 3);
     const int j0 = n & ~3;
@@ -140,7 +143,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
   volatile uint32_t *fail = tmem_slot + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool producer = warp == kTqEpiWarps;
+  const bool producer = warp == kTqMmaWarp, loader = warp == kTqTmaWarp;
   const long long per_cta = (args.total_tiles + gridDim.x - 1) / gridDim.x;
   const long long tile_begin = static_cast<long long>(blockIdx.x) * per_cta;
   long long tile_end = tile_begin + per_cta;
@@ -181,17 +184,40 @@ __global__ void __launch_bounds__(kTqThreads, 1)
     tma_load_3d(st, &xmap, bar, 0, v0, head);
     tma_load_3d(st + kTqBlk, &xmap, bar, 64, v0, head);
   };
-  int loaded = 0, mma_done = 0;
-  if (producer && lane == 0)
-    for (; loaded < n_mine && loaded < kTqStages; ++loaded) load(loaded);
+  int mma_done = 0;
 
   // Epilogue geometry.
   const int grp = warp >> 3, sub = warp & 3, half = (warp >> 2) & 1;
   const int r = 32 * sub + lane;
   const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * sub) << 16);
 
+  if (loader) {
+    // ---- TMA loads: stage s is refilled once the product and the norms of
+    // the tile before have released it ----
+    if (lane == 0) {
+      int loaded = 0;
+      bool ok = true;
+      for (; loaded < n_mine; ++loaded) {
+        const int s = loaded % kTqStages;
+        if (loaded >= kTqStages)
+          ok = mbar_wait_bounded(&empty[s], static_cast<uint32_t>(loaded / kTqStages - 1) & 1u);
+        if (*fail) ok = false;
+        if (!ok) break;
+        load(loaded);
+      }
+      if (!ok) {
+        *fail = 1u;
+        atomicOr(&g_quant_error, kErrWaitTimeout);
+      }
+      // every copy issued lands before the CTA may exit
+      for (int j = loaded - kTqStages < 0 ? 0 : loaded - kTqStages; j < loaded; ++j)
+        if (!mbar_wait_bounded(&full[j % kTqStages], static_cast<uint32_t>(j / kTqStages) & 1u)) break;
+    }
+    __syncwarp();
+  }
+
   int i_seg = 0;
-  while (i_seg < n_mine) {
+  while (!loader && i_seg < n_mine) {
     // One run of tiles of one head.
     const int head = static_cast<int>((tile_begin + i_seg) / args.tiles_per_head);
     long long seg_end_ll = static_cast<long long>(head + 1) * args.tiles_per_head - tile_begin;
@@ -199,7 +225,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
     build_rotation_operand<FULL>(args.params + static_cast<size_t>(head) * 2 * kTqD, rot, whi, wlo, tid);
     fence_proxy_async_smem();   // W is read by the tensor core (async proxy)
     tc_fence_before();
-    __syncthreads();
+    named_barrier(1, kTqRunThreads);
     tc_fence_after();
 
     if (producer) {
@@ -226,12 +252,6 @@ __global__ void __launch_bounds__(kTqThreads, 1)
           tc_commit(&tfull[b]);
           tc_commit(&empty[s]);
           mma_done = i + 1;
-          // Refill the stage of tile i - 1 (its product was issued a step ago).
-          if (i >= 1 && loaded < n_mine) {
-            const int sp = (i - 1) % kTqStages;
-            ok = mbar_wait_bounded(&empty[sp], static_cast<uint32_t>((i - 1) / kTqStages) & 1u);
-            if (ok) load(loaded++);
-          }
         }
         if (!ok) {
           *fail = 1u;
@@ -344,17 +364,14 @@ __global__ void __launch_bounds__(kTqThreads, 1)
     }
     // Every product of the run has been read back: W may be rebuilt.
     tc_fence_before();
-    __syncthreads();
+    named_barrier(1, kTqRunThreads);
     tc_fence_after();
     if (*fail) break;
     i_seg = seg_end;
   }
-  if (producer && lane == 0) {
-    // Let every copy and product this CTA issued finish before it exits.
-    for (int i = mma_done; i < loaded; ++i)
-      if (!mbar_wait_bounded(&full[i % kTqStages], static_cast<uint32_t>(i / kTqStages) & 1u)) break;
-    if (mma_done > 0)
-      mbar_wait_bounded(&empty[(mma_done - 1) % kTqStages], static_cast<uint32_t>((mma_done - 1) / kTqStages) & 1u);
+  if (producer && lane == 0 && mma_done > 0) {
+    // The last products finish before the CTA frees the tensor memory.
+    mbar_wait_bounded(&tfull[(mma_done - 1) % kTqBufs], static_cast<uint32_t>((mma_done - 1) / kTqBufs) & 1u);
   }
   tc_fence_before();
   __syncthreads();
