@@ -342,10 +342,25 @@ __device__ __forceinline__ void quantize_group(const uint64_t (&xp)[NP], int bas
       f2_unpack(xp[base + p], y0, y1);
       const float a0 = fabsf(y0), a1 = fabsf(y1);
       // m + 1/2
-      uint64_t m = f2_pack(fma_sat(a0, big, tb[0]), fma_sat(a1, big, tb[0]));
+      uint64_t m;
+      if constexpr (NPOS == 3) {
+        // Two levels: s2 = [|y| > t_2], then |y| against t_3 if s2 else t_1
+        // (the thresholds increase, so m = 2 s2 + [|y| > that threshold]).
+        // The selected threshold s2 t_3 + (1 - s2) t_1 is exact: one of the
+        // two products is zero.
+        const uint64_t s2 = f2_pack(fma_sat(a0, big, tb[1]), fma_sat(a1, big, tb[1]));
+        const uint64_t tsel = f2_fma(s2, f2_pack(tb[2], tb[2]),
+                                     f2_fma(s2, f2_pack(-tb[0], -tb[0]), f2_pack(tb[0], tb[0])));
+        float t0, t1;
+        f2_unpack(tsel, t0, t1);
+        const uint64_t s13 = f2_pack(fma_sat(a0, big, t0), fma_sat(a1, big, t1));
+        m = f2_fma(s2, f2_pack(2.f, 2.f), f2_add(s13, half2));
+      } else {
+        m = f2_pack(fma_sat(a0, big, tb[0]), fma_sat(a1, big, tb[0]));
 #pragma unroll
-      for (int k = 1; k < NPOS; ++k) m = f2_add(m, f2_pack(fma_sat(a0, big, tb[k]), fma_sat(a1, big, tb[k])));
-      m = f2_add(m, half2);
+        for (int k = 1; k < NPOS; ++k) m = f2_add(m, f2_pack(fma_sat(a0, big, tb[k]), fma_sat(a1, big, tb[k])));
+        m = f2_add(m, half2);
+      }
       // sg w: the field weight with y's sign (negative for a zero vector)
       const uint32_t wb = __float_as_uint(static_cast<float>(1u << (FIELD * j))) | zmask;
       const uint32_t s0 = wb | (__float_as_uint(y0) & 0x80000000u);

@@ -329,26 +329,33 @@ __global__ void __launch_bounds__(kTqThreads, 1)
         const long long v = (t % args.tiles_per_head) * kTqRows + r;
         const bool live = v < args.n_vec;
         const long long idx = static_cast<long long>(head) * args.out_head_stride + v;
-        // Pass 2: this thread's two 32-element groups, one at a time, held as
-        // pairs (e, e + 16).
+        // This thread's two 32-element groups, held as pairs (e, e + 16); the
+        // second group's tensor-memory read is in flight while the first is
+        // quantised (the first group's words are paired before it is issued,
+        // so that 96 registers hold both).
+        uint64_t xp[kGP];
+        {
+          uint32_t va[32];
+          tc_ld32_nowait(t_row + 64 * half, va);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) xp[e] = f2_pack(__uint_as_float(va[e]), __uint_as_float(va[e + 16]));
+        }
+        uint32_t vb[32];
+        tc_ld32_nowait(t_row + 64 * half + 32, vb);
 #pragma unroll
         for (int G = 0; G < 2; ++G) {
-          const int gi = 2 * half + G;
-          uint32_t va[32];
-          tc_ld32_nowait(t_row + 32 * gi, va);
-          tc_wait_ld();
           if (G == 1) {
-            // every read of this buffer is done: it is free for tile i + 2
+            tc_wait_ld();
             tc_fence_before();
-            mbar_arrive(&tempty[b]);
+            mbar_arrive(&tempty[b]);   // every read of this buffer is done: free for tile i + 4
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xp[e] = f2_pack(__uint_as_float(vb[e]), __uint_as_float(vb[e + 16]));
           }
           if (live) {
-            uint64_t xp[kGP];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) xp[e] = f2_pack(__uint_as_float(va[e]), __uint_as_float(va[e + 16]));
             uint32_t w[GB / 4];
             quantize_group<BITS>(xp, 0, tb, big, zmask, w);
-            uint8_t *gd = args.codes + idx * PB + gi * GB;
+            uint8_t *gd = args.codes + idx * PB + (2 * half + G) * GB;
             if constexpr (GB == 16) {
               *reinterpret_cast<uint4 *>(gd) = make_uint4(w[0], w[1], w[2], w[3]);
             } else if constexpr (GB == 8) {
