@@ -91,7 +91,8 @@ struct I8Cfg {
   // GP <= 2: the block's scores go through shared memory to one token per
   // lane (see the softmax), kBlk tokens x 2 heads per warp.
   static constexpr bool COMPACT = GP <= 2;
-  static constexpr int ZX_FLOATS = COMPACT ? kI8Warps * kBlk * 2 : 0;
+  // GP = 2: the three query parts' sums of each score go there separately.
+  static constexpr int ZX_FLOATS = COMPACT ? kI8Warps * kBlk * 2 * (GP == 2 ? 3 : 1) : 0;
   static constexpr int SMEM = kI8Warps * RING_BYTES + SCRATCH_FLOATS * 4 + ZX_FLOATS * 4 +
                               2 * kI8Warps * 8 * 4 + kI8Warps * kI8Stages * 8 + 128;
   static constexpr int MIN_BLOCKS = (D == 256 && GP == 8) ? 2 : ((D == 256 && GP == 4) || GP == 8 ? 3 : 4);
@@ -484,6 +485,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     const unsigned char *nk = st + 2 * C::BLK_CODES;                 // float16 [32]
     const unsigned char *nv = st + 2 * C::BLK_CODES + C::BLK_NORMS;
 
+    float *zw = zx + warp * (C::ZX_FLOATS / kI8Warps);   // the warp's score buffer (GP <= 2)
     // ---- QK: exact int32 sums of C * Q_part over the lane's dims, per tile ----
     // sc[T][e]: token 16T + g + 8 (e >> 1), head 2t + (e & 1).
     float sc[2][4];
@@ -558,11 +560,11 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
         sc[T][2] = fmaf(f[0][2], 16384.f, fmaf(f[0][3], 128.f, lo2));
         sc[T][1] = sc[T][3] = 0.f;
       } else if constexpr (GP == 2) {
-        // lane t = 0: hi, t = 1: mid, t = 2: lo of heads 0, 1
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          sc[T][e] = fmaf(f[0][e], 16384.f, fmaf(__shfl_xor_sync(0xffffffffu, f[0][e], 1), 128.f,
-                                                 __shfl_xor_sync(0xffffffffu, f[0][e], 2)));
+        // lane t = 0: hi, t = 1: mid, t = 2: lo of heads 0, 1; each part goes
+        // to its own region of the warp's score buffer (slots as below) and
+        // the lane that takes the token in the softmax weights them.
+        if (t < 3)
+          *reinterpret_cast<float4 *>(zw + 64 * t + 8 * g + 4 * T) = make_float4(f[0][0], f[0][1], f[0][2], f[0][3]);
       } else if constexpr (GP == 4) {
         // tile 0: lanes t = 0, 1 hi, t = 2, 3 mid; tile 1: lanes t = 0, 1 lo
 #pragma unroll
@@ -580,21 +582,35 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     uint32_t u[2][2];
     float dinv[C::NV];
     if constexpr (C::COMPACT) {
-      // One token per lane: the scores (valid in the t = 0 lanes) go through
-      // shared memory so that lane L holds token L's scores of heads 0, 1,
-      // and every softmax step below runs on 2 values per lane instead of 8
-      // (of which 6 belong to padded heads at GP <= 2).  Slot of token
-      // 16 T + 8 hh + g, head h: g 8 + T 4 + hh 2 + h.
-      float *zw = zx + warp * (kBlk * 2);
-      if (t == 0) {
-        *reinterpret_cast<float4 *>(zw + 8 * g) = make_float4(sc[0][0], sc[0][1], sc[0][2], sc[0][3]);
-        *reinterpret_cast<float4 *>(zw + 8 * g + 4) = make_float4(sc[1][0], sc[1][1], sc[1][2], sc[1][3]);
+      // One token per lane: the scores (GP = 1: combined in the t = 0 lanes;
+      // GP = 2: the three parts, stored above) go through shared memory so
+      // that lane L holds token L's scores of heads 0, 1, and every softmax
+      // step below runs on 2 values per lane instead of 8 (of which 6 belong
+      // to padded heads at GP <= 2).  Slot of token 16 T + 8 hh + g, head h:
+      // g 8 + T 4 + hh 2 + h (GP = 2: in the region of each part).
+      if constexpr (GP == 1) {
+        if (t == 0) {
+          *reinterpret_cast<float4 *>(zw + 8 * g) = make_float4(sc[0][0], sc[0][1], sc[0][2], sc[0][3]);
+          *reinterpret_cast<float4 *>(zw + 8 * g + 4) = make_float4(sc[1][0], sc[1][1], sc[1][2], sc[1][3]);
+        }
       }
       __syncwarp();
-      const float2 z = *reinterpret_cast<const float2 *>(zw + 8 * (lane & 7) + 4 * (lane >> 4) + 2 * ((lane >> 3) & 1));
+      const int zs = 8 * (lane & 7) + 4 * (lane >> 4) + 2 * ((lane >> 3) & 1);
+      float z0, z1;
+      if constexpr (GP == 2) {
+        const float2 zh = *reinterpret_cast<const float2 *>(zw + zs);
+        const float2 zm = *reinterpret_cast<const float2 *>(zw + 64 + zs);
+        const float2 zl = *reinterpret_cast<const float2 *>(zw + 128 + zs);
+        z0 = fmaf(zh.x, 16384.f, fmaf(zm.x, 128.f, zl.x));
+        z1 = fmaf(zh.y, 16384.f, fmaf(zm.y, 128.f, zl.y));
+      } else {
+        const float2 z = *reinterpret_cast<const float2 *>(zw + zs);
+        z0 = z.x;
+        z1 = z.y;
+      }
       const float sk = lds_half(nk + 2 * lane);
       float svl = lds_half(nv + 2 * lane);
-      float x0 = z.x * sk * qk0, x1 = z.y * sk * qk1;
+      float x0 = z0 * sk * qk0, x1 = z1 * sk * qk1;
       if (nvalid < kBlk && lane >= nvalid) {   // the chunk's partial last block
         x0 = x1 = -INFINITY;
         svl = 0.f;
@@ -623,12 +639,11 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
       l0 += p0;
       l1 += p1;
       const float pw0 = p0 * svl, pw1 = p1 * svl;
-      float pm0 = pw0, pm1 = pw1;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, o));
-        pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, o));
-      }
+      // Block maxima by one warp reduction each on the bit patterns: as
+      // signed integers they order the non-negative floats as floats do and
+      // put every negative one below them.
+      const float pm0 = __int_as_float(__reduce_max_sync(0xffffffffu, __float_as_int(pw0)));
+      const float pm1 = __int_as_float(__reduce_max_sync(0xffffffffu, __float_as_int(pw1)));
       // W_q = rint(p s^V kWMax / pm) <= kWMax from the low 16 bits of
       // p s^V r + 2^23 (r needs no IEEE division: any r <= kWMax (1 + 2^-22)
       // / pm keeps W_q within 16 bits, and dinv below uses pm itself).

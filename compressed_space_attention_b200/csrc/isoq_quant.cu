@@ -346,11 +346,12 @@ __device__ __forceinline__ void quantize_group(const uint64_t (&xp)[NP], int bas
       if constexpr (NPOS == 3) {
         // Two levels: s2 = [|y| > t_2], then |y| against t_3 if s2 else t_1
         // (the thresholds increase, so m = 2 s2 + [|y| > that threshold]).
-        // The selected threshold s2 t_3 + (1 - s2) t_1 is exact: one of the
-        // two products is zero.
+        // The selected threshold t_1 + s2 (t_3 - t_1) is t_1 exactly or t_3
+        // to within two roundings (a few 1e-8 of it, far inside the band
+        // where the pages' real-valued decision is itself that close).
         const uint64_t s2 = f2_pack(fma_sat(a0, big, tb[1]), fma_sat(a1, big, tb[1]));
-        const uint64_t tsel = f2_fma(s2, f2_pack(tb[2], tb[2]),
-                                     f2_fma(s2, f2_pack(-tb[0], -tb[0]), f2_pack(tb[0], tb[0])));
+        const float d31 = tb[2] - tb[0];
+        const uint64_t tsel = f2_fma(s2, f2_pack(d31, d31), f2_pack(tb[0], tb[0]));
         float t0, t1;
         f2_unpack(tsel, t0, t1);
         const uint64_t s13 = f2_pack(fma_sat(a0, big, t0), fma_sat(a1, big, t1));

@@ -265,14 +265,10 @@ __global__ void __launch_bounds__(kTqThreads, 1)
         const long long t = tile_begin + i;
         const int s = i % kTqStages;
         // The norm from the X tile (row r), while the product runs.
+        // A wait that gives up leaves ok false; the tile is still carried
+        // through (its reads are of this CTA's own memory and its stores go
+        // to this tile's rows), and the loop stops after it.
         bool ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / kTqStages) & 1u);
-        if (__any_sync(0xffffffffu, !ok) || *fail) {
-          if (lane == 0) {
-            *fail = 1u;
-            atomicOr(&g_quant_error, kErrWaitTimeout);
-          }
-          break;
-        }
         const uint32_t xrow = smem_u32(xs + s * kTqXBytes);
         uint64_t ss2 = f2_pack(0.f, 0.f);
 #pragma unroll
@@ -299,14 +295,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
         const float *theirs = xch + (((grp * 2 + (half ^ 1)) * 4 + sub) * 2 + slot) * 32;
         mine[lane] = s_lo + s_hi;
         mbar_arrive(&pbar[2 * warp + slot]);
-        ok = mbar_wait_bounded(&pbar[2 * (warp ^ 4) + slot], static_cast<uint32_t>(k >> 1) & 1u);
-        if (__any_sync(0xffffffffu, !ok) || *fail) {
-          if (lane == 0) {
-            *fail = 1u;
-            atomicOr(&g_quant_error, kErrWaitTimeout);
-          }
-          break;
-        }
+        ok = mbar_wait_bounded(&pbar[2 * (warp ^ 4) + slot], static_cast<uint32_t>(k >> 1) & 1u) && ok;
         const float other = theirs[lane];
         const float ssq = half == 0 ? mine[lane] + other : other + mine[lane];   // ||x||^2, same order in both
         const uint32_t zmask = ssq > 0.f ? 0u : 0x80000000u;
@@ -317,14 +306,7 @@ __global__ void __launch_bounds__(kTqThreads, 1)
         for (int j = 0; j < NPOS; ++j) tb[j] = -(args.tau[j] * S) * big;
         const int b = i % kTqBufs;
         const uint32_t t_row = t_lane + 128 * b;
-        ok = mbar_wait_bounded(&tfull[b], static_cast<uint32_t>(i / kTqBufs) & 1u);
-        if (__any_sync(0xffffffffu, !ok) || *fail) {
-          if (lane == 0) {
-            *fail = 1u;
-            atomicOr(&g_quant_error, kErrWaitTimeout);
-          }
-          break;
-        }
+        ok = mbar_wait_bounded(&tfull[b], static_cast<uint32_t>(i / kTqBufs) & 1u) && ok;
         tc_fence_after();
         const long long v = (t % args.tiles_per_head) * kTqRows + r;
         const bool live = v < args.n_vec;
@@ -367,6 +349,13 @@ __global__ void __launch_bounds__(kTqThreads, 1)
           }
         }
         if (live && half == 0) args.norms[idx] = __half_as_ushort(__float2half_rn(sqrtf(ssq)));
+        if (__any_sync(0xffffffffu, !ok) || *fail) {
+          if (lane == 0) {
+            *fail = 1u;
+            atomicOr(&g_quant_error, kErrWaitTimeout);
+          }
+          break;
+        }
       }
     }
     // Every product of the run has been read back: W may be rebuilt.
