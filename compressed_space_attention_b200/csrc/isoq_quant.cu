@@ -622,6 +622,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
 }
 
 #include "quant_tc.cuh"
+#include "dequant_tc.cuh"
 
 // ---------------------------------------------------------------------------
 // Dequantize
@@ -924,10 +925,77 @@ int launch_quantize(const void *x, int n_heads, long long n_vec, long long head_
   return ISOQ_OK;
 }
 
+template <bool FULL>
+int launch_dequantize_tc(const uint8_t *codes, const uint16_t *norms, int n_heads, long long n_vec,
+                         long long in_head_stride, const float *params, void *out, long long head_stride,
+                         long long vec_stride, cudaStream_t stream) {
+  auto kernel = dequantize_tc_kernel<FULL>;
+  static bool configured = false;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured) {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTdSmem);
+      if (e != cudaSuccess)
+        return set_error(ISOQ_ERR_CUDA, "dequantize (tcgen05): cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      configured = true;
+    }
+  }
+  EncodeTiledFn encode = encode_tiled_fn();
+  if (!encode) return set_error(ISOQ_ERR_CUDA, "dequantize: cuTensorMapEncodeTiled unavailable");
+  CUtensorMap map;
+  const cuuint64_t gdim[3] = {static_cast<cuuint64_t>(kTdD), static_cast<cuuint64_t>(n_vec),
+                              static_cast<cuuint64_t>(n_heads)};
+  const long long hs = n_heads > 1 ? head_stride : vec_stride * n_vec;
+  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(vec_stride * 2), static_cast<cuuint64_t>(hs * 2)};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(kTdRows), 1u};
+  const cuuint32_t estride[3] = {1u, 1u, 1u};
+  const CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, out, gdim, gstride, box, estride,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(ISOQ_ERR_UNSUPPORTED, "dequantize: tensor map encode failed (%d)", (int)r);
+
+  DequantTcArgs a;
+  a.codes = codes;
+  a.norms = norms;
+  a.params = params;
+  a.in_head_stride = in_head_stride;
+  a.n_vec = n_vec;
+  a.tiles_per_head = static_cast<int>((n_vec + kTdRows - 1) / kTdRows);
+  a.total_tiles = static_cast<long long>(a.tiles_per_head) * n_heads;
+  // float16 hi and lo parts of the unit-variance centroids, as byte tables
+  double cu[16];
+  codebook_unit_f64(3, cu);
+  uint8_t tb[4][8];
+  for (int j = 0; j < 8; ++j) {
+    const __half hi = __float2half_rn(static_cast<float>(cu[j]));
+    const __half lo = __float2half_rn(static_cast<float>(cu[j] - static_cast<double>(__half2float(hi))));
+    const uint16_t hb = __half_as_ushort(hi), lb = __half_as_ushort(lo);
+    tb[0][j] = static_cast<uint8_t>(hb & 0xFF);
+    tb[1][j] = static_cast<uint8_t>(hb >> 8);
+    tb[2][j] = static_cast<uint8_t>(lb & 0xFF);
+    tb[3][j] = static_cast<uint8_t>(lb >> 8);
+  }
+  uint32_t *dst[4] = {a.hi_lo, a.hi_hi, a.lo_lo, a.lo_hi};
+  for (int k = 0; k < 4; ++k)
+    for (int w = 0; w < 2; ++w)
+      dst[k][w] = static_cast<uint32_t>(tb[k][4 * w]) | (static_cast<uint32_t>(tb[k][4 * w + 1]) << 8) |
+                  (static_cast<uint32_t>(tb[k][4 * w + 2]) << 16) | (static_cast<uint32_t>(tb[k][4 * w + 3]) << 24);
+  long long grid = num_sms();
+  if (grid > a.total_tiles) grid = a.total_tiles;
+  kernel<<<static_cast<unsigned>(grid), kTdThreads, kTdSmem, stream>>>(map, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(ISOQ_ERR_CUDA, "dequantize (tcgen05) launch: %s", cudaGetErrorString(e));
+  return ISOQ_OK;
+}
+
 template <typename T, int D, int BITS, int RK>
 int launch_dequantize(const uint8_t *codes, const uint16_t *norms, int n_heads, long long n_vec,
                       long long in_head_stride, const float *params, void *out,
                       long long head_stride, long long vec_stride, cudaStream_t stream) {
+  if constexpr (std::is_same<T, __half>::value && D == 128 && BITS == 3 && RK != kRotBlock)
+    return launch_dequantize_tc<RK == kRotWhtFull>(codes, norms, n_heads, n_vec, in_head_stride, params, out,
+                                                   head_stride, vec_stride, stream);
   constexpr int NV = kDequantThreads / Lanes<D>::P;
   auto kernel = dequantize_kernel<T, D, BITS, RK>;
   static int max_ctas_per_sm = -1;
