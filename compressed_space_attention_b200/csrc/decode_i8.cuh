@@ -54,9 +54,11 @@
 //       32-code group g (d = 256) or half of group g/2 (d = 128); M-block mb
 //       maps row g to the lane's quad 2mb and row g+8 to quad 2mb+1.
 //
-// Staging: each warp streams 32-token blocks (packed K and V rows, float16
-// norms) through its own 2-deep ring with CTA-local bulk copies and mbarrier
-// completion, refilling a stage as soon as it has consumed it.
+// Staging: the CTA streams rounds of 128 tokens (warp w takes the round's
+// 32-token block w) through a 2-deep ring of CTA-local bulk copies with
+// mbarrier completion: four copies per round (packed K and V rows, float16
+// norms), issued by the last warp to finish with the stage, so that the
+// copies' operands are computed once per round instead of once per block.
 //
 // Selectors.  A prmt selector is four 3-bit codes in the low nibbles of its
 // low 16 bits.  The 32-code group layout (codes in 4-bit fields, codes
@@ -77,8 +79,13 @@ struct I8Cfg {
   static constexpr int PB = D * 3 / 8;                      // packed bytes per token
   static constexpr int BLK_CODES = kBlk * PB;
   static constexpr int BLK_NORMS = kBlk * 2;
-  static constexpr int STAGE_BYTES = 2 * BLK_CODES + 2 * BLK_NORMS;
-  static constexpr int RING_BYTES = kI8Stages * STAGE_BYTES;
+  static constexpr int STAGE_BYTES = 2 * BLK_CODES + 2 * BLK_NORMS;   // one warp's block
+  static constexpr int RING_BYTES = kI8Stages * STAGE_BYTES;            // per warp
+  // A round stage: K codes, V codes, K norms, V norms of the four warps' blocks.
+  static constexpr int ROUND_BYTES = kI8Warps * STAGE_BYTES;
+  static constexpr int R_V = kI8Warps * BLK_CODES;
+  static constexpr int R_NK = 2 * kI8Warps * BLK_CODES;
+  static constexpr int R_NV = R_NK + kI8Warps * BLK_NORMS;
   static constexpr int KK = D / 32;                         // QK k-steps (8 codes per lane-row each)
   static constexpr int GRP_QK = D / 128;                    // 32-code groups per QK lane segment
   static constexpr int MB = D / 64;                         // PV M-blocks (64 dims each)
@@ -381,12 +388,14 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.group;
 
-  unsigned char *ring = smem + warp * C::RING_BYTES;
+  unsigned char *ring = smem;                       // [stage][round]
   float *scratch = reinterpret_cast<float *>(smem + kI8Warps * C::RING_BYTES);
   float *zx = scratch + C::SCRATCH_FLOATS;          // [warps][kBlk * 2] (GP <= 2)
   float *wm = zx + C::ZX_FLOATS;                    // [warps][8]
   float *wl = wm + kI8Warps * 8;                    // [warps][8]
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(wl + kI8Warps * 8) + warp * kI8Stages;
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(wl + kI8Warps * 8);   // [stage]
+  uint32_t *done_cnt = reinterpret_cast<uint32_t *>(full_bar + kI8Stages);   // [stage]
+  uint32_t *rounds_issued = done_cnt + kI8Stages;
 
   int tlen = a.seq_lens[b];
   tlen = tlen < 0 ? 0 : (tlen > a.tmax ? static_cast<int>(a.tmax) : tlen);
@@ -403,29 +412,33 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
   const uint16_t *nkb = a.norms_k + pair * a.tmax;
   const uint16_t *nvb = a.norms_v + pair * a.tmax;
 
-  // Lane 0 of each warp issues the copies of the warp's i-th block into ring
-  // stage i % kI8Stages.
-  auto issue = [&](int i) {
-    const int j = warp + kI8Warps * i;
-    const long long t = t0 + static_cast<long long>(j) * kBlk;
-    int n = n_tok - j * kBlk;
-    if (n > kBlk) n = kBlk;
+  // One thread issues the copies of round r (tokens 128 r .. 128 r + 127 of
+  // the chunk) into stage r % kI8Stages.
+  const int n_rounds = (n_blk + kI8Warps - 1) / kI8Warps;
+  auto issue = [&](int r) {
+    const long long t = t0 + static_cast<long long>(r) * (kI8Warps * kBlk);
+    int n = n_tok - r * (kI8Warps * kBlk);
+    if (n > kI8Warps * kBlk) n = kI8Warps * kBlk;
     const int n8 = (n + 7) & ~7;
-    const int s = i % kI8Stages;
-    unsigned char *st = ring + s * C::STAGE_BYTES;
+    const int s = r % kI8Stages;
+    unsigned char *st = ring + s * C::ROUND_BYTES;
     mbar_arrive_expect_tx(&full_bar[s], 2u * n * C::PB + 4u * n8);
     bulk_load(st, kb + t * C::PB, n * C::PB, &full_bar[s]);
-    bulk_load(st + C::BLK_CODES, vb + t * C::PB, n * C::PB, &full_bar[s]);
-    bulk_load(st + 2 * C::BLK_CODES, nkb + t, 2 * n8, &full_bar[s]);
-    bulk_load(st + 2 * C::BLK_CODES + C::BLK_NORMS, nvb + t, 2 * n8, &full_bar[s]);
+    bulk_load(st + C::R_V, vb + t * C::PB, n * C::PB, &full_bar[s]);
+    bulk_load(st + C::R_NK, nkb + t, 2 * n8, &full_bar[s]);
+    bulk_load(st + C::R_NV, nvb + t, 2 * n8, &full_bar[s]);
+    *rounds_issued = static_cast<uint32_t>(r + 1);
   };
-  int issued = 0;
-  if (lane == 0) {
-    for (int s = 0; s < kI8Stages; ++s) mbar_init(&full_bar[s], 1);
+  if (tid == 0) {
+    for (int s = 0; s < kI8Stages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      done_cnt[s] = 0u;
+    }
+    *rounds_issued = 0u;
     mbar_fence_init();
-    for (; issued < kI8Stages && issued < n_mine; ++issued) issue(issued);
+    for (int r = 0; r < kI8Stages && r < n_rounds; ++r) issue(r);
   }
-  __syncwarp();   // the other lanes wait on the barriers lane 0 initialised
+  __syncthreads();   // every warp waits on the barriers thread 0 initialised
 
   const int g = lane >> 2, t = lane & 3;
 
@@ -468,7 +481,6 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
   // maximum and sum.
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-  int consumed = 0;
   bool failed = false;
   for (int i = 0; i < n_mine; ++i) {
     const int s = i % kI8Stages;
@@ -479,11 +491,11 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     }
     int nvalid = n_tok - (warp + kI8Warps * i) * kBlk;
     nvalid = nvalid > kBlk ? kBlk : nvalid;
-    const unsigned char *st = ring + s * C::STAGE_BYTES;
-    const unsigned char *kc = st;
-    const unsigned char *vc = st + C::BLK_CODES;
-    const unsigned char *nk = st + 2 * C::BLK_CODES;                 // float16 [32]
-    const unsigned char *nv = st + 2 * C::BLK_CODES + C::BLK_NORMS;
+    const unsigned char *st = ring + s * C::ROUND_BYTES;
+    const unsigned char *kc = st + warp * C::BLK_CODES;
+    const unsigned char *vc = st + C::R_V + warp * C::BLK_CODES;
+    const unsigned char *nk = st + C::R_NK + warp * C::BLK_NORMS;   // float16 [32]
+    const unsigned char *nv = st + C::R_NV + warp * C::BLK_NORMS;
 
     float *zw = zx + warp * (C::ZX_FLOATS / kI8Warps);   // the warp's score buffer (GP <= 2)
     // ---- QK: exact int32 sums of C * Q_part over the lane's dims, per tile ----
@@ -845,18 +857,29 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
       }
     }
     __syncwarp();
-    consumed = i + 1;
-    // The warp is done reading stage s: refill it with the block kI8Stages on.
-    if (lane == 0 && issued < n_mine) {
-      fence_proxy_async_smem();
-      issue(issued);
-      ++issued;
+    // The warp is done reading stage s.  When round i + kI8Stages exists,
+    // round i is full (all four warps read stage s) and the fourth warp to
+    // finish refills it; the counter's acquire-release add orders the other
+    // warps' reads before that copy.
+    if (lane == 0 && kI8Warps * (i + kI8Stages) < n_blk) {
+      uint32_t old;
+      asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                   : "=r"(old)
+                   : "r"(smem_u32(&done_cnt[s]))
+                   : "memory");
+      if ((old & (kI8Warps - 1)) == kI8Warps - 1) {
+        fence_proxy_async_smem();
+        issue(i + kI8Stages);
+      }
     }
   }
-  if (failed && lane == 0) {
-    // Let every copy still in flight land before the CTA may exit.
-    for (int k = consumed; k < issued; ++k)
-      if (!mbar_wait_bounded(&full_bar[k % kI8Stages], (k / kI8Stages) & 1)) break;
+  // Every copy issued lands before the ring is reused or the CTA exits (in
+  // the normal path each was waited for; after a timed-out wait not).
+  __syncthreads();
+  if (tid == 0) {
+    const int ri = static_cast<int>(*rounds_issued);
+    for (int r = ri - kI8Stages < 0 ? 0 : ri - kI8Stages; r < ri; ++r)
+      if (!mbar_wait_bounded(&full_bar[r % kI8Stages], (r / kI8Stages) & 1)) break;
   }
 
   // Per-warp totals over the 8 lanes sharing t (over all 32 lanes with
@@ -867,7 +890,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<D, GP>::MIN_BLOCKS)
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
   if constexpr (SLICES) {
-    __syncthreads();   // every warp is done with its ring, and its copies have landed
+    __syncthreads();   // every warp is done with the ring, and its copies have landed
     // Each warp's accumulators go raw into its own slice [warp][head][dim]
     // (rotated domain) over the ring memory; after one barrier the slices are
     // scaled to the common maximum and summed in warp order (a fixed order).
