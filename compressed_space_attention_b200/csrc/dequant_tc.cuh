@@ -79,8 +79,11 @@ __device__ void build_inverse_operand(const float *params_head, float *rot, unsi
     }
   }
   named_barrier(1, kTdThreads);
+  // Consecutive threads take consecutive rows n of one 8-column chunk, so
+  // that the rotation entries they read (which depend on k only) are
+  // broadcasts and their 16-byte stores fall in distinct banks.
   for (int idx = tid; idx < kTdD * kTdD / 8; idx += kTdThreads) {
-    const int n = idx / (kTdD / 8), k0 = 8 * (idx % (kTdD / 8));
+    const int n = idx % kTdD, k0 = 8 * (idx / kTdD);
     uint32_t hw[4], lw[4];
 #pragma unroll
     for (int j = 0; j < 8; j += 2) {
