@@ -178,6 +178,38 @@ def test_dequantize_parity(d, bits, variant, out_dtype):
     assert np.all(np.abs(got - ref) <= tol), float(np.max(np.abs(got - ref) - tol))
 
 
+@pytest.mark.parametrize("variant", [O.FULL, O.FAST])
+def test_dequantize_tensor_core_strided_heads(variant):
+    """The tensor-core dequantizer (d = 128, 3-bit, float16 out) on five heads
+    of 20,000 vectors whose codes sit in a longer per-head buffer, written into
+    a strided window of a larger output: the values match the oracle, the
+    rows and columns around the window keep their sentinel, and CTAs whose
+    tiles span two heads rebuild the rotation between them."""
+    d, bits, H, n, pad_v, pad_d = 128, 3, 5, 20000, 24, 8
+    params = O.make_params(d, variant, seed=41, n_heads=H)
+    x = synth.unit_vectors(H * n, d, seed=42, dtype=np.float32).reshape(H, n, d)
+    oc, on = O.quantize(x.astype(np.float64), params, bits, variant)
+    ref = O.dequantize(oc, on, params, bits, variant, d)
+    pb = oc.shape[-1]
+    codes_big = torch.zeros((H, n + 20, pb), dtype=torch.uint8, device=DEV)
+    norms_big = torch.zeros((H, n + 20), dtype=torch.float16, device=DEV)
+    codes_big[:, :n] = torch.from_numpy(oc).to(DEV)
+    norms_big[:, :n] = torch.from_numpy(on).to(DEV)
+    sentinel = 3.25
+    out_big = torch.full((H, n + 2 * pad_v, d + pad_d), sentinel, dtype=torch.float16, device=DEV)
+    out = out_big[:, pad_v:pad_v + n, :d]
+    isoq.isoq_dequantize(codes_big[:, :n], norms_big[:, :n], torch.from_numpy(params).to(DEV), d, bits, variant,
+                         out=out, in_head_stride=n + 20)
+    torch.cuda.synchronize()
+    assert isoq.isoq_check_device_error() == 0
+    big = out_big.cpu().numpy()
+    got = big[:, pad_v:pad_v + n, :d].astype(np.float64)
+    tol = DEQ_REL * on.astype(np.float64)[..., None] + f16_half_ulp(ref)
+    assert np.all(np.abs(got - ref) <= tol), float(np.max(np.abs(got - ref) - tol))
+    assert np.all(big[:, :pad_v] == sentinel) and np.all(big[:, pad_v + n:] == sentinel)
+    assert np.all(big[:, :, d:] == sentinel)
+
+
 def test_stage1_round_trip_mse_matches_oracle():
     """GPU quantize then GPU dequantize of unit vectors: the reconstruction
     MSE equals the oracle's (same codes up to boundary flips)."""
