@@ -67,16 +67,24 @@ template <bool FULL>
 __device__ void build_inverse_operand(const float *params_head, float *rot, unsigned char *whi,
                                       unsigned char *wlo, int tid) {   // tid < kTdThreads
   if (tid < kTdD / 4) {
+    // M_i = R_i H_4 (H_4[c][m] = (-1)^popc(c & m)), sums in the order c = 0..3.
+    float R[4][4];
     const Quat ql = load_quat(params_head + 8 * tid);
     const Quat qr = load_quat(params_head + 8 * tid + 4);
     for (int c = 0; c < 4; ++c) {
       const Quat e{c == 0 ? 1.f : 0.f, c == 1 ? 1.f : 0.f, c == 2 ? 1.f : 0.f, c == 3 ? 1.f : 0.f};
       const Quat u = block_forward(ql, qr, e, FULL);   // column c of R_i
-      rot[16 * tid + 4 * 0 + c] = u.w;
-      rot[16 * tid + 4 * 1 + c] = u.x;
-      rot[16 * tid + 4 * 2 + c] = u.y;
-      rot[16 * tid + 4 * 3 + c] = u.z;
+      R[0][c] = u.w;
+      R[1][c] = u.x;
+      R[2][c] = u.y;
+      R[3][c] = u.z;
     }
+    for (int row = 0; row < 4; ++row)
+      for (int m = 0; m < 4; ++m) {
+        float acc = 0.f;
+        for (int c = 0; c < 4; ++c) acc += (__popc(c & m) & 1) ? -R[row][c] : R[row][c];
+        rot[16 * tid + 4 * row + m] = acc;
+      }
   }
   named_barrier(1, kTdThreads);
   // Consecutive threads take consecutive rows n of one 8-column chunk, so
@@ -91,13 +99,10 @@ __device__ void build_inverse_operand(const float *params_head, float *rot, unsi
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
         // W[k][n] = sum_c R_{k/4}[k mod 4][c] H[4 (k/4) + c][n]
+        //         = (-1)^popc((k & ~3) & n) M_{k/4}[k mod 4][n mod 4]
         const int k = k0 + j + jj;
-        const float *rr = rot + 16 * (k >> 2) + 4 * (k & 3);
-        const int j0 = k & ~3;
-        float acc = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc += (__popc((j0 + c) & n) & 1) ? -rr[c] : rr[c];
-        w[jj] = acc;
+        const float m = rot[16 * (k >> 2) + 4 * (k & 3) + (n & 3)];
+        w[jj] = (__popc((k & ~3) & n) & 1) ? -m : m;
       }
       const __half2 h = __floats2half2_rn(w[0], w[1]);
       const float2 hf = __half22float2(h);

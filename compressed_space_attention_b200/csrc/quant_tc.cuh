@@ -57,7 +57,7 @@ constexpr int kTqXBytes = 2 * kTqBlk;           // one X tile (32 KB)
 constexpr int kTqWBytes = kTqD * kTqD * 2;      // W_hi or W_lo (32 KB each)
 constexpr int kTqOffWlo = kTqWBytes;
 constexpr int kTqOffX = 2 * kTqWBytes;
-constexpr int kTqOffRot = kTqOffX + kTqStages * kTqXBytes;    // the head's 4 x 4 blocks, 32 x 16 floats
+constexpr int kTqOffRot = kTqOffX + kTqStages * kTqXBytes;    // the head's 4 x 4 blocks R_i H_4, 32 x 16 floats
 constexpr int kTqOffBar = kTqOffRot + kTqD / 4 * 16 * 4;
 constexpr int kTqBufs = 4;                      // TMEM buffers of 128 columns
 constexpr int kTqOffXch = kTqOffBar;            // partial norms [group][half][sub][slot][lane]
@@ -83,22 +83,34 @@ template <bool FULL>
 __device__ void build_rotation_operand(const float *params_head, float *rot, unsigned char *whi,
                                        unsigned char *wlo, int tid) {   // tid < kTqRunThreads
   if (tid < kTqD / 4) {
+    // M_i = R_i H_4 (H_4[c][m] = (-1)^popc(c & m)), sums in the order c = 0..3.
+    float R[4][4];
     const Quat ql = load_quat(params_head + 8 * tid);
     const Quat qr = load_quat(params_head + 8 * tid + 4);
     for (int c = 0; c < 4; ++c) {
       const Quat e{c == 0 ? 1.f : 0.f, c == 1 ? 1.f : 0.f, c == 2 ? 1.f : 0.f, c == 3 ? 1.f : 0.f};
       const Quat u = block_forward(ql, qr, e, FULL);   // column c of R_i
-      rot[16 * tid + 4 * 0 + c] = u.w;
-      rot[16 * tid + 4 * 1 + c] = u.x;
-      rot[16 * tid + 4 * 2 + c] = u.y;
-      rot[16 * tid + 4 * 3 + c] = u.z;
+      R[0][c] = u.w;
+      R[1][c] = u.x;
+      R[2][c] = u.y;
+      R[3][c] = u.z;
     }
+    for (int row = 0; row < 4; ++row)
+      for (int m = 0; m < 4; ++m) {
+        float acc = 0.f;
+        for (int c = 0; c < 4; ++c) acc += (__popc(c & m) & 1) ? -R[row][c] : R[row][c];
+        rot[16 * tid + 4 * row + m] = acc;
+      }
   }
   named_barrier(1, kTqRunThreads);
+  // W[n][k] = sum_c R_{n/4}[n mod 4][c] H[4 (n/4) + c][k]
+  //         = (-1)^popc((n & ~3) & k) M_{n/4}[n mod 4][k mod 4]: the rows 4 (n/4) + c
+  // and the column k share no bits outside c's, so the sign splits off
+  // (the same four products, summed in the same order, with one sign).
   for (int idx = tid; idx < kTqD * kTqD / 8; idx += kTqRunThreads) {
     const int n = idx / (kTqD / 8), k0 = 8 * (idx % (kTqD / 8));
-    const float *rr = rot + 16 * (n >> 2) + 4 * (n & 3);
-    const int j0 = n & ~3;
+    const float *mm = rot + 16 * (n >> 2) + 4 * (n & 3);
+    const int n4 = n & ~3;
     uint32_t hw[4], lw[4];
 #pragma unroll
     for (int j = 0; j < 8; j += 2) {
@@ -106,10 +118,7 @@ __device__ void build_rotation_operand(const float *params_head, float *rot, uns
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
         const int k = k0 + j + jj;
-        float acc = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc += (__popc((j0 + c) & k) & 1) ? -rr[c] : rr[c];
-        w[jj] = acc;
+        w[jj] = (__popc(n4 & k) & 1) ? -mm[k & 3] : mm[k & 3];
       }
       const __half2 h = __floats2half2_rn(w[0], w[1]);
       const float2 hf = __half22float2(h);
