@@ -1,5 +1,5 @@
-// Dequantizer for d = 128, 3-bit codes, float16 output, with the whole
-// inverse rotation on the 5th-generation tensor cores (tcgen05 + TMEM).
+// Dequantizer for d = 128, 2- and 3-bit codes, float16 output, with the
+// whole inverse rotation on the 5th-generation tensor cores (tcgen05 + TMEM).
 // Included by isoq_quant.cu inside namespace isoq::quant, after quant_tc.cuh
 // (build_rotation_operand's pieces, tc_ld32_nowait).
 //
@@ -16,9 +16,11 @@
 // The codes become the A operand on the CUDA cores: each pair of threads
 // takes one vector (row), each thread 64 dims (two 32-code groups); one prmt
 // per four codes and byte table (the low and high bytes of the float16 hi and
-// lo parts of the 8 centroids, 8-entry tables) and two more that interleave
-// the bytes give the float16 pairs, which go to the thread's TMEM lane with
-// tcgen05.st.  After the product the same threads read their 64 output
+// lo parts of the 8 or 4 centroids) and two more that interleave the bytes
+// give the float16 pairs, which go to the thread's TMEM lane with
+// tcgen05.st.  The selectors are the codes in 4-bit fields: the 3-bit layout
+// has them there already (plus the spare-bit codes), the 2-bit bitstream is
+// spread into them.  After the product the same threads read their 64 output
 // columns back, scale by ||x|| / 128, round to float16 and write them into a
 // 128B-swizzled tile in shared memory that one thread stores with TMA.
 //
@@ -133,6 +135,29 @@ __device__ __forceinline__ void dq_group_sel8(uint32_t w0, uint32_t w1, uint32_t
   s[7] = sum >> 16;
 }
 
+// The same for one 32-code 2-bit group (two words of the LSB-first
+// bitstream: code j of a word at bits 2 j .. 2 j + 1), spread to 4-bit
+// fields.
+__device__ __forceinline__ uint32_t dq_spread2(uint32_t x) {   // 8 codes in bits 0..15 -> 8 nibbles
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  x = (x | (x << 2)) & 0x33333333u;
+  return x;
+}
+
+__device__ __forceinline__ void dq_group_sel8_b2(uint32_t w0, uint32_t w1, uint32_t (&s)[8]) {
+  const uint32_t a = dq_spread2(w0 & 0xFFFFu), b = dq_spread2(w0 >> 16);
+  const uint32_t c = dq_spread2(w1 & 0xFFFFu), d = dq_spread2(w1 >> 16);
+  s[0] = a;
+  s[1] = a >> 16;
+  s[2] = b;
+  s[3] = b >> 16;
+  s[4] = c;
+  s[5] = c >> 16;
+  s[6] = d;
+  s[7] = d >> 16;
+}
+
 // Named barrier that also ORs a predicate over its threads (every thread
 // gets the same answer, so a group of warps can stop together).
 __device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool p) {
@@ -152,10 +177,12 @@ __device__ __forceinline__ uint32_t dq_prmt(uint32_t a, uint32_t b, uint32_t sel
   return r;
 }
 
-template <bool FULL>
+template <int BITS, bool FULL>
 __global__ void __launch_bounds__(kTdThreads, 1)
     dequantize_tc_kernel(const __grid_constant__ CUtensorMap omap, const DequantTcArgs args) {
-  constexpr int PB = kTdD * 3 / 8;   // 48 bytes per vector
+  static_assert(BITS == 2 || BITS == 3, "2- or 3-bit codes");
+  constexpr int PB = kTdD * BITS / 8;   // 32 or 48 bytes per vector
+  constexpr int TB = PB / 2;            // bytes of one thread's two groups
   extern __shared__ unsigned char smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char *smem = smem_raw + pad;
@@ -202,21 +229,34 @@ __global__ void __launch_bounds__(kTdThreads, 1)
   unsigned char *out_s = otile + (2 * grp + half) * kTdBlk;
   const bool issuer = (warp & 7) == 0 && lane == 0;   // stores the group's output tiles
 
-  // The codes (24 bytes: groups 2 half, 2 half + 1) and the norm of this
+  // The codes (TB bytes: groups 2 half, 2 half + 1) and the norm of this
   // thread's vector in local tile i.
-  auto load_vec = [&](int i, uint2 (&c)[3], uint32_t &nrm) {
+  auto load_vec = [&](int i, uint32_t (&c)[6], uint32_t &nrm) {
     const long long t = tile_begin + i;
     const int head = static_cast<int>(t / args.tiles_per_head);
     const long long v = (t % args.tiles_per_head) * kTdRows + r;
     if (i < n_mine && v < args.n_vec) {
       const long long idx = static_cast<long long>(head) * args.in_head_stride + v;
-      const uint2 *src = reinterpret_cast<const uint2 *>(args.codes + idx * PB + 24 * half);
-      c[0] = src[0];
-      c[1] = src[1];
-      c[2] = src[2];
+      if constexpr (BITS == 3) {
+        const uint2 *src = reinterpret_cast<const uint2 *>(args.codes + idx * PB + TB * half);
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const uint2 u = src[k];
+          c[2 * k] = u.x;
+          c[2 * k + 1] = u.y;
+        }
+      } else {
+        const uint4 u = *reinterpret_cast<const uint4 *>(args.codes + idx * PB + TB * half);
+        c[0] = u.x;
+        c[1] = u.y;
+        c[2] = u.z;
+        c[3] = u.w;
+        c[4] = c[5] = 0u;
+      }
       nrm = args.norms[idx];
     } else {
-      c[0] = c[1] = c[2] = make_uint2(0u, 0u);
+#pragma unroll
+      for (int k = 0; k < 6; ++k) c[k] = 0u;
       nrm = 0u;
     }
   };
@@ -267,14 +307,16 @@ __global__ void __launch_bounds__(kTdThreads, 1)
     } else {
       // ---- workers: tiles of parity grp ----
       const int i0 = i_seg + ((i_seg & 1) != grp ? 1 : 0);
-      uint2 cw[3];
+      uint32_t cw[6];
       uint32_t nw = 0u;
       load_vec(i0, cw, nw);
       for (int i = i0; i < seg_end; i += 2) {
         const int k = i >> 1;
         const long long t = tile_begin + i;
         const int v0 = static_cast<int>((t % args.tiles_per_head) * kTdRows);
-        uint2 c[3] = {cw[0], cw[1], cw[2]};
+        uint32_t c[6];
+#pragma unroll
+        for (int k = 0; k < 6; ++k) c[k] = cw[k];
         const uint32_t nrm = nw;
         if (i + 2 < seg_end) load_vec(i + 2, cw, nw);   // the group's next tile, in flight meanwhile
 
@@ -283,7 +325,10 @@ __global__ void __launch_bounds__(kTdThreads, 1)
 #pragma unroll
         for (int G = 0; G < 2; ++G) {
           uint32_t s[8];
-          dq_group_sel8(G == 0 ? c[0].x : c[1].y, G == 0 ? c[0].y : c[2].x, G == 0 ? c[1].x : c[2].y, s);
+          if constexpr (BITS == 3)
+            dq_group_sel8(c[3 * G], c[3 * G + 1], c[3 * G + 2], s);
+          else
+            dq_group_sel8_b2(c[2 * G], c[2 * G + 1], s);
           uint32_t hw[16], lw[16];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {

@@ -925,11 +925,11 @@ int launch_quantize(const void *x, int n_heads, long long n_vec, long long head_
   return ISOQ_OK;
 }
 
-template <bool FULL>
+template <int BITS, bool FULL>
 int launch_dequantize_tc(const uint8_t *codes, const uint16_t *norms, int n_heads, long long n_vec,
                          long long in_head_stride, const float *params, void *out, long long head_stride,
                          long long vec_stride, cudaStream_t stream) {
-  auto kernel = dequantize_tc_kernel<FULL>;
+  auto kernel = dequantize_tc_kernel<BITS, FULL>;
   static bool configured = false;
   static std::mutex mu;
   {
@@ -965,9 +965,9 @@ int launch_dequantize_tc(const uint8_t *codes, const uint16_t *norms, int n_head
   a.total_tiles = static_cast<long long>(a.tiles_per_head) * n_heads;
   // float16 hi and lo parts of the unit-variance centroids, as byte tables
   double cu[16];
-  codebook_unit_f64(3, cu);
-  uint8_t tb[4][8];
-  for (int j = 0; j < 8; ++j) {
+  codebook_unit_f64(BITS, cu);
+  uint8_t tb[4][8] = {};
+  for (int j = 0; j < (1 << BITS); ++j) {
     const __half hi = __float2half_rn(static_cast<float>(cu[j]));
     const __half lo = __float2half_rn(static_cast<float>(cu[j] - static_cast<double>(__half2float(hi))));
     const uint16_t hb = __half_as_ushort(hi), lb = __half_as_ushort(lo);
@@ -993,9 +993,9 @@ template <typename T, int D, int BITS, int RK>
 int launch_dequantize(const uint8_t *codes, const uint16_t *norms, int n_heads, long long n_vec,
                       long long in_head_stride, const float *params, void *out,
                       long long head_stride, long long vec_stride, cudaStream_t stream) {
-  if constexpr (std::is_same<T, __half>::value && D == 128 && BITS == 3 && RK != kRotBlock)
-    return launch_dequantize_tc<RK == kRotWhtFull>(codes, norms, n_heads, n_vec, in_head_stride, params, out,
-                                                   head_stride, vec_stride, stream);
+  if constexpr (std::is_same<T, __half>::value && D == 128 && (BITS == 2 || BITS == 3) && RK != kRotBlock)
+    return launch_dequantize_tc<BITS, RK == kRotWhtFull>(codes, norms, n_heads, n_vec, in_head_stride, params,
+                                                         out, head_stride, vec_stride, stream);
   constexpr int NV = kDequantThreads / Lanes<D>::P;
   auto kernel = dequantize_kernel<T, D, BITS, RK>;
   static int max_ctas_per_sm = -1;

@@ -178,14 +178,15 @@ def test_dequantize_parity(d, bits, variant, out_dtype):
     assert np.all(np.abs(got - ref) <= tol), float(np.max(np.abs(got - ref) - tol))
 
 
+@pytest.mark.parametrize("bits", [2, 3])
 @pytest.mark.parametrize("variant", [O.FULL, O.FAST])
-def test_dequantize_tensor_core_strided_heads(variant):
-    """The tensor-core dequantizer (d = 128, 3-bit, float16 out) on five heads
+def test_dequantize_tensor_core_strided_heads(variant, bits):
+    """The tensor-core dequantizer (d = 128, 2 and 3 bits, float16 out) on five heads
     of 20,000 vectors whose codes sit in a longer per-head buffer, written into
     a strided window of a larger output: the values match the oracle, the
     rows and columns around the window keep their sentinel, and CTAs whose
     tiles span two heads rebuild the rotation between them."""
-    d, bits, H, n, pad_v, pad_d = 128, 3, 5, 20000, 24, 8
+    d, H, n, pad_v, pad_d = 128, 5, 20000, 24, 8
     params = O.make_params(d, variant, seed=41, n_heads=H)
     x = synth.unit_vectors(H * n, d, seed=42, dtype=np.float32).reshape(H, n, d)
     oc, on = O.quantize(x.astype(np.float64), params, bits, variant)
