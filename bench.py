@@ -1127,7 +1127,8 @@ def run_isoq(args):
                      "frac": q_bytes * args.steps / (t_quant * 1e-3) / 1e9 / hbm,
                      "workload": "2^20 float16 unit vectors, d=128, 3-bit, Full"},
         "dequantize": {"value": n_ranks * n1 * args.steps / (t_deq * 1e-3) / 1e6, "unit": "Mvec/s",
-                       "gbps": dq_bytes * args.steps / (t_deq * 1e-3) / 1e9},
+                       "gbps": dq_bytes * args.steps / (t_deq * 1e-3) / 1e9,
+                       "frac": dq_bytes * args.steps / (t_deq * 1e-3) / 1e9 / hbm},
         "step_ms": {"quantize": t_quant / args.steps, "dequantize": t_deq / args.steps,
                     "decode_split": t_split / args.steps, "decode_combine": t_comb / args.steps},
         "e2e": {"value": (n_ranks * kv_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9) if e2e_steps else None, "unit": "GB/s",
