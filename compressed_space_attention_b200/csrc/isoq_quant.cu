@@ -42,6 +42,11 @@
 // Data movement.  Each warp of a quantize CTA streams its own rows through a
 // ring of 128B-swizzled TMA tiles (no producer warp); each lane reads its own
 // 128-byte row segments conflict-free.  Each lane writes whole 32-code groups.
+//
+// The kernels above serve every shape; for d = 128 with the WHT, float16
+// input (quantize) or float16 output with 2- or 3-bit codes (dequantize), the
+// launchers take the tensor-core forms instead (quant_tc.cuh, dequant_tc.cuh),
+// where the whole rotation is one tcgen05 product per 128-vector tile.
 
 #include <cuda.h>
 #include <cuda_fp16.h>
